@@ -1,0 +1,318 @@
+"""CPU oracle for the weight-only quantized matmul (test infrastructure only).
+
+Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never does; it
+shares no code with this oracle (see ``qmm_oracle.c`` for the definitions and
+the pages each one follows).
+
+This module compiles ``qmm_oracle.c`` with gcc (``-O2 -ffp-contract=off``)
+into ``liboracle.so`` next to it and wraps it with ctypes, taking and
+returning numpy arrays.  Large calls are split over output rows and run on a
+thread pool: ctypes drops the GIL during the foreign call, so the C code runs
+in parallel while each thread stays plain single-threaded C.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qmm_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, F16, BF16 = 0, 1, 2
+_NP_STORAGE = {F32: np.float32, F16: np.uint16, BF16: np.uint16}
+ORC_OK, ORC_ERR_ARG, ORC_ERR_ID = 0, 1, 7
+
+_lock = threading.Lock()
+_lib = None
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile the oracle shared library (idempotent); returns its path."""
+    with _lock:
+        fresh = os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)
+        if force or not fresh:
+            tmp = _LIB + f".tmp{os.getpid()}"
+            cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+                   "-shared", "-o", tmp, _SRC, "-lm"]
+            subprocess.run(cmd, check=True)
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Stack(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("biases", ctypes.c_void_p), ("s_dtype", ctypes.c_int),
+                ("num_experts", ctypes.c_int64), ("n_rows", ctypes.c_int64),
+                ("n_cols", ctypes.c_int64), ("gs", ctypes.c_int), ("bits", ctypes.c_int)]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build_oracle())
+        vp, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
+        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_bf16_to_f32.restype = ctypes.c_float
+        L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+        L.orc_f16_to_f32.restype = ctypes.c_float
+        L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+        L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_f32_to_f16.argtypes = [ctypes.c_float]
+        L.orc_f32_to_f16.restype = ctypes.c_uint16
+        L.orc_words_per_row.argtypes = [i64, c_int]
+        L.orc_words_per_row.restype = i64
+        L.orc_pack_row.argtypes = [vp, i64, c_int, vp]
+        L.orc_pack_row.restype = None
+        L.orc_code_integral.argtypes = [vp, c_int, i64]
+        L.orc_code_integral.restype = ctypes.c_uint32
+        L.orc_code_u64.argtypes = [vp, i64, c_int, i64]
+        L.orc_code_u64.restype = ctypes.c_uint32
+        L.orc_quantize.argtypes = [vp, c_int, i64, i64, c_int, c_int, c_int, vp, vp, vp, i64, i64]
+        L.orc_dequantize.argtypes = [vp, vp, vp, c_int, i64, i64, c_int, c_int, vp, c_int, i64, i64]
+        L.orc_matmul.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int, c_int, c_int,
+                                 vp, i64, i64]
+        L.orc_matmul_element.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int,
+                                         c_int, c_int, i64, i64]
+        L.orc_matmul_element.restype = ctypes.c_double
+        sp = ctypes.POINTER(_Stack)
+        L.orc_moe_gemv_id.argtypes = [vp, c_int, vp, i64, i64, sp, vp, i64, i64]
+        L.orc_moe_gemv_id_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, vp, i64, i64]
+        L.orc_moe_gate_up_silu.argtypes = [vp, c_int, vp, i64, sp, sp, vp, i64, i64]
+        L.orc_moe_gate_up_silu_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, sp, vp,
+                                                   i64, i64]
+        _ = (i32,)
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data
+
+
+def _threads(n_threads):
+    if n_threads is None:
+        try:
+            n_threads = len(os.sched_getaffinity(0))
+        except AttributeError:
+            n_threads = os.cpu_count() or 1
+    return max(1, int(n_threads))
+
+
+def _split(lo, hi, parts):
+    n = hi - lo
+    if n <= 0:
+        return []
+    parts = max(1, min(parts, n))
+    step = (n + parts - 1) // parts
+    return [(a, min(a + step, hi)) for a in range(lo, hi, step)]
+
+
+def _run(fn, lo, hi, n_threads):
+    chunks = _split(lo, hi, _threads(n_threads) * 2)
+    if len(chunks) <= 1:
+        rcs = [fn(a, b) for a, b in chunks]
+    else:
+        with ThreadPoolExecutor(max_workers=_threads(n_threads)) as ex:
+            rcs = list(ex.map(lambda ab: fn(*ab), chunks))
+    return max(rcs) if rcs else ORC_OK
+
+
+def dtype_code(storage: str) -> int:
+    return {"f32": F32, "f16": F16, "bf16": BF16}[storage]
+
+
+# ---------------------------------------------------------------- conversions
+def bf16_to_f32(h: int) -> float:
+    return float(lib().orc_bf16_to_f32(int(h)))
+
+
+def f16_to_f32(h: int) -> float:
+    return float(lib().orc_f16_to_f32(int(h)))
+
+
+def f32_to_bf16(v: float) -> int:
+    return int(lib().orc_f32_to_bf16(float(v)))
+
+
+def f32_to_f16(v: float) -> int:
+    return int(lib().orc_f32_to_f16(float(v)))
+
+
+def words_per_row(cols: int, bits: int) -> int:
+    return int(lib().orc_words_per_row(cols, bits))
+
+
+# ---------------------------------------------------------------- packing
+def pack_row(codes: np.ndarray, bits: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    words = np.zeros(words_per_row(codes.size, bits), dtype=np.uint32)
+    lib().orc_pack_row(_ptr(codes), codes.size, bits, _ptr(words))
+    return words
+
+
+def code_integral(row: np.ndarray, bits: int, i: int) -> int:
+    row = np.ascontiguousarray(row, dtype=np.uint32)
+    return int(lib().orc_code_integral(_ptr(row), bits, i))
+
+
+def code_u64(row: np.ndarray, bits: int, i: int) -> int:
+    row = np.ascontiguousarray(row, dtype=np.uint32)
+    return int(lib().orc_code_u64(_ptr(row), row.size, bits, i))
+
+
+# ---------------------------------------------------------------- quantize / dequantize
+def quantize(w: np.ndarray, w_dtype: int, group_size: int, bits: int, s_dtype: int,
+             n_threads=None):
+    """w: [rows, cols] array in its storage form (float32, or uint16 bits for f16/bf16).
+    Returns (packed u32 [rows, cols*bits/32], scales, biases [rows, cols/gs]) in storage form."""
+    w = np.ascontiguousarray(w)
+    rows, cols = w.shape
+    packed = np.zeros((rows, cols * bits // 32), dtype=np.uint32)
+    G = cols // group_size
+    scales = np.zeros((rows, G), dtype=_NP_STORAGE[s_dtype])
+    biases = np.zeros((rows, G), dtype=_NP_STORAGE[s_dtype])
+    L = lib()
+
+    def fn(a, b):
+        return L.orc_quantize(_ptr(w), w_dtype, rows, cols, group_size, bits, s_dtype,
+                              _ptr(packed), _ptr(scales), _ptr(biases), a, b)
+    rc = _run(fn, 0, rows, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle quantize rejected the arguments (rc={rc})")
+    return packed, scales, biases
+
+
+def dequantize(packed, scales, biases, s_dtype: int, cols: int, group_size: int, bits: int,
+               out_dtype: int, n_threads=None) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+    rows = packed.shape[0]
+    out = np.zeros((rows, cols), dtype=_NP_STORAGE[out_dtype])
+    L = lib()
+
+    def fn(a, b):
+        return L.orc_dequantize(_ptr(packed), _ptr(scales), _ptr(biases), s_dtype, rows, cols,
+                                group_size, bits, _ptr(out), out_dtype, a, b)
+    rc = _run(fn, 0, rows, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle dequantize rejected the arguments (rc={rc})")
+    return out
+
+
+# ---------------------------------------------------------------- matmul
+def matmul(x, x_dtype: int, packed, scales, biases, s_dtype: int, N: int, group_size: int,
+           bits: int, transpose: bool = True, n_threads=None) -> np.ndarray:
+    """fp64 y[M, N] = x . dequant(W)^T (transpose) or x . dequant(W)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    y = np.zeros((M, N), dtype=np.float64)
+    L = lib()
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+
+    def fn(a, b):
+        return L.orc_matmul(_ptr(x), x_dtype, M, K, _ptr(packed), _ptr(scales), _ptr(biases),
+                            s_dtype, N, group_size, bits, int(bool(transpose)), _ptr(y), a, b)
+    rc = _run(fn, 0, N, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle matmul rejected the arguments (rc={rc})")
+    return y
+
+
+def matmul_elements(x, x_dtype: int, packed, scales, biases, s_dtype: int, N: int,
+                    group_size: int, bits: int, coords, transpose: bool = True,
+                    n_threads=None) -> np.ndarray:
+    """fp64 y[m, n] for each (m, n) in coords (sampled checks at full size)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+    coords = list(coords)
+    out = np.zeros(len(coords), dtype=np.float64)
+    L = lib()
+
+    def fn(a, b):
+        for i in range(a, b):
+            m, n = coords[i]
+            out[i] = L.orc_matmul_element(_ptr(x), x_dtype, M, K, _ptr(packed), _ptr(scales),
+                                          _ptr(biases), s_dtype, N, group_size, bits,
+                                          int(bool(transpose)), int(m), int(n))
+        return ORC_OK
+    _run(fn, 0, len(coords), n_threads)
+    return out
+
+
+# ---------------------------------------------------------------- MoE
+class Stack:
+    """Host-side expert stack: packed [E*n_rows, n_cols*bits/32] u32, scales and
+    biases [E*n_rows, n_cols/gs] in storage form."""
+
+    def __init__(self, packed, scales, biases, s_dtype, num_experts, n_rows, n_cols, group_size,
+                 bits):
+        self.packed = np.ascontiguousarray(packed, dtype=np.uint32)
+        self.scales = np.ascontiguousarray(scales)
+        self.biases = np.ascontiguousarray(biases)
+        self.c = _Stack(self.packed.ctypes.data, self.scales.ctypes.data,
+                        self.biases.ctypes.data, s_dtype, num_experts, n_rows, n_cols,
+                        group_size, bits)
+        self.n_rows = n_rows
+        self.n_cols = n_cols
+
+
+def moe_gemv_id(a, a_dtype, ids, n_selected, src1_stride, st: Stack, n_threads=None):
+    a = np.ascontiguousarray(a)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    out = np.zeros((n_selected, st.n_rows), dtype=np.float64)
+    L = lib()
+
+    def fn(lo, hi):
+        return L.orc_moe_gemv_id(_ptr(a), a_dtype, _ptr(ids), n_selected, src1_stride,
+                                 ctypes.byref(st.c), _ptr(out), lo, hi)
+    rc = _run(fn, 0, n_selected, n_threads)
+    return out, rc
+
+
+def moe_gemv_id_batched(a, a_dtype, ids, m, top_k, outer, inner, st: Stack, n_threads=None):
+    a = np.ascontiguousarray(a)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    out = np.zeros((m * top_k, st.n_rows), dtype=np.float64)
+    L = lib()
+
+    def fn(lo, hi):
+        return L.orc_moe_gemv_id_batched(_ptr(a), a_dtype, _ptr(ids), m, top_k, outer, inner,
+                                         ctypes.byref(st.c), _ptr(out), lo, hi)
+    rc = _run(fn, 0, m * top_k, n_threads)
+    return out, rc
+
+
+def moe_gate_up_silu(a, a_dtype, ids, n_selected, gate: Stack, up: Stack, n_threads=None):
+    a = np.ascontiguousarray(a)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    out = np.zeros((n_selected, gate.n_rows), dtype=np.float64)
+    L = lib()
+
+    def fn(lo, hi):
+        return L.orc_moe_gate_up_silu(_ptr(a), a_dtype, _ptr(ids), n_selected,
+                                      ctypes.byref(gate.c), ctypes.byref(up.c), _ptr(out), lo, hi)
+    rc = _run(fn, 0, n_selected, n_threads)
+    return out, rc
+
+
+def moe_gate_up_silu_batched(a, a_dtype, ids, m, top_k, outer, inner, gate: Stack, up: Stack,
+                             n_threads=None):
+    a = np.ascontiguousarray(a)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    out = np.zeros((m * top_k, gate.n_rows), dtype=np.float64)
+    L = lib()
+
+    def fn(lo, hi):
+        return L.orc_moe_gate_up_silu_batched(_ptr(a), a_dtype, _ptr(ids), m, top_k, outer,
+                                              inner, ctypes.byref(gate.c), ctypes.byref(up.c),
+                                              _ptr(out), lo, hi)
+    rc = _run(fn, 0, m * top_k, n_threads)
+    return out, rc
