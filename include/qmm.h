@@ -1,0 +1,187 @@
+/*
+ * qmm.h -- C ABI of libqmm.so: weight-only quantized matmul on NVIDIA B200
+ * (sm_100a), affine mode.
+ *
+ * What is computed (sources cited by page title and section):
+ *   - Packed weights: b-bit codes (b in {2,3,4,6,8}) stored LSB-first along
+ *     the row in little-endian uint32 words; code i of a row sits at stream
+ *     bits [i*b, (i+1)*b) and may straddle two words when b is 3 or 6
+ *     ("emily 0.5.1 lib/emily/quantization.ex", dequantize_defn/1,
+ *     unpack_integral_lanes, unpack_cross_word_lanes).
+ *   - Affine dequantization: w_hat[r][i] = q * scale[r][g] + bias[r][g],
+ *     g = i / group_size (same page, dequantize_defn/1 doc).  This library
+ *     evaluates it as one fp32 fused multiply-add.
+ *   - Quantized matmul: y = x . dequant(W)^T for transpose = 1, the AWQ
+ *     layout y = x . dequant(W) for transpose = 0 (same page,
+ *     quantized_matmul/2); affine mode requires x and the scales to share a
+ *     dtype (same page, validate_dtype_match!).
+ *   - MoE stacked experts: out[i] = a[off(i)] . dequant(W[ids[i]])^T and the
+ *     fused SiLU(gate) * up form, single and batched
+ *     ("ferrum-kernels 0.7.7 src/stacked_expert.rs", StackedExpertGgufLinear:
+ *     gemv_moe_id, gemv_moe_id_batched, gemv_moe_id_gate_up_silu,
+ *     gemv_moe_id_gate_up_silu_batched).  The offset-aware form
+ *     (gemv_moe_id_offset) is the same call with `a` and `ids` advanced by
+ *     the caller.
+ *   - Quantizer: per (row, group) min/max; the page that calls it
+ *     ("ollama x/create/client/quantize.go", loadAndQuantizeArray) does not
+ *     print its body, so this library uses the min/max rule of
+ *     "mlex 0.1.3 src/quant.rs" quantize_dynamic_int8 applied per group:
+ *     scale = max((max-min)/(2^b-1), FLT_EPSILON), bias = min,
+ *     q = clamp(round_half_away((w - bias)/scale), 0, 2^b-1), with scale and
+ *     bias first rounded to the scales dtype.
+ *
+ * Conventions for every call:
+ *   - All buffer pointers are DEVICE pointers owned by the caller; the
+ *     library keeps no allocation across calls and allocates nothing.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronizes the host.
+ *   - Host-side argument errors are returned before anything is launched.
+ *     Errors found on the device (a bad expert id) are OR-ed into *d_status
+ *     (a caller-zeroed device int32, may be NULL), read by the caller after
+ *     the stream has synchronized.  The library never aborts.
+ *   - Shapes: group_size in {32, 64, 128}; cols % group_size == 0 and
+ *     cols * bits % 32 == 0 for the quantized axis.
+ *   - Alignment: packed, scales, biases, x, y and out must be 16-byte
+ *     aligned (QMM_ERR_ALIGNMENT otherwise); MoE activation rows `a + off`
+ *     only need element alignment.
+ *   - Requires a compute-capability 10.0 device (QMM_ERR_UNSUPPORTED
+ *     otherwise).
+ */
+#ifndef QMM_H_
+#define QMM_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QMM_OK = 0,
+  QMM_ERR_INVALID_ARG = 1,   /* bad bits/group_size/shape/mode/flag */
+  QMM_ERR_UNSUPPORTED = 2,   /* non-affine mode, unsupported device or size */
+  QMM_ERR_DTYPE = 3,         /* dtype rule violated (x vs scales, out dtype) */
+  QMM_ERR_ALIGNMENT = 4,     /* null or under-aligned pointer */
+  QMM_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+  QMM_ERR_TIMEOUT = 6,       /* a bounded device-side wait gave up */
+  QMM_ERR_BAD_EXPERT_ID = 7  /* (device) an id outside [0, num_experts) */
+} qmm_status;
+
+typedef enum { QMM_F32 = 0, QMM_F16 = 1, QMM_BF16 = 2 } qmm_dtype;
+
+/* Only affine is implemented; the microscaled modes named on the emily page
+ * (mxfp4, mxfp8, nvfp4) are rejected with QMM_ERR_UNSUPPORTED. */
+typedef enum {
+  QMM_MODE_AFFINE = 0,
+  QMM_MODE_MXFP4 = 1,
+  QMM_MODE_MXFP8 = 2,
+  QMM_MODE_NVFP4 = 3
+} qmm_mode;
+
+/* A quantized matrix ("emily" %QuantizedWeight{value, scales, biases,
+ * group_size, bits, mode}).  packed: [rows, cols*bits/32] uint32 row-major;
+ * scales, biases: [rows, cols/group_size] row-major in `sdtype`.  The
+ * quantized axis is `cols`. */
+typedef struct {
+  const uint32_t* packed;
+  const void* scales;
+  const void* biases;
+  qmm_dtype sdtype;
+  int64_t rows;
+  int64_t cols;
+  int group_size;
+  int bits;
+  qmm_mode mode;
+} qmm_qweight;
+
+/* N experts of one role (gate, up or down) stored contiguously ("ferrum"
+ * StackedExpertGgufLinear): expert e is rows [e*n_rows, (e+1)*n_rows) of
+ * packed [num_experts*n_rows, n_cols*bits/32] and of scales/biases
+ * [num_experts*n_rows, n_cols/group_size]. */
+typedef struct {
+  const uint32_t* packed;
+  const void* scales;
+  const void* biases;
+  qmm_dtype sdtype;
+  int64_t num_experts;
+  int64_t n_rows;
+  int64_t n_cols;
+  int group_size;
+  int bits;
+} qmm_expert_stack;
+
+/* cols*bits/32, or -1 when (cols, bits) cannot be packed without a partial
+ * word (bits not in {2,3,4,6,8}, cols <= 0, or cols*bits % 32 != 0). */
+int64_t qmm_packed_words_per_row(int64_t cols, int bits);
+
+/* cols/group_size, or -1 (group_size not in {32,64,128}, cols % gs != 0). */
+int64_t qmm_groups_per_row(int64_t cols, int group_size);
+
+/* Static English text for a status code (never NULL). */
+const char* qmm_status_string(int status);
+
+/* QMM_OK when the current CUDA device is compute capability 10.0. */
+qmm_status qmm_device_check(void);
+
+/* Dense -> (packed, scales, biases).  w: [rows, cols] in w_dtype.  Output
+ * scales/biases in s_dtype.  Bit-exact with the oracle's definition (see the
+ * quantizer paragraph above).  rows == 0 is a no-op. */
+qmm_status qmm_quantize(const void* w, qmm_dtype w_dtype, int64_t rows, int64_t cols,
+                        int group_size, int bits, qmm_dtype s_dtype, uint32_t* packed,
+                        void* scales, void* biases, void* stream);
+
+/* out[r][i] = fmaf(q, scale, bias) stored in out_dtype (one RNE rounding
+ * for f16/bf16).  out: [w->rows, w->cols] row-major. */
+qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, void* stream);
+
+/* y[M, N] = x[M, K] . dequant(W)^T  (transpose = 1: W is [N, K], w->rows = N,
+ *                                    w->cols = K)
+ * y[M, N] = x[M, K] . dequant(W)    (transpose = 0: W is [K, N] quantized
+ *                                    along N, w->rows = K, w->cols = N)
+ * x_dtype must equal w->sdtype; y_dtype is x_dtype or QMM_F32 (same
+ * arithmetic, different final store).  Accumulation is fp32.  M == 0 is a
+ * no-op.  bf16/f16 with transpose = 1 use the tensor-core kernels. */
+qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
+                      const qmm_qweight* w, int transpose, void* y, qmm_dtype y_dtype,
+                      void* stream);
+
+/* out[i, :] = a[i*src1_stride : i*src1_stride + n_cols] . dequant(W[ids[i]])^T,
+ * i in [0, n_selected).  ids: device int32[n_selected].  out: [n_selected,
+ * n_rows] in out_dtype (a_dtype or QMM_F32).  A pair whose id is outside
+ * [0, num_experts) gets a zero row and sets QMM_ERR_BAD_EXPERT_ID in
+ * *d_status. */
+qmm_status qmm_moe_gemv_id(const void* a, qmm_dtype a_dtype, const int32_t* ids,
+                           int64_t n_selected, int64_t src1_stride, const qmm_expert_stack* w,
+                           void* out, qmm_dtype out_dtype, int32_t* d_status, void* stream);
+
+/* Batched form: ids is [m, top_k] row-major; pair p in [0, m*top_k) reads
+ * a[(p/top_k)*outer_stride + (p%top_k)*inner_stride : ... + n_cols] and
+ * writes out[p, :]. */
+qmm_status qmm_moe_gemv_id_batched(const void* a, qmm_dtype a_dtype, const int32_t* ids,
+                                   int64_t m, int64_t top_k, int64_t outer_stride,
+                                   int64_t inner_stride, const qmm_expert_stack* w, void* out,
+                                   qmm_dtype out_dtype, int32_t* d_status, void* stream);
+
+/* silu_out[i, :] = SiLU(a . gate_e^T) * (a . up_e^T), e = ids[i], with
+ * SiLU(g) = g / (1 + exp(-g)); every pair reads a[0 : n_cols] (the call has
+ * no stride).  gate and up must have identical shapes and parameters
+ * (QMM_ERR_INVALID_ARG otherwise).  Gate and up are computed in one pass. */
+qmm_status qmm_moe_gemv_id_gate_up_silu(const void* a, qmm_dtype a_dtype, const int32_t* ids,
+                                        int64_t n_selected, const qmm_expert_stack* gate,
+                                        const qmm_expert_stack* up, void* silu_out,
+                                        qmm_dtype out_dtype, int32_t* d_status, void* stream);
+
+/* Batched fused form: pair offsets as in qmm_moe_gemv_id_batched. */
+qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype,
+                                                const int32_t* ids, int64_t m, int64_t top_k,
+                                                int64_t outer_stride, int64_t inner_stride,
+                                                const qmm_expert_stack* gate,
+                                                const qmm_expert_stack* up, void* silu_out,
+                                                qmm_dtype out_dtype, int32_t* d_status,
+                                                void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QMM_H_ */

@@ -1,0 +1,117 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/qmm.h declares, and rejects bad arguments on the host before any
+CUDA call.  No computation is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_quantized_qmm_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = open(os.path.join(ROOT, "include", "qmm.h")).read()
+
+
+@pytest.fixture(scope="module")
+def L():
+    return _lib.load()
+
+
+def declared_functions():
+    body = re.sub(r"/\*.*?\*/", "", HEADER, flags=re.S)
+    return sorted(set(re.findall(r"\b(qmm_[a-z0-9_]+)\s*\(", body)))
+
+
+def test_header_declares_the_abi():
+    names = declared_functions()
+    assert set(names) == set(_lib.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} missing from libqmm.so"
+
+
+def test_enum_values_match_header():
+    for name, val in [("QMM_OK", 0), ("QMM_ERR_INVALID_ARG", 1), ("QMM_ERR_UNSUPPORTED", 2),
+                      ("QMM_ERR_DTYPE", 3), ("QMM_ERR_ALIGNMENT", 4), ("QMM_ERR_CUDA", 5),
+                      ("QMM_ERR_TIMEOUT", 6), ("QMM_ERR_BAD_EXPERT_ID", 7), ("QMM_F32", 0),
+                      ("QMM_F16", 1), ("QMM_BF16", 2)]:
+        assert re.search(rf"\b{name}\s*=\s*{val}\b", HEADER), name
+        assert getattr(_lib, name) == val
+
+
+def test_size_helpers(L):
+    assert L.qmm_packed_words_per_row(4096, 4) == 512
+    assert L.qmm_packed_words_per_row(4096, 3) == 384
+    assert L.qmm_packed_words_per_row(32, 6) == 6
+    assert L.qmm_packed_words_per_row(33, 3) == -1
+    assert L.qmm_packed_words_per_row(64, 5) == -1
+    assert L.qmm_groups_per_row(4096, 64) == 64
+    assert L.qmm_groups_per_row(96, 64) == -1
+    assert L.qmm_groups_per_row(64, 16) == -1
+    for code in range(8):
+        assert len(_lib.status_string(code)) > 0
+
+
+A = 0x10000  # an aligned fake device address: never dereferenced by these calls
+
+
+def qw(bits=4, gs=64, rows=8, cols=128, sdtype=_lib.QMM_BF16, mode=0, packed=A):
+    return _lib.QWeightC(packed, A, A, sdtype, rows, cols, gs, bits, mode)
+
+
+def matmul(L, w, x=A, x_dtype=_lib.QMM_BF16, M=1, K=128, transpose=1, y=A, y_dtype=_lib.QMM_BF16):
+    return L.qmm_matmul(x, x_dtype, M, K, ctypes.byref(w), transpose, y, y_dtype, None)
+
+
+def test_matmul_validation(L):
+    assert matmul(L, qw(bits=5)) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(gs=48)) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(cols=96, gs=64)) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(mode=_lib.QMM_MODE_NVFP4)) == _lib.QMM_ERR_UNSUPPORTED
+    assert matmul(L, qw(), x_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
+    assert matmul(L, qw(), y_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
+    assert matmul(L, qw(), K=256) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(), transpose=2) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(packed=0)) == _lib.QMM_ERR_ALIGNMENT
+    assert matmul(L, qw(packed=A + 4)) == _lib.QMM_ERR_ALIGNMENT
+    assert matmul(L, qw(), x=A + 2) == _lib.QMM_ERR_ALIGNMENT
+    assert matmul(L, qw(), M=-1) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(), M=0) == _lib.QMM_OK  # empty: nothing launched
+
+
+def test_quantize_dequantize_validation(L):
+    q = L.qmm_quantize
+    assert q(A, 0, 4, 128, 64, 7, 2, A, A, A, None) == _lib.QMM_ERR_INVALID_ARG
+    assert q(A, 0, 4, 100, 64, 4, 2, A, A, A, None) == _lib.QMM_ERR_INVALID_ARG
+    assert q(A, 9, 4, 128, 64, 4, 2, A, A, A, None) == _lib.QMM_ERR_DTYPE
+    assert q(A, 0, 4, 128, 64, 4, 2, A + 8, A, A, None) == _lib.QMM_ERR_ALIGNMENT
+    assert q(A, 0, 0, 128, 64, 4, 2, A, A, A, None) == _lib.QMM_OK
+    w = qw(rows=0)
+    assert L.qmm_dequantize(ctypes.byref(w), A, _lib.QMM_F32, None) == _lib.QMM_OK
+    w = qw(bits=1)
+    assert L.qmm_dequantize(ctypes.byref(w), A, _lib.QMM_F32, None) == _lib.QMM_ERR_INVALID_ARG
+
+
+def stack(E=4, rows=16, cols=128, bits=4, gs=64, sdtype=_lib.QMM_BF16):
+    return _lib.ExpertStackC(A, A, A, sdtype, E, rows, cols, gs, bits)
+
+
+def test_moe_validation(L):
+    s = stack()
+    f = L.qmm_moe_gemv_id
+    assert f(A, _lib.QMM_BF16, A, 0, 128, ctypes.byref(s), A, _lib.QMM_BF16, None, None) == _lib.QMM_OK
+    assert f(A, _lib.QMM_F16, A, 2, 128, ctypes.byref(s), A, _lib.QMM_F16, None, None) == _lib.QMM_ERR_DTYPE
+    assert f(A, _lib.QMM_BF16, A + 2, 2, 128, ctypes.byref(s), A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_ALIGNMENT
+    bad = stack(E=0)
+    assert f(A, _lib.QMM_BF16, A, 2, 128, ctypes.byref(bad), A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_INVALID_ARG
+    g, u = stack(), stack(rows=32)
+    h = L.qmm_moe_gemv_id_gate_up_silu
+    assert h(A, _lib.QMM_BF16, A, 2, ctypes.byref(g), ctypes.byref(u), A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_INVALID_ARG
+    assert h(A, _lib.QMM_BF16, A, 2, ctypes.byref(g), None, A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_INVALID_ARG
+    b = L.qmm_moe_gemv_id_batched
+    assert b(A, _lib.QMM_BF16, A, 2, 0, 0, 0, ctypes.byref(s), A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_INVALID_ARG
+    bb = L.qmm_moe_gemv_id_gate_up_silu_batched
+    assert bb(A, _lib.QMM_BF16, A, 0, 8, 0, 0, ctypes.byref(g), ctypes.byref(g), A, _lib.QMM_BF16, None, None) == _lib.QMM_OK

@@ -1,0 +1,140 @@
+"""GPU parity of the MoE indirect-dispatch GEMVs (single, batched, fused
+gate+up+SiLU) against the CPU oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import ORC, gate, np_storage, qweight_np, rne_equal
+from weight_only_quantized_qmm_b200 import api
+from weight_only_quantized_qmm_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def make_stack(E, n_rows, n_cols, bits, gs, seed, dtype=torch.bfloat16):
+    w = wl.gen_weight(E * n_rows, n_cols, seed)
+    qw = api.qmm_quantize(w.to(DEV), gs, bits, dtype)
+    torch.cuda.synchronize()
+    p, s, b = qweight_np(qw)
+    st = api.ExpertStack.from_qweight(qw, E)
+    ost = oracle.Stack(p, s, b, ORC[dtype], E, n_rows, n_cols, gs, bits)
+    return st, ost
+
+
+@pytest.mark.parametrize("bits,gs", [(4, 64), (3, 32), (8, 128), (2, 64), (6, 64)])
+def test_moe_gemv_id_single(bits, gs):
+    E, n_rows, n_cols = 9, 80, 2 * gs * 2
+    st, ost = make_stack(E, n_rows, n_cols, bits, gs, 10 + bits)
+    n_sel, stride = 6, n_cols + 32
+    a = wl.gen_x(1, stride * n_sel, 11).reshape(-1)
+    ids = torch.tensor([3, 0, 8, 3, 5, 3], dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out32 = api.qmm_moe_gemv_id(a.to(DEV), ids.to(DEV), n_sel, stride, st, torch.float32, d_status=status)
+    out16 = api.qmm_moe_gemv_id(a.to(DEV), ids.to(DEV), n_sel, stride, st)
+    torch.cuda.synchronize()
+    ref, rc = oracle.moe_gemv_id(np_storage(a), oracle.BF16, ids.numpy(), n_sel, stride, ost)
+    assert rc == oracle.ORC_OK and int(status.item()) == 0
+    gate(out32.cpu().numpy(), ref, f"moe b{bits}")
+    rne_equal(out16, out32)
+
+
+@pytest.mark.parametrize("m,top_k", [(3, 2), (5, 4), (20, 4)])
+def test_moe_gemv_id_batched(m, top_k):
+    E, n_rows, n_cols, bits, gs = 16, 64, 256, 4, 64
+    st, ost = make_stack(E, n_rows, n_cols, bits, gs, 20 + m)
+    outer, inner = top_k * n_cols, n_cols  # [m, top_k, n_cols] activations
+    a = wl.gen_x(m * top_k, n_cols, 21).reshape(-1)
+    ids = wl.gen_moe_ids(m, E, top_k, 22)
+    out32 = api.qmm_moe_gemv_id_batched(a.to(DEV), ids.to(DEV), m, top_k, outer, inner, st,
+                                        torch.float32)
+    torch.cuda.synchronize()
+    ref, rc = oracle.moe_gemv_id_batched(np_storage(a), oracle.BF16, ids.numpy(), m, top_k, outer,
+                                         inner, ost)
+    assert rc == oracle.ORC_OK
+    gate(out32.cpu().numpy(), ref, "batched")
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_moe_gate_up_silu(bits):
+    E, n_rows, n_cols, gs = 12, 96, 512, 64
+    g, og = make_stack(E, n_rows, n_cols, bits, gs, 30)
+    u, ou = make_stack(E, n_rows, n_cols, bits, gs, 31)
+    a = wl.gen_x(1, n_cols, 32).reshape(-1)
+    ids = torch.tensor([7, 1, 11, 0, 4, 7, 2, 9], dtype=torch.int32)
+    out32 = api.qmm_moe_gemv_id_gate_up_silu(a.to(DEV), ids.to(DEV), 8, g, u, torch.float32)
+    out16 = api.qmm_moe_gemv_id_gate_up_silu(a.to(DEV), ids.to(DEV), 8, g, u)
+    torch.cuda.synchronize()
+    ref, rc = oracle.moe_gate_up_silu(np_storage(a), oracle.BF16, ids.numpy(), 8, og, ou)
+    assert rc == oracle.ORC_OK
+    gate(out32.cpu().numpy(), ref, "gate_up_silu")
+    rne_equal(out16, out32)
+
+
+def test_moe_gate_up_silu_batched_many_tokens_per_expert():
+    """more than 16 pairs on one expert: the kernel makes several token passes"""
+    E, n_rows, n_cols, bits, gs = 4, 48, 256, 4, 64
+    g, og = make_stack(E, n_rows, n_cols, bits, gs, 40)
+    u, ou = make_stack(E, n_rows, n_cols, bits, gs, 41)
+    m, top_k = 24, 2
+    a = wl.gen_x(m, n_cols, 42).reshape(-1)
+    ids = wl.gen_moe_ids(m, E, top_k, 43)
+    out32 = api.qmm_moe_gemv_id_gate_up_silu_batched(a.to(DEV), ids.to(DEV), m, top_k, n_cols, 0,
+                                                     g, u, torch.float32)
+    torch.cuda.synchronize()
+    ref, rc = oracle.moe_gate_up_silu_batched(np_storage(a), oracle.BF16, ids.numpy(), m, top_k,
+                                              n_cols, 0, og, ou)
+    assert rc == oracle.ORC_OK
+    gate(out32.cpu().numpy(), ref, "batched gate_up_silu")
+
+
+def test_moe_bad_id_zero_row_and_status():
+    E, n_rows, n_cols, bits, gs = 3, 32, 128, 4, 64
+    st, ost = make_stack(E, n_rows, n_cols, bits, gs, 50)
+    a = wl.gen_x(1, n_cols, 51).reshape(-1)
+    ids = torch.tensor([1, 7, -2, 0], dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.full((4, n_rows), float("nan"), device=DEV)
+    api.qmm_moe_gemv_id(a.to(DEV), ids.to(DEV), 4, 0, st, out=out, d_status=status)
+    torch.cuda.synchronize()
+    ref, rc = oracle.moe_gemv_id(np_storage(a), oracle.BF16, ids.numpy(), 4, 0, ost)
+    assert rc == oracle.ORC_ERR_ID
+    assert int(status.item()) & 7 == 7  # QMM_ERR_BAD_EXPERT_ID
+    o = out.cpu().numpy()
+    assert np.all(o[1] == 0) and np.all(o[2] == 0)
+    gate(o[[0, 3]], ref[[0, 3]], "valid pairs")
+
+
+@pytest.mark.parametrize("case", wl.WORKLOADS.moe, ids=lambda c: c.name)
+def test_moe_config_full_size(case):
+    """128 experts, gate/up [768 x 2048], down [2048 x 768], top-8, T tokens:
+    fused gate+up+SiLU then down (src1_stride = 768), compared on sampled rows."""
+    E, dff, dm = case.num_experts, case.d_ff, case.d_model
+    gate_s, og = make_stack(E, dff, dm, case.bits, case.group_size, case.seed)
+    up_s, ou = make_stack(E, dff, dm, case.bits, case.group_size, case.seed + 1)
+    down_s, od = make_stack(E, dm, dff, case.bits, case.group_size, case.seed + 2)
+    T, k = case.tokens, case.top_k
+    a = wl.gen_x(T, dm, case.seed + 3)
+    ids = wl.gen_moe_ids(T, E, k, case.seed + 4)
+    h = api.qmm_moe_gemv_id_gate_up_silu_batched(a.to(DEV).reshape(-1), ids.to(DEV), T, k, dm, 0,
+                                                 gate_s, up_s, torch.float32)
+    h16 = api.qmm_moe_gemv_id_gate_up_silu_batched(a.to(DEV).reshape(-1), ids.to(DEV), T, k, dm, 0,
+                                                   gate_s, up_s)
+    out = api.qmm_moe_gemv_id(h16.reshape(-1), ids.to(DEV).reshape(-1), T * k, dff, down_s,
+                              torch.float32)
+    torch.cuda.synchronize()
+    rne_equal(h16, h)
+    rng = np.random.default_rng(case.seed)
+    pairs = np.unique(rng.integers(0, T * k, min(T * k, 12)))
+    a_np = np_storage(a).reshape(-1)
+    ids_np = ids.numpy().reshape(-1)
+    for p in pairs:
+        tok = p // k
+        ref, rc = oracle.moe_gate_up_silu(a_np[tok * dm:(tok + 1) * dm], oracle.BF16,
+                                          ids_np[p:p + 1], 1, og, ou)
+        gate(h.cpu().numpy()[p], ref[0], f"gate_up pair {p}")
+    h16_np = np_storage(h16).reshape(-1)
+    ref_d, rc = oracle.moe_gemv_id(h16_np, oracle.BF16, ids_np, T * k, dff, od)
+    assert rc == oracle.ORC_OK
+    gate(out.cpu().numpy(), ref_d, "down")

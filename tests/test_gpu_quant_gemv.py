@@ -1,0 +1,200 @@
+"""GPU parity: quantize, dequantize and the decode-shaped matmul against the
+CPU oracle, through the C ABI (libqmm.so via the ctypes binding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.helpers import ORC, gate, np_storage, packed_np, qweight_np, rne_equal
+from weight_only_quantized_qmm_b200 import api
+from weight_only_quantized_qmm_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+BITS = [2, 3, 4, 6, 8]
+GROUPS = [32, 64, 128]
+DEV = "cuda"
+
+
+def _quant_pair(n, k, bits, gs, s_dtype, seed, w_dtype=torch.float32):
+    w = wl.gen_weight(n, k, seed).to(w_dtype)
+    qw = api.qmm_quantize(w.to(DEV), gs, bits, s_dtype)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(np_storage(w), ORC[w_dtype], gs, bits, ORC[s_dtype])
+    return w, qw, ref
+
+
+# ------------------------------------------------------------------ quantize / dequantize
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("gs", GROUPS)
+@pytest.mark.parametrize("s_dtype", [torch.bfloat16, torch.float16, torch.float32])
+def test_quantize_bit_exact(bits, gs, s_dtype):
+    _, qw, (p_ref, s_ref, b_ref) = _quant_pair(37, 4 * gs, bits, gs, s_dtype, 10 + bits + gs)
+    p, s, b = qweight_np(qw)
+    assert np.array_equal(p, p_ref), "packed words differ"
+    assert np.array_equal(s, s_ref), "scales differ"
+    assert np.array_equal(b, b_ref), "biases differ"
+
+
+@pytest.mark.parametrize("w_dtype", [torch.bfloat16, torch.float16])
+def test_quantize_half_inputs_bit_exact(w_dtype):
+    _, qw, (p_ref, s_ref, b_ref) = _quant_pair(64, 256, 4, 64, w_dtype, 5, w_dtype)
+    p, s, b = qweight_np(qw)
+    assert np.array_equal(p, p_ref) and np.array_equal(s, s_ref) and np.array_equal(b, b_ref)
+
+
+def test_quantize_degenerate_groups():
+    """constant groups, -0.0, on-grid values and a tie of the rounding rule"""
+    w = torch.zeros(4, 64)
+    w[1] = 0.75
+    w[2] = -0.0
+    w[3, :4] = torch.tensor([0.0, 6.5, 7.5, 15.0])
+    qw = api.qmm_quantize(w.to(DEV), 32, 4, torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(w.numpy(), oracle.F32, 32, 4, oracle.F32)
+    for got, exp in zip(qweight_np(qw), ref):
+        assert np.array_equal(got, exp)
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("gs", GROUPS)
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_dequantize_bit_exact(bits, gs, out_dtype):
+    _, qw, (p_ref, s_ref, b_ref) = _quant_pair(19, 2 * gs, bits, gs, torch.bfloat16, 40 + bits)
+    out = api.qmm_dequantize(qw, out_dtype)
+    torch.cuda.synchronize()
+    ref = oracle.dequantize(p_ref, s_ref, b_ref, oracle.BF16, 2 * gs, gs, bits, ORC[out_dtype])
+    assert np.array_equal(np_storage(out), ref)
+
+
+# ------------------------------------------------------------------ decode GEMV (M <= 16)
+def _gemv_case(M, N, K, bits, gs, dtype, seed):
+    w, qw, (p, s, b) = _quant_pair(N, K, bits, gs, dtype, seed)
+    x = wl.gen_x(M, K, seed + 1, {torch.bfloat16: "bf16", torch.float16: "f16",
+                                  torch.float32: "f32"}[dtype])
+    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
+    y16 = api.qmm_matmul(x.to(DEV), qw, True, dtype)
+    torch.cuda.synchronize()
+    yref = oracle.matmul(np_storage(x), ORC[dtype], p, s, b, ORC[dtype], N, gs, bits)
+    return y32, y16, yref
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("gs", GROUPS)
+def test_gemv_all_widths_and_groups(bits, gs):
+    y32, y16, yref = _gemv_case(3, 200, 4 * gs + 2 * gs, bits, gs, torch.bfloat16, 100 + bits + gs)
+    gate(y32.cpu().numpy(), yref, f"b{bits} g{gs}")
+    rne_equal(y16, y32)
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 9, 13, 16])
+def test_gemv_token_counts(M):
+    y32, y16, yref = _gemv_case(M, 333, 1024, 4, 64, torch.bfloat16, 200 + M)
+    gate(y32.cpu().numpy(), yref, f"M={M}")
+    rne_equal(y16, y32)
+
+
+@pytest.mark.parametrize("bits", [4, 8, 3])
+def test_gemv_fp16(bits):
+    y32, y16, yref = _gemv_case(4, 160, 512, bits, 64, torch.float16, 300 + bits)
+    gate(y32.cpu().numpy(), yref, "f16")
+    rne_equal(y16, y32)
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (15, 32), (17, 128), (3000, 64)])
+def test_gemv_ragged_shapes(N, K):
+    gs = 32 if K % 64 else 64
+    y32, y16, yref = _gemv_case(2, N, K, 4, gs, torch.bfloat16, 400 + N)
+    gate(y32.cpu().numpy(), yref, f"N={N} K={K}")
+    rne_equal(y16, y32)
+
+
+def test_gemv_long_k_chunks_x_staging():
+    """M=16 with K large enough that staged x is split into several K chunks."""
+    y32, y16, yref = _gemv_case(16, 64, 8192, 8, 32, torch.bfloat16, 500)
+    gate(y32.cpu().numpy(), yref, "chunked K")
+    rne_equal(y16, y32)
+
+
+def test_tiny_config():
+    """W fp32 [256, 512] ~ N(0, 0.02), g64 b4; x bf16 [4, 512] ~ N(0, 1); seed 0."""
+    c = wl.WORKLOADS.tiny
+    w = wl.gen_weight(c.N, c.K, c.seed)
+    x = wl.gen_x(c.M, c.K, c.seed + 1)
+    qw = api.qmm_quantize(w.to(DEV), c.group_size, c.bits, torch.bfloat16)
+    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
+    y16 = api.qmm_matmul(x.to(DEV), qw, True)
+    torch.cuda.synchronize()
+    p, s, b = oracle.quantize(w.numpy(), oracle.F32, c.group_size, c.bits, oracle.BF16)
+    assert np.array_equal(packed_np(qw.packed), p)
+    yref = oracle.matmul(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, c.N, c.group_size, c.bits)
+    assert tuple(y16.shape) == (4, 256)
+    gate(y32.cpu().numpy(), yref, "tiny")
+    rne_equal(y16, y32)
+
+
+def test_iota_example_on_gpu():
+    """the page's iota example in fp32 (x and scales f32) -> shape (3, 4)"""
+    w = wl.iota(4, 128)
+    x = wl.iota(3, 128)
+    qw = api.qmm_quantize(w.to(DEV), 64, 4, torch.float32)
+    y = api.qmm_matmul(x.to(DEV), qw)
+    torch.cuda.synchronize()
+    p, s, b = oracle.quantize(w.numpy(), oracle.F32, 64, 4, oracle.F32)
+    yref = oracle.matmul(x.numpy(), oracle.F32, p, s, b, oracle.F32, 4, 64, 4)
+    assert tuple(y.shape) == (3, 4)
+    np.testing.assert_allclose(y.cpu().numpy(), yref, rtol=1e-6)
+
+
+# ------------------------------------------------------------------ generic paths
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_fp32_activations_and_wide_m(bits):
+    M, N, K, gs = 21, 96, 256, 32
+    w, qw, (p, s, b) = _quant_pair(N, K, bits, gs, torch.float32, 600 + bits)
+    x = wl.gen_x(M, K, 601, "f32")
+    y = api.qmm_matmul(x.to(DEV), qw)
+    torch.cuda.synchronize()
+    yref = oracle.matmul(x.numpy(), oracle.F32, p, s, b, oracle.F32, N, gs, bits)
+    gate(y.cpu().numpy(), yref, "f32")
+
+
+@pytest.mark.parametrize("bits", [2, 4, 6])
+def test_transpose_false_awq_layout(bits):
+    M, K, N, gs = 5, 96, 128, 64
+    # W stored [K, N] quantized along N
+    w, qw, (p, s, b) = _quant_pair(K, N, bits, gs, torch.bfloat16, 700 + bits)
+    x = wl.gen_x(M, K, 701)
+    y = api.qmm_matmul(x.to(DEV), qw, transpose=False, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    yref = oracle.matmul(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, N, gs, bits, False)
+    gate(y.cpu().numpy(), yref, "transpose=0")
+
+
+def test_zero_rows_is_noop():
+    qw = api.qmm_quantize(wl.gen_weight(64, 128, 1).to(DEV), 64, 4, torch.bfloat16)
+    x = torch.empty(0, 128, dtype=torch.bfloat16, device=DEV)
+    y = api.qmm_matmul(x, qw)
+    assert tuple(y.shape) == (0, 64)
+
+
+# ------------------------------------------------------------------ full-size decode, sampled
+@pytest.mark.parametrize("case", wl.WORKLOADS.decode, ids=lambda c: c.name)
+def test_decode_full_size_sampled(case):
+    w = wl.gen_weight(case.N, case.K, case.seed)
+    x = wl.gen_x(case.M, case.K, case.seed + 1)
+    qw = api.qmm_quantize(w.to(DEV), case.group_size, case.bits, torch.bfloat16)
+    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
+    y16 = api.qmm_matmul(x.to(DEV), qw)
+    torch.cuda.synchronize()
+    p, s, b = qweight_np(qw)
+    rng = np.random.default_rng(case.seed)
+    cols = np.unique(np.concatenate([rng.integers(0, case.N, 384), [0, case.N - 1]]))
+    coords = [(0, int(n)) for n in cols]
+    yref = oracle.matmul_elements(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
+                                  case.group_size, case.bits, coords)
+    ys = y32.cpu().numpy()[0, cols]
+    gate(ys, yref, case.name)
+    rne_equal(y16, y32)
+    # the quantizer itself is exact at full size: spot-check 64 rows
+    rows = rng.integers(0, case.N, 64)
+    pr, sr, br = oracle.quantize(w.numpy()[rows], oracle.F32, case.group_size, case.bits, oracle.BF16)
+    assert np.array_equal(p[rows], pr) and np.array_equal(s[rows], sr) and np.array_equal(b[rows], br)
