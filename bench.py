@@ -1,0 +1,627 @@
+#!/usr/bin/env python3
+"""Benchmark: decode GEMV achieved HBM GB/s on B200 (plus the prefill GEMM
+TFLOP/s and the MoE GEMV GB/s as secondary lines of the same JSON record).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One *step* = the decode workload once: y = x . dequant(W)^T at M = 1 for the
+three weight shapes 4096x4096, 14336x4096 and 4096x14336 (4-bit affine,
+group 64, bf16 activations, scales and biases).  `value` is the algorithmic
+bytes of those three calls (packed codes + scales + biases + x + y) summed over
+all steps of all ranks, divided by the timed device time (max over ranks).
+
+Timing: W warm-up steps, then K steps bracketed by barrier +
+cuda.synchronize, CUDA events on the launching stream.  The steps are
+replayed from a CUDA graph (host launch overhead is larger than the kernels)
+and rotate over weight copies larger than L2.  Under torchrun each rank runs
+the same workload on its own GPU (independent replicas, weak scaling).
+
+--impl reference times the CPU oracle (oracle/) on the same workload and
+metric, on a bounded sample per step; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode GEMV achieved HBM GB/s (% of peak); prefill GEMM TFLOP/s (% of bf16 peak)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def decode_bytes(M, N, K, bits, gs):
+    # packed codes + bf16 scales and biases + bf16 x + bf16 y
+    return N * K * bits // 8 + N * (K // gs) * 4 + 2 * M * K + 2 * M * N
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    HW_SLOW, HW_THERM, SW_THERM, SW_POWER = 0x8, 0x40, 0x20, 0x4
+
+    def __init__(self, device_index: int, period_s: float = 0.05):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            props = torch.cuda.get_device_properties(device_index)
+            self.h = None
+            bus = getattr(props, "pci_bus_id", None)
+            if bus is not None:
+                busid = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), bus,
+                                             getattr(props, "pci_device_id", 0))
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = device_index
+                if vis and vis.split(",")[0].strip().isdigit():
+                    idx = int(vis.split(",")[device_index].strip())
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((sm, int(r)))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = {self.HW_SLOW: "hw_slowdown", self.HW_THERM: "hw_thermal_slowdown",
+                 self.SW_THERM: "sw_thermal_slowdown", self.SW_POWER: "sw_power_cap"}
+        seen = set()
+        for _, r in self.samples:
+            for bit, n in names.items():
+                if r & bit:
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(seen), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- traffic record
+def traffic_record(name):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (sha256 of the .cu file recorded in the summary)."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None, None
+    rec = {}
+    for line in txt.splitlines():
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            rec[k.strip()] = v.strip()
+    src = rec.get("source_file")
+    if not src:
+        return None, None
+    try:
+        cur = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+    except OSError:
+        return None, None
+    if cur != rec.get("source_sha256"):
+        return None, "stale"
+    return rec, "current"
+
+
+# ---------------------------------------------------------------- our arm
+def build_decode(torch, api, wl, n_sets, dev):
+    cases = wl.WORKLOADS.decode
+    sets = []
+    base = []
+    for c in cases:
+        w = wl.gen_weight(c.N, c.K, c.seed)
+        qw = api.qmm_quantize(w.to(dev), c.group_size, c.bits, torch.bfloat16)
+        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+        base.append((c, qw, x))
+    torch.cuda.synchronize()
+    for s in range(n_sets):
+        cur = []
+        for c, qw, x in base:
+            q2 = qw if s == 0 else api.QWeight(qw.packed.clone(), qw.scales.clone(),
+                                               qw.biases.clone(), qw.rows, qw.cols,
+                                               qw.group_size, qw.bits)
+            y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+            cur.append((c, q2, x, y))
+        sets.append(cur)
+    torch.cuda.synchronize()
+    return sets
+
+
+def run_ours(args):
+    import torch
+
+    from weight_only_quantized_qmm_b200 import api
+    from weight_only_quantized_qmm_b200 import workloads as wl
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    hbm_peak, bf16_peak, bf16_sust, peak_src = peaks()
+    assert api.qmm_device_check() == 0, "needs a compute capability 10.0 GPU"
+
+    cases = wl.WORKLOADS.decode
+    step_bytes = sum(decode_bytes(c.M, c.N, c.K, c.bits, c.group_size) for c in cases)
+    n_sets = max(2, int(np.ceil(3 * L2_BYTES / step_bytes)))  # rotate > 3x L2 of weights
+    sets = build_decode(torch, api, wl, n_sets, dev)
+
+    stream = torch.cuda.Stream(device=dev)
+    launches_per_step = len(cases)
+
+    def one_step(s):
+        for c, qw, x, y in sets[s % n_sets]:
+            api.qmm_matmul(x, qw, True, out=y, stream=stream)
+
+    # capture G steps (one full rotation, repeated) into one graph
+    G = n_sets * max(1, 48 // n_sets)
+    with torch.cuda.stream(stream):
+        for s in range(max(args.warmup, 3)):  # eager warm-up (also configures the kernels)
+            one_step(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(G):
+            one_step(s)
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // G)
+    steps = reps * G
+    # warm-up replays (W steps at least); graphs replay on the current stream
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-args.warmup // G))):
+            graph.replay()
+    torch.cuda.synchronize()
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler, torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(world, ms)
+    ms_step = ms / steps
+    value = step_bytes * steps * world / (ms * 1e-3) / 1e9
+
+    # per-shape launch durations (events around each launch inside one graph)
+    per_shape = {}
+    g2 = torch.cuda.CUDAGraph()
+    # external events: recorded as graph nodes, so each one is a GPU timestamp
+    evs = [[(torch.cuda.Event(enable_timing=True, external=True),
+             torch.cuda.Event(enable_timing=True, external=True))
+            for _ in cases] for _ in range(n_sets)]
+    with torch.cuda.graph(g2, stream=stream):
+        for s in range(n_sets):
+            for i, (c, qw, x, y) in enumerate(sets[s]):
+                evs[s][i][0].record(stream)
+                api.qmm_matmul(x, qw, True, out=y, stream=stream)
+                evs[s][i][1].record(stream)
+    durs = [[] for _ in cases]
+    for _ in range(20):
+        with torch.cuda.stream(stream):
+            g2.replay()
+        torch.cuda.synchronize()
+        for s in range(n_sets):
+            for i in range(len(cases)):
+                durs[i].append(evs[s][i][0].elapsed_time(evs[s][i][1]))
+    tot_b, tot_ms = 0.0, 0.0
+    for i, c in enumerate(cases):
+        d = statistics.median(durs[i])
+        b = decode_bytes(c.M, c.N, c.K, c.bits, c.group_size)
+        per_shape[c.name] = {"us": round(d * 1e3, 3), "GB/s": round(b / (d * 1e-3) / 1e9, 1),
+                             "frac": round(b / (d * 1e-3) / 1e9 / hbm_peak, 3)}
+        tot_b += b
+        tot_ms += d
+    achieved = tot_b / (tot_ms * 1e-3) / 1e9
+    rec, state = traffic_record("qgemv_decode_m1.txt")
+    traffic = None
+    if rec is not None and state == "current":
+        try:
+            traffic = float(rec["dram_bytes_per_launch_avg"])
+        except (KeyError, ValueError):
+            traffic = None
+
+    # end to end through the public API with host buffers (pinned), per step:
+    # H2D of x, the three calls, D2H of y, synchronize
+    e2e = None
+    if rank == 0 or world > 1:
+        xs_h = [x.cpu().pin_memory() for (_, _, x, _) in sets[0]]
+        ys_h = [torch.empty(c.M, c.N, dtype=torch.bfloat16).pin_memory() for c in cases]
+        h2d = sum(t.numel() * t.element_size() for t in xs_h)
+        d2h = sum(t.numel() * t.element_size() for t in ys_h)
+        n_e2e = min(2000, max(50, args.steps // 10))
+
+        def e2e_step(s):
+            for i, (c, qw, x, y) in enumerate(sets[s % n_sets]):
+                x.copy_(xs_h[i], non_blocking=True)
+                api.qmm_matmul(x, qw, True, out=y)
+                ys_h[i].copy_(y, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+        for s in range(10):
+            e2e_step(s)
+        barrier(world)
+        t0 = time.perf_counter()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(n_e2e):
+            e2e_step(s)
+        e1.record()
+        torch.cuda.synchronize()
+        ms_e2e = max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3)
+        ms_e2e = max_over_ranks(world, ms_e2e)
+        e2e = {"value": round(step_bytes * n_e2e * world / (ms_e2e * 1e-3) / 1e9, 2),
+               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ms_e2e / n_e2e, 4), "steps": n_e2e}
+
+    secondary = {}
+    if not args.no_secondary and rank == 0:
+        secondary = run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_seconds)
+
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: W=0.02*randn quantized 4-bit g64, x=randn->bf16)",
+        "config": {"workload": "decode GEMV M=1, 4-bit affine g64, bf16 x/scales/biases; "
+                               "N x K = 4096x4096 + 14336x4096 + 4096x14336 per step",
+                   "global_batch": world, "M": 1, "bits": 4, "group_size": 64,
+                   "l2": f"rotates {n_sets} weight copies ({n_sets * step_bytes / 1e6:.0f} MB) > L2 126 MB",
+                   "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
+                     "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                     "peak_source": peak_src, "kernel": "qgemv_kernel<4,64,bf16,1,false>",
+                     "per_shape": per_shape},
+        "e2e": e2e,
+        "gpu_launches": steps * launches_per_step,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "secondary": secondary,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph, g2
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def time_graph(torch, fn, stream, reps=20, inner=4):
+    with torch.cuda.stream(stream):
+        fn()
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(inner):
+            fn()
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    times = []
+    for _ in range(reps):
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / inner)
+    del g
+    return statistics.median(times)
+
+
+def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    out = {}
+    # MoE decode: fused gate+up+SiLU then down, T = 1 and 16, top-8 of 128
+    for case in wl.WORKLOADS.moe[:2]:
+        E, dff, dm, T, k = case.num_experts, case.d_ff, case.d_model, case.tokens, case.top_k
+        n_sets = 3
+        stacks = []
+        for s in range(n_sets):
+            g = api.qmm_quantize(wl.gen_weight(E * dff, dm, case.seed + 10 * s).to(dev), 64, 4, torch.bfloat16)
+            u = api.qmm_quantize(wl.gen_weight(E * dff, dm, case.seed + 10 * s + 1).to(dev), 64, 4, torch.bfloat16)
+            d = api.qmm_quantize(wl.gen_weight(E * dm, dff, case.seed + 10 * s + 2).to(dev), 64, 4, torch.bfloat16)
+            stacks.append((api.ExpertStack.from_qweight(g, E), api.ExpertStack.from_qweight(u, E),
+                           api.ExpertStack.from_qweight(d, E)))
+        a = wl.gen_x(T, dm, case.seed + 3).to(dev).reshape(-1)
+        ids = wl.gen_moe_ids(T, E, k, case.seed + 4)
+        n_dist = len(np.unique(ids.numpy()))
+        ids = ids.to(dev)
+        h = torch.empty(T * k, dff, dtype=torch.bfloat16, device=dev)
+        o = torch.empty(T * k, dm, dtype=torch.bfloat16, device=dev)
+        it = [0]
+
+        def gu():
+            g, u, _ = stacks[it[0] % n_sets]
+            it[0] += 1
+            api.qmm_moe_gemv_id_gate_up_silu_batched(a, ids, T, k, dm, 0, g, u, out=h, stream=stream)
+
+        def dn():
+            _, _, d = stacks[it[0] % n_sets]
+            it[0] += 1
+            api.qmm_moe_gemv_id(h.reshape(-1), ids.reshape(-1), T * k, dff, d, out=o, stream=stream)
+        t_gu = time_graph(torch, gu, stream, inner=n_sets)
+        t_dn = time_graph(torch, dn, stream, inner=n_sets)
+        b_gu = n_dist * 2 * (dff * dm // 2 + dff * (dm // 64) * 4) + 2 * T * dm + 2 * T * k * dff
+        b_dn = n_dist * (dm * dff // 2 + dm * (dff // 64) * 4) + 2 * T * k * dff + 2 * T * k * dm
+        out[f"moe_gate_up_silu_t{T}"] = {"GB/s": round(b_gu / (t_gu * 1e-3) / 1e9, 1),
+                                         "frac": round(b_gu / (t_gu * 1e-3) / 1e9 / hbm_peak, 3),
+                                         "us": round(t_gu * 1e3, 2), "distinct_experts": n_dist}
+        out[f"moe_down_t{T}"] = {"GB/s": round(b_dn / (t_dn * 1e-3) / 1e9, 1),
+                                 "frac": round(b_dn / (t_dn * 1e-3) / 1e9 / hbm_peak, 3),
+                                 "us": round(t_dn * 1e3, 2)}
+        del stacks
+    # prefill GEMM M=2048, 14336x4096 (when the tensor-core GEMM path is built)
+    try:
+        c = [p for p in wl.WORKLOADS.prefill if p.M == 2048 and p.N == 14336][0]
+        qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), 64, 4, torch.bfloat16)
+        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        if _has_tc_gemm():
+            t = time_graph(torch, lambda: api.qmm_matmul(x, qw, True, out=y, stream=stream), stream,
+                           reps=10, inner=5)
+            tf = 2 * c.M * c.N * c.K / (t * 1e-3) / 1e12
+            out["prefill_gemm_m2048_14336x4096"] = {"TFLOP/s": round(tf, 1),
+                                                    "frac_of_measured_burst": round(tf / bf16_peak, 3),
+                                                    "frac_of_2250_dense": round(tf / 2250.0, 3),
+                                                    "us": round(t * 1e3, 1)}
+    except Exception as e:  # pragma: no cover
+        out["prefill_error"] = str(e)[:200]
+    return out
+
+
+# the prefill line is timed once the tensor-core GEMM serves M > 16
+PREFILL_READY = False
+
+
+def _has_tc_gemm():
+    return PREFILL_READY
+
+
+# ---------------------------------------------------------------- oracle arms
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_decode_inputs(wl, oracle):
+    ins = []
+    for c in wl.WORKLOADS.decode:
+        w = wl.gen_weight(c.N, c.K, c.seed).numpy()
+        p, s, b = oracle.quantize(w, oracle.F32, c.group_size, c.bits, oracle.BF16)
+        x = wl.storage_numpy(wl.gen_x(c.M, c.K, c.seed + 1))
+        ins.append((c, p, s, b, x))
+    return ins
+
+
+def _oracle_step(oracle, ins, threads, frac):
+    """one sampled step: the first `frac` of the output rows of each decode call"""
+    nbytes = 0.0
+    for c, p, s, b, x in ins:
+        n = max(1, int(c.N * frac))
+        oracle.matmul(x, oracle.BF16, p[:n], s[:n], b[:n], oracle.BF16, n, c.group_size, c.bits,
+                      n_threads=threads)
+        nbytes += decode_bytes(c.M, c.N, c.K, c.bits, c.group_size) * n / c.N
+    return nbytes
+
+
+def cpu_baseline(wl, seconds):
+    import oracle
+    ins = _oracle_decode_inputs(wl, oracle)
+    threads = cpu_threads()
+    frac = 1.0
+    t0 = time.perf_counter()
+    nb = _oracle_step(oracle, ins, threads, 0.05)
+    dt = time.perf_counter() - t0
+    frac = min(1.0, max(0.01, 0.05 * (seconds / 3) / max(dt, 1e-3)))
+    total_b, t0 = 0.0, time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < seconds and reps < 1000:
+        total_b += _oracle_step(oracle, ins, threads, frac)
+        reps += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(total_b / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{reps} passes over the first {frac:.1%} of output rows of the 3 decode "
+                      f"GEMVs (M=1), fp64 oracle, {threads} threads, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from weight_only_quantized_qmm_b200 import workloads as wl
+    threads = cpu_threads()
+    ins = _oracle_decode_inputs(wl, oracle)
+    frac = 0.02  # bounded sample per step: 2% of the output rows
+    for _ in range(max(args.warmup, 3)):
+        _oracle_step(oracle, ins, threads, frac)
+    steps = args.steps if args.steps_given else 5
+    t0 = time.perf_counter()
+    total_b = 0.0
+    for _ in range(steps):
+        total_b += _oracle_step(oracle, ins, threads, frac)
+    dt = time.perf_counter() - t0
+    value = total_b / dt / 1e9
+    sample = (f"each step: first {frac:.0%} of the output rows of the 3 decode GEMVs (M=1), "
+              f"fp64 oracle on {threads} threads")
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": round(dt * 1e3 / steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, same bytes as the GPU arm)", "impl": "reference",
+        "config": {"workload": "decode GEMV M=1, 4-bit affine g64, bf16 x/scales/biases; "
+                               "N x K = 4096x4096 + 14336x4096 + 4096x14336 per step",
+                   "global_batch": 1, "M": 1, "bits": 4, "group_size": 64},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_profile(args):
+    """A few eager launches of one case, for ncu (no timing output)."""
+    import torch
+
+    from weight_only_quantized_qmm_b200 import api
+    from weight_only_quantized_qmm_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    name = args.profile
+    if name.startswith("decode"):
+        c = [d for d in wl.WORKLOADS.decode if d.name == name][0]
+        qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), c.group_size, c.bits,
+                              torch.bfloat16)
+        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+        fn = lambda: api.qmm_matmul(x, qw)  # noqa: E731
+    elif name.startswith("prefill"):
+        c = [d for d in wl.WORKLOADS.prefill if d.name == name][0]
+        qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), c.group_size, c.bits,
+                              torch.bfloat16)
+        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+        fn = lambda: api.qmm_matmul(x, qw)  # noqa: E731
+    elif name.startswith("moe"):
+        case = [d for d in wl.WORKLOADS.moe if d.name == name][0]
+        E, dff, dm, T, k = case.num_experts, case.d_ff, case.d_model, case.tokens, case.top_k
+        g = api.ExpertStack.from_qweight(api.qmm_quantize(wl.gen_weight(E * dff, dm, case.seed).to(dev), 64, 4, torch.bfloat16), E)
+        u = api.ExpertStack.from_qweight(api.qmm_quantize(wl.gen_weight(E * dff, dm, case.seed + 1).to(dev), 64, 4, torch.bfloat16), E)
+        a = wl.gen_x(T, dm, case.seed + 3).to(dev).reshape(-1)
+        ids = wl.gen_moe_ids(T, E, k, case.seed + 4).to(dev)
+        fn = lambda: api.qmm_moe_gemv_id_gate_up_silu_batched(a, ids, T, k, dm, 0, g, u)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    for _ in range(args.profile_launches):
+        fn()
+    torch.cuda.synchronize()
+    print(f"profiled {name}: {args.profile_launches} launches")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", default=None,
+                    help="run a few launches of one named case (e.g. decode_14336x4096) for ncu")
+    ap.add_argument("--profile-launches", type=int, default=3)
+    args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
+    args.steps_given = args.steps is not None
+    if args.steps is None:
+        args.steps = 20000
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

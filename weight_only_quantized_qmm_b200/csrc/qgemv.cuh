@@ -28,7 +28,10 @@ struct QgemvParams {
   int kchunk;          // groups staged per K chunk
   int tok_stride;      // bytes between token rows of staged x
   // shared memory carve-up (byte offsets)
-  int off_plan, off_xs, off_xsum, off_part;
+  int use_tma;         // 1: take the TMA path when the shape allows it
+  int sb_rows;         // rows of the staged scale/bias block
+  int sb_words;        // 4-byte words staged per row and array (covers kchunk + 1 elements)
+  int off_plan, off_ring, off_part, off_corr, off_xs, off_xsum, off_sb;
 };
 
 
@@ -56,6 +59,7 @@ inline QgemvParams make_dense_params(const void* x, int64_t M, int64_t K, const 
   p.out_dtype = y_dtype;
   p.out_ld = w->rows;
   p.d_status = nullptr;
+  p.use_tma = 1;
   return p;
 }
 
@@ -89,6 +93,7 @@ inline QgemvParams make_moe_params(const void* a, const int32_t* ids, int64_t n_
   p.out_dtype = out_dtype;
   p.out_ld = w0->n_rows;
   p.d_status = d_status;
+  p.use_tma = 1;
   return p;
 }
 

@@ -1,0 +1,18 @@
+// Instantiations of the decode GEMV / MoE kernel family for 6-bit codes.
+#include "qgemv_impl.cuh"
+
+namespace qmm {
+
+cudaError_t launch_qgemv_b6(const QgemvParams& prm, int gs, int dtype, int mt, bool dual,
+                            cudaStream_t st) {
+  if (dtype == QMM_BF16) {
+    if (gs == 32) return launch_mt<6, 32, __nv_bfloat16>(prm, mt, dual, st);
+    if (gs == 64) return launch_mt<6, 64, __nv_bfloat16>(prm, mt, dual, st);
+    return launch_mt<6, 128, __nv_bfloat16>(prm, mt, dual, st);
+  }
+  if (gs == 32) return launch_mt<6, 32, __half>(prm, mt, dual, st);
+  if (gs == 64) return launch_mt<6, 64, __half>(prm, mt, dual, st);
+  return launch_mt<6, 128, __half>(prm, mt, dual, st);
+}
+
+}  // namespace qmm
