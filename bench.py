@@ -272,30 +272,16 @@ def run_ours(args):
     ms_step = ms / steps
     value = step_bytes * steps * world / (ms * 1e-3) / 1e9
 
-    # per-shape launch durations (events around each launch inside one graph)
+    # per-shape launch durations: one graph per shape (rotating its weight
+    # copies), timed from outside, so no event sits between two kernels
     per_shape = {}
-    g2 = torch.cuda.CUDAGraph()
-    # external events: recorded as graph nodes, so each one is a GPU timestamp
-    evs = [[(torch.cuda.Event(enable_timing=True, external=True),
-             torch.cuda.Event(enable_timing=True, external=True))
-            for _ in cases] for _ in range(n_sets)]
-    with torch.cuda.graph(g2, stream=stream):
-        for s in range(n_sets):
-            for i, (c, qw, x, y) in enumerate(sets[s]):
-                evs[s][i][0].record(stream)
-                api.qmm_matmul(x, qw, True, out=y, stream=stream)
-                evs[s][i][1].record(stream)
-    durs = [[] for _ in cases]
-    for _ in range(20):
-        with torch.cuda.stream(stream):
-            g2.replay()
-        torch.cuda.synchronize()
-        for s in range(n_sets):
-            for i in range(len(cases)):
-                durs[i].append(evs[s][i][0].elapsed_time(evs[s][i][1]))
     tot_b, tot_ms = 0.0, 0.0
     for i, c in enumerate(cases):
-        d = statistics.median(durs[i])
+        def shape_fn(i=i):
+            for s in range(n_sets):
+                _, qw, x, y = sets[s][i]
+                api.qmm_matmul(x, qw, True, out=y, stream=stream)
+        d = time_graph(torch, shape_fn, stream, reps=10, inner=max(1, 48 // n_sets)) / n_sets
         b = decode_bytes(c.M, c.N, c.K, c.bits, c.group_size)
         per_shape[c.name] = {"us": round(d * 1e3, 3), "GB/s": round(b / (d * 1e-3) / 1e9, 1),
                              "frac": round(b / (d * 1e-3) / 1e9 / hbm_peak, 3)}
@@ -374,7 +360,7 @@ def run_ours(args):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, g2
+    del graph
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -467,7 +453,7 @@ def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
 
 
 # the prefill line is timed once the tensor-core GEMM serves M > 16
-PREFILL_READY = False
+PREFILL_READY = True
 
 
 def _has_tc_gemm():

@@ -14,6 +14,8 @@ cudaError_t launch_quantize(int w_dtype, int s_dtype, int bits, const void* w, i
 cudaError_t launch_dequantize(const qmm_qweight* w, void* out, int out_dtype, cudaStream_t st);
 cudaError_t launch_generic(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
                            int transpose, void* y, int y_dtype, cudaStream_t st);
+cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
+                            void* y, int y_dtype, cudaStream_t st);
 }  // namespace qmm
 
 #include "qgemv.cuh"
@@ -152,6 +154,10 @@ qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
     const cudaError_t e = qmm::launch_qgemv(p, w->bits, w->group_size, x_dtype, false, st);
     if (e == cudaErrorInvalidValue) return QMM_ERR_UNSUPPORTED;
     return launch_status(e);
+  }
+  if (transpose && half_types) {  // M > 16: tcgen05 tensor-core GEMM
+    const cudaError_t e = qmm::launch_qgemm_tc(x, x_dtype, M, K, w, y, y_dtype, st);
+    if (e != cudaErrorNotSupported) return launch_status(e);
   }
   return launch_status(qmm::launch_generic(x, x_dtype, M, K, w, transpose, y, y_dtype, st));
 }

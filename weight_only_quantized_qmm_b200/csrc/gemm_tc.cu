@@ -1,0 +1,472 @@
+// Prefill-shaped quantized matmul on the 5th-generation tensor cores:
+//   y[m, n] = sum_k x[m, k] * w_hat[n, k],  w_hat = q * s_g + b_g
+// ("emily 0.5.1 lib/emily/quantization.ex", quantized_matmul/2 with
+//  transpose = true), for bf16 or f16 activations with matching scales.
+//
+// One CTA computes a 128 (weight rows) x 256 (tokens) tile of y^T with
+// tcgen05.mma (kind::f16, M = 128, N = 256, K = 16 per instruction), fp32
+// accumulator in tensor memory (256 columns):
+//   warp 0      TMA producer: x tiles [256 tokens x 64 k] bf16, 128-byte
+//               swizzle, one mbarrier per pipeline stage (transaction bytes)
+//   warp 1      allocates TMEM, one elected thread issues the MMAs and
+//               commits each stage back to the producers
+//   warps 2..5  dequantize: each thread owns one weight row, reads its packed
+//               codes and the group's scale/bias from global memory (prefetched
+//               one stage ahead), forms w_hat in bf16x2/f16x2 exactly once
+//               ((OFF + q) - OFF is exact, then one fused q*s + b rounding) and
+//               writes it into the stage's A tile in the UMMA K-major 128-byte
+//               swizzled layout; then the same warps run the epilogue
+//               (tcgen05.ld -> shared-memory transpose -> coalesced stores).
+// Every mbarrier wait is bounded; on a timeout the tile is written as NaN.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace qmm {
+
+namespace gemm {
+constexpr int kBM = 128;                 // weight rows per CTA (UMMA M)
+constexpr int kBN = 256;                 // tokens per CTA (UMMA N)
+constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row of 16-bit values
+constexpr int kStages = 4;
+constexpr int kThreads = 192;            // 6 warps
+constexpr int kXStage = kBN * kBK * 2;   // 32 KB
+constexpr int kAStage = kBM * kBK * 2;   // 16 KB
+constexpr int kTileBytes = kStages * (kXStage + kAStage);
+constexpr int kSmem = 1024 + kTileBytes + 256;  // + alignment slack + barriers
+constexpr uint32_t kSpins = 1u << 22;
+}  // namespace gemm
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t su32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bar_init(uint32_t b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(n));
+}
+__device__ __forceinline__ void bar_arrive(uint32_t b) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
+}
+__device__ __forceinline__ void bar_expect(uint32_t b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(b),
+               "r"(bytes)
+               : "memory");
+}
+// Bounded wait on an mbarrier phase.  Gives up (returns false) after kSpins
+// polls, or as soon as another role of the CTA has raised the abort flag.
+__device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity, const int* abort_flag) {
+  for (uint32_t i = 0; i < gemm::kSpins; ++i) {
+    if ((i & 1023u) == 1023u && *reinterpret_cast<const volatile int*>(abort_flag)) return false;
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(b), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* m, int c0, int c1,
+                                       uint32_t b) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(m), "r"(c0), "r"(c1), "r"(b)
+      : "memory");
+}
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;             // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024u >> 4) << 32;   // stride byte offset
+  d |= (uint64_t)1u << 46;             // descriptor version (sm_100)
+  d |= (uint64_t)2u << 61;             // 128-byte swizzle
+  return d;
+}
+// instruction descriptor: fp32 accumulator, A/B = bf16 (1) or f16 (0), both K-major
+template <typename T>
+__device__ __forceinline__ uint32_t mma_idesc() {
+  constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(gemm::kBN >> 3) << 17) |
+         ((uint32_t)(gemm::kBM >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// 16-bit float pair arithmetic on raw 32-bit registers
+template <typename T>
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if constexpr (std::is_same<T, __half>::value)
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <typename T>
+__device__ __forceinline__ uint32_t h2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  if constexpr (std::is_same<T, __half>::value)
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  else
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+
+struct GemmParams {
+  const uint32_t* packed;
+  const void* scales;
+  const void* biases;
+  void* y;
+  int y_dtype;
+  int M, N, K, G, wpr;
+};
+
+// ------------------------------------------------------------------ dequant helpers
+// packed words of 64 consecutive codes of one row (2*B words), zero past the row
+template <int B>
+__device__ __forceinline__ void load_codes(const uint32_t* row, int w0, int wpr, bool ok,
+                                           uint32_t (&w)[2 * B]) {
+  if constexpr (B == 4) {
+    if (ok && w0 + 8 <= wpr && ((reinterpret_cast<uintptr_t>(row + w0) & 15) == 0)) {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(row + w0));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(row + w0) + 1);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+      return;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 2 * B; ++i) w[i] = (ok && w0 + i < wpr) ? __ldg(row + w0 + i) : 0u;
+}
+
+// 64 codes -> 32 pairs of (OFF + q) as 16-bit floats (pair p = codes 2p, 2p+1)
+template <int B, typename T>
+__device__ __forceinline__ void codes_to_pairs(const uint32_t (&w)[2 * B], uint32_t (&pr)[32]) {
+  constexpr uint32_t M8 = std::is_same<T, __half>::value ? 0x64646464u : 0x43434343u;
+  if constexpr (B == 4) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t t0 = w[i] & 0x0F0F0F0Fu;         // codes 0,2,4,6 of the word
+      const uint32_t t1 = (w[i] >> 4) & 0x0F0F0F0Fu;  // codes 1,3,5,7
+      const uint32_t u = __byte_perm(t0, t1, 0x5140);  // c0 c1 c2 c3
+      const uint32_t v = __byte_perm(t0, t1, 0x7362);  // c4 c5 c6 c7
+      // f16 magic 0x6400 = 1024 needs the code in the low byte of the mantissa:
+      // both magics keep the code in the low byte and the magic in the high byte
+      pr[4 * i + 0] = __byte_perm(u, M8, 0x4140);
+      pr[4 * i + 1] = __byte_perm(u, M8, 0x4342);
+      pr[4 * i + 2] = __byte_perm(v, M8, 0x4140);
+      pr[4 * i + 3] = __byte_perm(v, M8, 0x4342);
+    }
+  } else {
+    constexpr uint32_t MG = std::is_same<T, __half>::value ? 0x64006400u : 0x43004300u;
+#pragma unroll
+    for (int p = 0; p < 32; ++p) {
+      const uint32_t c0 = stream_code<B>(w, 2 * p), c1 = stream_code<B>(w, 2 * p + 1);
+      pr[p] = c0 | (c1 << 16) | MG;
+    }
+  }
+}
+
+template <int B, int GS, typename T>
+__global__ void __launch_bounds__(gemm::kThreads, 1)
+qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
+  using namespace gemm;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* xs = smem;                                 // [kStages][256 x 128 B]
+  uint8_t* as = smem + kStages * kXStage;             // [kStages][128 x 128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTileBytes);
+  const uint32_t full0 = su32(bars), afull0 = full0 + 8 * kStages, empty0 = afull0 + 8 * kStages;
+  const uint32_t accf = empty0 + 8 * kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBM, m0 = blockIdx.y * kBN;
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      bar_init(full0 + 8 * s, 1);
+      bar_init(afull0 + 8 * s, 4);
+      bar_init(empty0 + 8 * s, 1);
+    }
+    bar_init(accf, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {  // 256 TMEM columns for the 128 x 256 fp32 accumulator
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(su32(tmem_slot)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % kStages, u = i / kStages;
+        if (i >= kStages && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) { *abort_flag = 1; break; }
+        bar_expect(full0 + 8 * s, kXStage);
+        tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, m0, full0 + 8 * s);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = mma_idesc<T>();
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % kStages, u = i / kStages;
+        if (!bar_wait(full0 + 8 * s, u & 1, abort_flag) || !bar_wait(afull0 + 8 * s, u & 1, abort_flag)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = su32(as + s * kAStage), b0 = su32(xs + s * kXStage);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_f16(tmem, sw128_desc(a0 + 32 * kk), sw128_desc(b0 + 32 * kk), idesc,
+                  (i | kk) != 0 ? 1u : 0u);
+        mma_commit(empty0 + 8 * s);  // frees the stage once these MMAs have read it
+      }
+      mma_commit(accf);  // accumulator complete
+    }
+  } else {
+    // ---------------- dequant (warps 2..5), then epilogue ----------------
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;  // weight row of the tile owned by this thread
+    const int n = n0 + r;
+    const bool nval = n < p.N;
+    const uint32_t* row = p.packed + (int64_t)(nval ? n : 0) * p.wpr;
+    const T* srow = reinterpret_cast<const T*>(p.scales) + (int64_t)(nval ? n : 0) * p.G;
+    const T* brow = reinterpret_cast<const T*>(p.biases) + (int64_t)(nval ? n : 0) * p.G;
+    constexpr int NGS = (kBK + GS - 1) / GS;  // groups touched by a stage (1 or 2)
+    constexpr uint32_t OFF2 = std::is_same<T, __half>::value ? 0x64006400u : 0x43004300u;
+    constexpr bool kF32Path = (B == 8) && !std::is_same<T, __half>::value;
+
+    // registers of the stage being converted (cw/cs/cb) and of the next one (nw/ns/nb)
+    uint32_t cw[2 * B], nw[2 * B];
+    T cs[NGS], cb[NGS], ns[NGS], nb[NGS];
+    auto load = [&](int i, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
+      const int k0 = i * kBK;
+      load_codes<B>(row, k0 * B / 32, p.wpr, nval && i < nk, w);
+#pragma unroll
+      for (int j = 0; j < NGS; ++j) {
+        const int gidx = (k0 + j * GS) / GS;
+        const bool ok = nval && i < nk && gidx < p.G;
+        sv[j] = ok ? srow[gidx] : from_f32<T>(0.0f);
+        bv[j] = ok ? brow[gidx] : from_f32<T>(0.0f);
+      }
+    };
+    load(0, nw, ns, nb);
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % kStages, u = i / kStages;
+#pragma unroll
+      for (int j = 0; j < 2 * B; ++j) cw[j] = nw[j];
+#pragma unroll
+      for (int j = 0; j < NGS; ++j) { cs[j] = ns[j]; cb[j] = nb[j]; }
+      load(i + 1, nw, ns, nb);  // prefetch the next stage while this one is converted
+      // the A buffer of this stage is free once its x tile has been refilled
+      if (!bar_wait(full0 + 8 * s, u & 1, abort_flag)) *abort_flag = 1;
+      uint32_t pr[32];
+      float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
+      if constexpr (kF32Path) {
+        sf0 = to_f32(cs[0]); bf0 = to_f32(cb[0]);
+        sf1 = to_f32(cs[NGS - 1]); bf1 = to_f32(cb[NGS - 1]);
+      } else {
+        codes_to_pairs<B, T>(cw, pr);
+      }
+      const uint32_t s2a = (uint32_t)bits16(cs[0]) * 0x00010001u;
+      const uint32_t b2a = (uint32_t)bits16(cb[0]) * 0x00010001u;
+      const uint32_t s2b = (uint32_t)bits16(cs[NGS - 1]) * 0x00010001u;
+      const uint32_t b2b = (uint32_t)bits16(cb[NGS - 1]) * 0x00010001u;
+      uint8_t* arow = as + s * kAStage + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = pairs 4c..4c+3 = codes 8c..8c+7
+        uint4 v;
+        uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int pi = 4 * c + e;
+          const bool second = NGS > 1 && (2 * pi) >= GS;
+          if constexpr (kF32Path) {
+            // 8-bit codes do not fit the bf16 magic: q exact in fp32, fmaf, one bf16 rounding
+            const float q0 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi)) - 8388608.0f;
+            const float q1 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi + 1)) - 8388608.0f;
+            const float sv = second ? sf1 : sf0, bv = second ? bf1 : bf0;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(q0, sv, bv), fmaf(q1, sv, bv));
+            vv[e] = *reinterpret_cast<const uint32_t*>(&h);
+          } else {
+            const uint32_t qv = h2_sub<T>(pr[pi], OFF2);  // exact q
+            vv[e] = h2_fma<T>(qv, second ? s2b : s2a, second ? b2b : b2a);
+          }
+        }
+        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = v;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) bar_arrive(afull0 + 8 * s);
+    }
+
+    // ---------------- epilogue: TMEM -> registers -> smem transpose -> y ----------------
+    const bool ok = bar_wait(accf, 0, abort_flag) && !*reinterpret_cast<volatile int*>(abort_flag);
+    tc_fence_after();
+    const bool f32out = p.y_dtype == QMM_F32;
+    // staging tile [256 tokens][128 rows] in the (now idle) pipeline buffers
+    uint8_t* stg = smem;
+    const int esz = f32out ? 4 : 2;
+    for (int c = 0; c < kBN / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int tok = c * 32 + j;
+        const float f = ok ? __uint_as_float(v[j]) : __int_as_float(0x7fc00000);
+        if (f32out)
+          *reinterpret_cast<float*>(stg + ((size_t)tok * kBM + r) * 4) = f;
+        else
+          *reinterpret_cast<T*>(stg + ((size_t)tok * kBM + r) * 2) = from_f32<T>(f);
+      }
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
+    // coalesced stores: 16 bytes per thread per step along each token row
+    const int row_bytes = kBM * esz;
+    const int chunks = kBN * row_bytes / 16;
+    const int et = threadIdx.x - 64;
+    for (int ci = et; ci < chunks; ci += 128) {
+      const int tok = ci / (row_bytes / 16);
+      const int col = (ci % (row_bytes / 16)) * (16 / esz);  // first weight row of the chunk
+      const int m = m0 + tok, nn = n0 + col;
+      if (m >= p.M || nn >= p.N) continue;
+      const uint8_t* src = stg + (size_t)tok * row_bytes + (size_t)col * esz;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.y) + ((int64_t)m * p.N + nn) * esz;
+      const int nvalid = min(16 / esz, p.N - nn);
+      if (nvalid == 16 / esz && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      } else {
+        for (int e = 0; e < nvalid * esz; ++e) dst[e] = src[e];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+  }
+}
+
+// ------------------------------------------------------------------ host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tensor_map_encoder();
+
+template <int B, int GS, typename T>
+static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, cudaStream_t st) {
+  auto k = qgemm_tc_kernel<B, GS, T>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  dim3 grid((prm.N + gemm::kBM - 1) / gemm::kBM, (prm.M + gemm::kBN - 1) / gemm::kBN);
+  k<<<grid, gemm::kThreads, gemm::kSmem, st>>>(prm, tmx);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const CUtensorMap& tmx,
+                                 cudaStream_t st) {
+#define QMM_G(BB)                                                             \
+  if (gs == 32) return launch_gemm_t<BB, 32, T>(prm, tmx, st);                \
+  if (gs == 64) return launch_gemm_t<BB, 64, T>(prm, tmx, st);                \
+  return launch_gemm_t<BB, 128, T>(prm, tmx, st);
+  switch (bits) {
+    case 2: { QMM_G(2) }
+    case 3: { QMM_G(3) }
+    case 4: { QMM_G(4) }
+    case 6: { QMM_G(6) }
+    default: { QMM_G(8) }
+  }
+#undef QMM_G
+}
+
+// cudaErrorNotSupported: the call does not fit this kernel (the caller falls back)
+cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
+                            void* y, int y_dtype, cudaStream_t st) {
+  if (M > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->rows > (int64_t)INT32_MAX)
+    return cudaErrorNotSupported;
+  if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tmx;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
+  const cuuint32_t box[2] = {gemm::kBK, gemm::kBN};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      x_dtype == QMM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (enc(&tmx, dt, 2, const_cast<void*>(x), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorNotSupported;
+  GemmParams prm;
+  prm.packed = w->packed;
+  prm.scales = w->scales;
+  prm.biases = w->biases;
+  prm.y = y;
+  prm.y_dtype = y_dtype;
+  prm.M = (int)M;
+  prm.N = (int)w->rows;
+  prm.K = (int)K;
+  prm.G = (int)(K / w->group_size);
+  prm.wpr = (int)(K * w->bits / 32);
+  if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16>(w->bits, w->group_size, prm, tmx, st);
+  return launch_gemm_b<__half>(w->bits, w->group_size, prm, tmx, st);
+}
+
+}  // namespace qmm

@@ -39,8 +39,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait on a phase of an mbarrier: gives up after kMbarSpins polls
 // (each try_wait may suspend the thread for a while) and returns false.
 constexpr uint32_t kMbarSpins = 1u << 20;
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMbarSpins; ++i)
+// After a first failure the warp only polls briefly (`failed`), so a broken
+// copy cannot stretch the kernel by one full timeout per remaining stage.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool failed) {
+  const uint32_t spins = failed ? 1024u : kMbarSpins;
+  for (uint32_t i = 0; i < spins; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
@@ -260,7 +263,7 @@ qgemv_tma_kernel(const QgemvParams p, const __grid_constant__ CUtensorMap tm0,
             const uint32_t k = (used + (uint32_t)st) % STAGES;
             const uint32_t parity = ((used + (uint32_t)st) / STAGES) & 1u;
             // every issued stage is waited on (bounded), so nothing is in flight at exit
-            if (!mbar_wait(bar_base + 8 * k, parity) && !failed) {
+            if (!mbar_wait(bar_base + 8 * k, parity, failed) && !failed) {
               failed = true;
               if (lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
             }
