@@ -154,13 +154,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, v: float) -> float:
+    """The slowest rank's time (the job's time): one all-reduce(MAX)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(bytes_per_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the max-over-ranks time."""
+    return bytes_per_step * steps * world / (ms_max * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------- traffic record
@@ -270,7 +277,7 @@ def run_ours(args):
     ms = ev0.elapsed_time(ev1)
     ms = max_over_ranks(world, ms)
     ms_step = ms / steps
-    value = step_bytes * steps * world / (ms * 1e-3) / 1e9
+    value = job_throughput(step_bytes, steps, world, ms)
 
     # per-shape launch durations: one graph per shape (rotating its weight
     # copies), timed from outside, so no event sits between two kernels
