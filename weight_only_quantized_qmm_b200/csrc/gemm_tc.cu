@@ -12,7 +12,7 @@
 //               commits each stage back to the producers
 //   warps 2..5  dequantize: each thread owns one weight row, reads its packed
 //               codes and the group's scale/bias from global memory (prefetched
-//               one stage ahead), forms w_hat in bf16x2/f16x2 exactly once
+//               three stages ahead), forms w_hat in bf16x2/f16x2 exactly once
 //               ((OFF + q) - OFF is exact, then one fused q*s + b rounding) and
 //               writes it into the stage's A tile in the UMMA K-major 128-byte
 //               swizzled layout; then the same warps run the epilogue
@@ -280,9 +280,11 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     constexpr uint32_t OFF2 = std::is_same<T, __half>::value ? 0x64006400u : 0x43004300u;
     constexpr bool kF32Path = (B == 8) && !std::is_same<T, __half>::value;
 
-    // registers of the stage being converted (cw/cs/cb) and of the next one (nw/ns/nb)
-    uint32_t cw[2 * B], nw[2 * B];
-    T cs[NGS], cb[NGS], ns[NGS], nb[NGS];
+    // codes and scales/biases are prefetched kAhead stages ahead into a register
+    // ring (compile-time indices: the stage loop is unrolled by kAhead)
+    constexpr int kAhead = 3;
+    uint32_t rw[kAhead][2 * B];
+    T rs[kAhead][NGS], rb[kAhead][NGS];
     auto load = [&](int i, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
       const int k0 = i * kBK;
       load_codes<B>(row, k0 * B / 32, p.wpr, nval && i < nk, w);
@@ -294,16 +296,23 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
         bv[j] = ok ? brow[gidx] : from_f32<T>(0.0f);
       }
     };
-    load(0, nw, ns, nb);
-    for (int i = 0; i < nk; ++i) {
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a) load(a, rw[a], rs[a], rb[a]);
+    for (int i0 = 0; i0 < nk; i0 += kAhead) {
+#pragma unroll
+    for (int a = 0; a < kAhead; ++a) {
+      const int i = i0 + a;
+      if (i >= nk) break;
       const int s = i % kStages, u = i / kStages;
+      uint32_t cw[2 * B];
+      T cs[NGS], cb[NGS];
 #pragma unroll
-      for (int j = 0; j < 2 * B; ++j) cw[j] = nw[j];
+      for (int j = 0; j < 2 * B; ++j) cw[j] = rw[a][j];
 #pragma unroll
-      for (int j = 0; j < NGS; ++j) { cs[j] = ns[j]; cb[j] = nb[j]; }
-      load(i + 1, nw, ns, nb);  // prefetch the next stage while this one is converted
-      // the A buffer of this stage is free once its x tile has been refilled
-      if (!bar_wait(full0 + 8 * s, u & 1, abort_flag)) *abort_flag = 1;
+      for (int j = 0; j < NGS; ++j) { cs[j] = rs[a][j]; cb[j] = rb[a][j]; }
+      load(i + kAhead, rw[a], rs[a], rb[a]);  // refill this ring slot kAhead stages ahead
+      // the A buffer of this stage is free once the MMAs of stage i - kStages are done
+      if (u > 0 && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) *abort_flag = 1;
       uint32_t pr[32];
       float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
       if constexpr (kF32Path) {
@@ -342,6 +351,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
       __syncwarp();
       if (lane == 0) bar_arrive(afull0 + 8 * s);
+    }
     }
 
     // ---------------- epilogue: TMEM -> registers -> smem transpose -> y ----------------

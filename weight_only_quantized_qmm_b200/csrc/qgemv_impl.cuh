@@ -235,15 +235,16 @@ __device__ __forceinline__ int64_t pair_offset(const QgemvParams& p, int pair) {
 __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int* s_start,
                                            int* s_fill, int* s_dist, int* s_list, int* s_nd) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nthr = blockDim.x;
   const int E = p.num_experts;
   if (p.ids == nullptr) {
-    for (int i = tid; i < p.n_pairs; i += kThreads) s_list[i] = i;
+    for (int i = tid; i < p.n_pairs; i += nthr) s_list[i] = i;
     if (tid == 0) { s_cnt[0] = p.n_pairs; s_start[0] = 0; s_dist[0] = 0; *s_nd = 1; }
     __syncthreads();
   } else {
-    for (int e = tid; e < E; e += kThreads) { s_cnt[e] = 0; s_fill[e] = 0; }
+    for (int e = tid; e < E; e += nthr) { s_cnt[e] = 0; s_fill[e] = 0; }
     __syncthreads();
-    for (int i = tid; i < p.n_pairs; i += kThreads) {
+    for (int i = tid; i < p.n_pairs; i += nthr) {
       const int e = p.ids[i];
       if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
     }
@@ -270,7 +271,7 @@ __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int
       if (lane == 0) *s_nd = nd;
     }
     __syncthreads();
-    for (int i = tid; i < p.n_pairs; i += kThreads) {
+    for (int i = tid; i < p.n_pairs; i += nthr) {
       const int e = p.ids[i];
       if (e >= 0 && e < E) {
         s_list[s_start[e] + atomicAdd(&s_fill[e], 1)] = i;
@@ -293,9 +294,9 @@ template <class S, typename T, int TOKP, bool SEP_S>
 __device__ __forceinline__ void stage_x(const QgemvParams& p, const int* pairs, int ntok, int gc0,
                                         int gcn, T* xs, uint2* xrec) {
   constexpr int GS = S::kCodes * 4;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, nthr = blockDim.x;
   const int nblk = ntok * gcn * 4;
-  for (int base = 0; base < nblk; base += kThreads) {
+  for (int base = 0; base < nblk; base += nthr) {
     const int idx = base + tid;
     const bool act = idx < nblk;
     float sc = 0.0f, sb = 0.0f;
@@ -352,7 +353,8 @@ template <int TOKP, int NS, bool DUAL>
 __device__ __forceinline__ void reduce_store(const QgemvParams& p, const float* part, int tiles,
                                              int KS, int ntok, int64_t blk_row0, int64_t r1,
                                              const int* pairs) {
-  for (int it = threadIdx.x; it < tiles * 16 * ntok; it += kThreads) {
+  const int nthr = blockDim.x;
+  for (int it = threadIdx.x; it < tiles * 16 * ntok; it += nthr) {
     const int tl = it / (16 * ntok);
     const int rr = (it / ntok) % 16;
     const int tk = it % ntok;
@@ -368,6 +370,46 @@ __device__ __forceinline__ void reduce_store(const QgemvParams& p, const float* 
     if (DUAL) yv = y0 / (1.0f + expf(-y0)) * y1;
     store_as(p.out, p.out_dtype, (int64_t)pairs[tk] * p.out_ld + row, yv);
   }
+}
+
+// Tensor-core partial dot of one group for 16 rows x TOKP tokens: d = sum over
+// the group's k-slots of (OFF + v) * x'.  Even and odd k16 steps accumulate
+// into separate registers so consecutive mmas do not wait on each other.
+template <int BITS, class S, typename T, int MT>
+__device__ __forceinline__ void group_dot(const uint32_t (&rawA)[S::kRegs],
+                                          const uint32_t (&rawB)[S::kRegs],
+                                          const uint32_t (&xb)[MT], uint32_t xo,
+                                          float (&d)[MT][4]) {
+  float e[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { d[mt][i] = 0.0f; e[mt][i] = 0.0f; }
+#pragma unroll
+  for (int q2 = 0; q2 < S::kSteps / 2; ++q2) {
+    uint4 bf[MT];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) bf[mt] = lds128(xb[mt] + xo + q2 * 16);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int q = 2 * q2 + h2;
+      const uint32_t a0 = share_pair<BITS, S>(rawA, 2 * q);
+      const uint32_t a1 = share_pair<BITS, S>(rawB, 2 * q);
+      const uint32_t a2 = share_pair<BITS, S>(rawA, 2 * q + 1);
+      const uint32_t a3 = share_pair<BITS, S>(rawB, 2 * q + 1);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        if (h2 == 0)
+          mma16816<T>(d[mt], a0, a1, a2, a3, bf[mt].x, bf[mt].y);
+        else
+          mma16816<T>(e[mt], a0, a1, a2, a3, bf[mt].z, bf[mt].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[mt][i] += e[mt][i];
 }
 
 // ------------------------------------------------------------------ kernel
@@ -599,28 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) qgemv_kernel(const QgemvParams p)
                   read_share<S>(slot + (uint32_t)((((u * NS + s) * 2 + 0) * 32) * C::SLOT * 4), t, rawA);
                   read_share<S>(slot + (uint32_t)((((u * NS + s) * 2 + 1) * 32) * C::SLOT * 4), t, rawB);
                   float d[MT][4];
-#pragma unroll
-                  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) d[mt][i] = 0.0f;
-#pragma unroll
-                  for (int q2 = 0; q2 < S::kSteps / 2; ++q2) {
-                    uint4 bf[MT];
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt) bf[mt] = lds128(xb_sa[mt] + xo + q2 * 16);
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                      const int q = 2 * q2 + h2;
-                      const uint32_t a0 = share_pair<BITS, S>(rawA, 2 * q);
-                      const uint32_t a1 = share_pair<BITS, S>(rawB, 2 * q);
-                      const uint32_t a2 = share_pair<BITS, S>(rawA, 2 * q + 1);
-                      const uint32_t a3 = share_pair<BITS, S>(rawB, 2 * q + 1);
-#pragma unroll
-                      for (int mt = 0; mt < MT; ++mt)
-                        mma16816<T>(d[mt], a0, a1, a2, a3, h2 ? bf[mt].z : bf[mt].x,
-                                    h2 ? bf[mt].w : bf[mt].y);
-                    }
-                  }
+                  group_dot<BITS, S, T, MT>(rawA, rawB, xb_sa, xo, d);
                   // y += s_g * d
                   const uint32_t sq = sbq + (uint32_t)(s * 4 * SBW * 4);
                   const float s0 = half_bits_to_f32<T>(lds16(sq + (uint32_t)((par0 + u) * 2)));
