@@ -357,7 +357,7 @@ def run_ours(args):
                    "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                     "peak_source": peak_src, "kernel": "qgemv_kernel<4,64,bf16,1,false>",
+                     "peak_source": peak_src, "kernel": "qgemv_stream_kernel<4,64,bf16,1>",
                      "per_shape": per_shape},
         "e2e": e2e,
         "gpu_launches": steps * launches_per_step,

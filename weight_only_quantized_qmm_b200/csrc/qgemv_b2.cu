@@ -1,5 +1,5 @@
 // Instantiations of the decode GEMV / MoE kernel family for 2-bit codes.
-#include "qgemv_tma.cuh"
+#include "qgemv_stream.cuh"
 
 namespace qmm {
 
@@ -34,6 +34,8 @@ static cudaError_t try_tma(const QgemvParams& prm, int gs, int dtype, int mt, bo
 cudaError_t launch_qgemv_b2(const QgemvParams& prm, int gs, int dtype, int mt, bool dual,
                             cudaStream_t st) {
   if (prm.use_tma) {
+    const cudaError_t es = stream::try_stream<2>(prm, gs, dtype, mt, dual, st);
+    if (es != cudaErrorNotSupported) return es;
     const cudaError_t e = try_tma(prm, gs, dtype, mt, dual, st);
     if (e != cudaErrorNotSupported) return e;
   }

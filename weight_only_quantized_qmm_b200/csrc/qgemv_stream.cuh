@@ -1,0 +1,617 @@
+// Streaming decode GEMV for the dense case y = x . dequant(W)^T with a few
+// tokens (M <= 16): the bandwidth-bound half of the weight-only quantized
+// matmul ("Quantized matmul" / affine mode, w = q * scale + bias per group).
+//
+// One persistent CTA per SM owns a contiguous range of 16-row tiles of W and
+// streams each tile through shared memory as units of GPU groups (all 16
+// rows).  A unit arrives with three TMA copies counted on the slot's `full`
+// mbarrier: the packed codes as one 3-D box (16 rows x Z slices of 128 bytes,
+// 128-byte swizzle; few large copies keep the copy engine off the critical
+// path), the unit's scales and its biases (16 rows x GPU 16-bit values each).
+// Warp roles:
+//   * producer (1 warp, one lane) issues the copies, slot by slot;
+//   * consumers (kC warps) all read every unit, consumer w taking groups
+//     [w * GPW, (w + 1) * GPW).  Per group a consumer turns codes into 16-bit
+//     floats (OFF + q, exact), takes the partial dot with x on the tensor
+//     cores (mma.m16n8k16; rows of W as m, tokens as n), and folds it into
+//     fp32 accumulators as
+//       y += s * d + (b - OFF * s) * X,   X = sum of x over the group,
+//     which is sum_k x_k (q_k s + b) rewritten per group.  The slot is free
+//     again once all kC consumers arrived on its `empty` mbarrier;
+//   * epilogue (1 warp): when every consumer posted its partial for a tile
+//     (mbarrier `pfull`), sums them in consumer order (the result does not
+//     depend on timing) and stores the tile's outputs.
+// x is staged once per CTA in the tensor-core k order with its per-group sums.
+// Every wait is bounded: a timeout sets QMM_ERR_TIMEOUT, skips the remaining
+// arithmetic and still drains the copies in flight before the CTA exits.
+//
+// Launched with programmatic stream serialization: the producer streams
+// weights (which no earlier kernel writes) before griddepcontrol.wait, so a
+// call's weight traffic can start while the previous kernel drains; x and y
+// are only touched after the wait.
+#pragma once
+
+#include <cuda.h>
+
+#include "qgemv_tma.cuh"
+
+namespace qmm {
+namespace stream {
+
+constexpr int kRB = 2;          // partial-sum ring entries (tiles)
+constexpr int kMaxStages = 8;
+
+struct Params {
+  const void* x;        // [M, K] activations (row stride K)
+  int M;                // tokens, 1..16
+  int64_t K;
+  int G;                // groups per row
+  int upt;              // units per tile (ceil(G / GPU))
+  int64_t N;            // rows of W
+  int ntiles;           // ceil(N / 16)
+  void* out;            // [M, N]
+  int out_dtype;
+  int64_t out_ld;
+  int32_t* d_status;
+  int tok_stride;       // bytes between staged token rows of x
+  int stages;           // ring depth
+  int off_code, off_sb, off_bar, off_part, off_xs, off_xsum;
+};
+
+// MODE 0: one token; 1: up to 8 tokens; 2: up to 16 tokens.
+template <int BITS, int GS, typename T, int MODE>
+struct Cfg {
+  using S = Share<BITS, GS, T>;
+  static constexpr int MT = MODE == 2 ? 2 : 1;
+  static constexpr bool ONE = MODE == 0;
+  static constexpr int KC = MT == 1 ? 16 : 8;                     // consumer warps
+  static constexpr int THREADS = (KC + 2) * 32;
+  static constexpr int STAGERS = (KC + 1) * 32;                   // consumers + epilogue
+  static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
+  static constexpr int WPG = S::kWordsPerGroup;                   // words per group per row
+  static constexpr int GPU = WPG >= 32 ? 16 : 32;                 // groups per unit
+  static constexpr int GPW = GPU / KC;                            // groups per consumer per unit
+  static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
+  static constexpr int CODE_BYTES = Z * 16 * 128;
+  static constexpr int SB_BYTES = 16 * GPU * 2;                   // scales (or biases) of a unit
+  static constexpr uint32_t TX = CODE_BYTES + 2 * SB_BYTES;
+  static constexpr int TOKP = 8 * MT;
+  static constexpr int XG = 4 * S::kVirt * (int)sizeof(T);        // staged x bytes per group
+  static constexpr int NX = S::kSplit ? 2 : 1;                    // per-group sums kept
+  static_assert(S::kFast, "integral-lane codes only");
+  static_assert(GPW >= 1 && GPW * KC == GPU, "whole groups per consumer");
+  static_assert(Z >= 1 && Z <= 256, "box depth");
+};
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// d = sum over the k16 steps of (OFF + v) * x' for 16 rows x 8 columns; the
+// first step starts from a zero accumulator.
+template <typename T>
+__device__ __forceinline__ void mma_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  const float z = 0.0f;
+  if constexpr (std::is_same<T, __half>::value) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+  }
+}
+
+template <int BITS, class S, typename T, int MT>
+__device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], const uint32_t (&rawB)[S::kRegs],
+                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4]) {
+#pragma unroll
+  for (int q2 = 0; q2 < S::kSteps / 2; ++q2) {
+    uint4 bf[MT];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) bf[mt] = lds128(xb[mt] + xo + q2 * 16);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int q = 2 * q2 + h2;
+      const uint32_t a0 = share_pair<BITS, S>(rawA, 2 * q);
+      const uint32_t a1 = share_pair<BITS, S>(rawB, 2 * q);
+      const uint32_t a2 = share_pair<BITS, S>(rawA, 2 * q + 1);
+      const uint32_t a3 = share_pair<BITS, S>(rawB, 2 * q + 1);
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t b0 = h2 ? bf[mt].z : bf[mt].x, b1 = h2 ? bf[mt].w : bf[mt].y;
+        if (q == 0)
+          mma_first<T>(d[mt], a0, a1, a2, a3, b0, b1);
+        else
+          mma16816<T>(d[mt], a0, a1, a2, a3, b0, b1);
+      }
+    }
+  }
+}
+
+// both 16-bit halves of a word as floats
+template <typename T>
+__device__ __forceinline__ float2 halves_to_f32(uint32_t v) {
+  if constexpr (std::is_same<T, __half>::value) {
+    __half2 h;
+    memcpy(&h, &v, 4);
+    return __half22float2(h);
+  } else {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+  }
+}
+template <typename T>
+__device__ __forceinline__ float half_to_f32(uint32_t v, int hi) {
+  if constexpr (std::is_same<T, __half>::value) {
+    const float2 f = halves_to_f32<T>(v);
+    return hi ? f.y : f.x;
+  } else {
+    return __uint_as_float(hi ? (v & 0xffff0000u) : (v << 16));
+  }
+}
+
+// Stage x for tokens [0, M) and groups [0, Gpad): per (token, group, quarter t)
+// the kVirt values of quarter t in slot order (the codes' mma k order), zero
+// past G; per (group, token) the fp32 sum of x over the group (and, for the
+// two-nibble 8-bit form, the sum of the slot values x').
+template <class S, typename T, int TOKP, int NX, int NTHR>
+__device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint8_t* xs, float* xsum) {
+  constexpr int GS = S::kCodes * 4;
+  const int ntask = p.M * Gpad * 4;
+  for (int base = 0; base < ntask; base += NTHR) {
+    const int idx = base + sid;
+    const bool act = idx < ntask;
+    const int tt = idx & 3, gq = idx >> 2;
+    const int m = act ? gq / Gpad : 0, gl = act ? gq - m * Gpad : 0;
+    float sb = 0.0f, so = 0.0f;
+    if (act) {
+      __align__(16) T xv[S::kCodes];
+      if (gl < p.G) {
+        const T* xa = reinterpret_cast<const T*>(p.x) + (int64_t)m * p.K + (int64_t)gl * GS + tt * S::kCodes;
+        if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
+#pragma unroll
+          for (int c = 0; c < S::kCodes * (int)sizeof(T) / 16; ++c)
+            reinterpret_cast<uint4*>(xv)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
+        } else {
+#pragma unroll
+          for (int c = 0; c < S::kCodes; ++c) xv[c] = xa[c];
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < S::kCodes * (int)sizeof(T) / 16; ++c)
+          reinterpret_cast<uint4*>(xv)[c] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __align__(16) T outv[S::kVirt];
+#pragma unroll
+      for (int q = 0; q < S::kVirt; ++q) {
+        const int vv = S::slot_virtual(q);
+        const float mult = S::virt_mult(vv);
+        const float xf = to_f32(xv[S::virt_code(vv)]) * mult;
+        outv[q] = from_f32<T>(xf);
+        so += xf;
+        if (mult == 1.0f) sb += xf;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)m * p.tok_stride +
+                                            (size_t)(gl * 4 + tt) * S::kVirt * sizeof(T));
+#pragma unroll
+      for (int q = 0; q < (int)(S::kVirt * sizeof(T) / 16); ++q)
+        dst[q] = reinterpret_cast<const uint4*>(outv)[q];
+    }
+    sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+    so += __shfl_xor_sync(0xffffffffu, so, 1);
+    sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+    so += __shfl_xor_sync(0xffffffffu, so, 2);
+    if (act && tt == 0) {
+      xsum[gl * TOKP + m] = sb;
+      if constexpr (NX == 2) xsum[(Gpad + gl) * TOKP + m] = so;
+    }
+  }
+  // padding tokens [M, TOKP) of the sums read as zero
+  for (int idx = sid; idx < Gpad * TOKP * NX; idx += NTHR)
+    if (idx % TOKP >= p.M) xsum[idx] = 0.0f;
+}
+
+template <int BITS, int GS, typename T, int MODE>
+__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE>::THREADS, 1)
+qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
+                    const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmb) {
+  using C = Cfg<BITS, GS, T, MODE>;
+  using S = typename C::S;
+  constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC;
+  constexpr float OFF = S::kOff;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int STAGES = p.stages;
+  const uint32_t code_ring = smem_u32(smem + p.off_code);
+  const uint32_t sb_ring = smem_u32(smem + p.off_sb);
+  const uint32_t bar_full = smem_u32(smem + p.off_bar);
+  const uint32_t bar_empty = bar_full + 8 * kMaxStages;
+  const uint32_t bar_pfull = bar_empty + 8 * kMaxStages;
+  const uint32_t bar_pempty = bar_pfull + 8 * kRB;
+  float4* part = reinterpret_cast<float4*>(smem + p.off_part);
+  uint8_t* xs = smem + p.off_xs;
+  float* xsum = reinterpret_cast<float*>(smem + p.off_xsum);
+
+  const int tb = (int)((int64_t)p.ntiles * blockIdx.x / gridDim.x);
+  const int te = (int)((int64_t)p.ntiles * (blockIdx.x + 1) / gridDim.x);
+  const int nt = te - tb;
+  const int nunits = nt * p.upt;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, KC);
+    }
+    for (int e = 0; e < kRB; ++e) {
+      mbar_init(bar_pfull + 8 * e, KC);
+      mbar_init(bar_pempty + 8 * e, 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // the next kernel in the stream may launch now; it waits for this grid's
+  // completion before it reads anything this grid writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---------------------------------------------------------------- producer
+  if (warp == C::PRODUCER) {
+    if (lane == 0) {
+      bool failed = false;
+      int tile = tb, ku = 0, issued = 0;
+      for (int i = 0; i < nunits; ++i) {
+        const int slot = i % STAGES;
+        if (i >= STAGES && !mbar_wait(bar_empty + 8 * slot, (uint32_t)((i / STAGES) - 1) & 1u, false)) {
+          failed = true;
+          set_status(p.d_status, QMM_ERR_TIMEOUT);
+          break;
+        }
+        const uint32_t fb = bar_full + 8 * slot;
+        mbar_arrive_expect_tx(fb, C::TX);
+        tma_load_3d(code_ring + (uint32_t)(slot * C::CODE_BYTES), &tmc, 0, tile * 16, ku * C::Z, fb);
+        const uint32_t sd = sb_ring + (uint32_t)(slot * 2 * C::SB_BYTES);
+        tma_load_2d(sd, &tms, ku * GPU, tile * 16, fb);
+        tma_load_2d(sd + C::SB_BYTES, &tmb, ku * GPU, tile * 16, fb);
+        issued = i + 1;
+        if (++ku == p.upt) { ku = 0; ++tile; }
+      }
+      // no copy may still be landing when the CTA exits
+      for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
+        if (!mbar_wait(bar_full + 8 * (i % STAGES), (uint32_t)(i / STAGES) & 1u, failed)) failed = true;
+    }
+    return;
+  }
+
+  // --------------------------------------------------- x staging (after the wait)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int Gpad = p.upt * GPU;
+  stage_x<S, T, TOKP, C::NX, C::STAGERS>(p, Gpad, warp < KC ? tid : tid - 32, xs, xsum);
+  asm volatile("bar.sync 1, %0;" ::"n"(C::STAGERS) : "memory");
+
+  // ---------------------------------------------------------------- epilogue
+  if (warp == C::EPILOGUE) {
+    bool failed = false;
+    for (int jt = 0; jt < nt; ++jt) {
+      const int e = jt % kRB;
+      const bool ok = mbar_wait(bar_pfull + 8 * e, (uint32_t)(jt / kRB) & 1u, failed);
+      if (__any_sync(0xffffffffu, !ok)) {
+        if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+        failed = true;
+      }
+      if (!failed) {
+        for (int idx = lane; idx < 16 * p.M; idx += 32) {
+          const int r = idx & 15, m = idx >> 4;
+          const int mt = m >> 3, col = m & 7;
+          const int src = ((r & 7) << 2) | (col >> 1);
+          const int ci = ((r >> 3) << 1) | (col & 1);
+          float y = 0.0f;
+#pragma unroll
+          for (int w = 0; w < KC; ++w) {
+            const float4 v = part[((e * KC + w) * MT + mt) * 32 + src];
+            y += ci == 0 ? v.x : ci == 1 ? v.y : ci == 2 ? v.z : v.w;
+          }
+          const int64_t row = (int64_t)(tb + jt) * 16 + r;
+          if (row < p.N) store_as(p.out, p.out_dtype, (int64_t)m * p.out_ld + row, y);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pempty + 8 * e);
+    }
+    return;
+  }
+
+  // --------------------------------------------------------------- consumers
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t xs_sa = smem_u32(xs), xsum_sa = smem_u32(xsum);
+  // this warp's groups of a unit: ug = warp * GPW + u
+  uint32_t xb[MT];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int tr = (mt * 8 + g) < p.M ? mt * 8 + g : 0;  // idle columns reread token 0
+    xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
+             (uint32_t)(warp * GPW * C::XG);
+  }
+  const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + 2 * t) * 4);
+  // shared offsets (within a slot) of this lane's code words, row g, per group u
+  uint32_t coff[GPW];
+#pragma unroll
+  for (int u = 0; u < GPW; ++u) {
+    const int ug = warp * GPW + u;
+    const int w0 = ug * WPG + t * S::kRegs;  // first word in the unit row
+    const int wb = w0 & 31;
+    coff[u] = (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
+  }
+  // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's groups
+  const uint32_t soff = (uint32_t)((g * GPU + warp * GPW) * 2);
+
+  float acc[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
+  bool failed = false;
+
+  for (int i = 0; i < nunits; ++i) {
+    const int jt = i / p.upt, ku = i - jt * p.upt;
+    const int slot = i % STAGES;
+    const bool ok = mbar_wait(bar_full + 8 * slot, (uint32_t)(i / STAGES) & 1u, failed);
+    if (__any_sync(0xffffffffu, !ok)) {
+      if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+      failed = true;
+    }
+    if (!failed) {
+      const uint32_t cslot = code_ring + (uint32_t)(slot * C::CODE_BYTES);
+      const uint32_t sslot = sb_ring + (uint32_t)(slot * 2 * C::SB_BYTES) + soff;
+      // GPW 16-bit scales (biases) of rows g and g + 8
+      uint32_t sv[2][(GPW + 1) / 2], bv[2][(GPW + 1) / 2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t ra = sslot + (uint32_t)(h * 8 * GPU * 2);
+        if constexpr (GPW == 1) {
+          sv[h][0] = lds16(ra);
+          bv[h][0] = lds16(ra + C::SB_BYTES);
+        } else if constexpr (GPW == 2) {
+          sv[h][0] = lds32(ra);
+          bv[h][0] = lds32(ra + C::SB_BYTES);
+        } else {
+#pragma unroll
+          for (int c = 0; c < GPW / 4; ++c) {
+            const uint2 s2 = lds64(ra + 8 * c), b2 = lds64(ra + C::SB_BYTES + 8 * c);
+            sv[h][2 * c] = s2.x; sv[h][2 * c + 1] = s2.y;
+            bv[h][2 * c] = b2.x; bv[h][2 * c + 1] = b2.y;
+          }
+        }
+      }
+      uint32_t xbu[MT];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt] + (uint32_t)(ku * GPU * C::XG);
+      const uint32_t su = xsum_lane + (uint32_t)(ku * GPU * TOKP * 4);
+#pragma unroll
+      for (int u = 0; u < GPW; ++u) {
+        uint32_t rA[S::kRegs], rB[S::kRegs];
+        const uint32_t ca = cslot + coff[u];
+        if constexpr (S::kRegs >= 4) {
+          const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
+#pragma unroll
+          for (int k = 0; k < S::kRegs / 4; ++k) {
+            const uint32_t ch = (uint32_t)(((c0 ^ (uint32_t)g) + k) ^ (uint32_t)g);
+            const uint4 va = lds128(cbase + (ch << 4)), vb = lds128(cbase + 1024 + (ch << 4));
+            rA[4 * k] = va.x; rA[4 * k + 1] = va.y; rA[4 * k + 2] = va.z; rA[4 * k + 3] = va.w;
+            rB[4 * k] = vb.x; rB[4 * k + 1] = vb.y; rB[4 * k + 2] = vb.z; rB[4 * k + 3] = vb.w;
+          }
+        } else if constexpr (S::kRegs == 2) {
+          const uint2 va = lds64(ca), vb = lds64(ca + 1024);
+          rA[0] = va.x; rA[1] = va.y; rB[0] = vb.x; rB[1] = vb.y;
+        } else {
+          rA[0] = lds32(ca);
+          rB[0] = lds32(ca + 1024);
+        }
+        float d[MT][4];
+        group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d);
+        const int hw = u & 1;
+        const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
+        const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          if constexpr (C::ONE) {
+            const float X0 = __uint_as_float(lds32(su + (uint32_t)(u * TOKP * 4) - (uint32_t)(8 * t)));
+            if constexpr (C::NX == 1) {
+              acc[0][0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], acc[0][0]));
+              acc[0][2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], acc[0][2]));
+            } else {
+              const float O0 = __uint_as_float(lds32(su + (uint32_t)((Gpad + u) * TOKP * 4) - (uint32_t)(8 * t)));
+              acc[0][0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], acc[0][0])));
+              acc[0][2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], acc[0][2])));
+            }
+          } else {
+            const uint2 xr = lds64(su + (uint32_t)((u * TOKP + mt * 8) * 4));
+            const float X0 = __uint_as_float(xr.x), X1 = __uint_as_float(xr.y);
+            if constexpr (C::NX == 1) {
+              const float ca_ = fmaf(-OFF, sa, ba), cb_ = fmaf(-OFF, sb_, bb);
+              acc[mt][0] = fmaf(ca_, X0, fmaf(sa, d[mt][0], acc[mt][0]));
+              acc[mt][1] = fmaf(ca_, X1, fmaf(sa, d[mt][1], acc[mt][1]));
+              acc[mt][2] = fmaf(cb_, X0, fmaf(sb_, d[mt][2], acc[mt][2]));
+              acc[mt][3] = fmaf(cb_, X1, fmaf(sb_, d[mt][3], acc[mt][3]));
+            } else {
+              // bias term on sum(x), offset term on sum(x') (x' = x and 16 x)
+              const uint2 xo = lds64(su + (uint32_t)(((Gpad + u) * TOKP + mt * 8) * 4));
+              const float O0 = __uint_as_float(xo.x), O1 = __uint_as_float(xo.y);
+              const float oa = -OFF * sa, ob = -OFF * sb_;
+              acc[mt][0] = fmaf(ba, X0, fmaf(oa, O0, fmaf(sa, d[mt][0], acc[mt][0])));
+              acc[mt][1] = fmaf(ba, X1, fmaf(oa, O1, fmaf(sa, d[mt][1], acc[mt][1])));
+              acc[mt][2] = fmaf(bb, X0, fmaf(ob, O0, fmaf(sb_, d[mt][2], acc[mt][2])));
+              acc[mt][3] = fmaf(bb, X1, fmaf(ob, O1, fmaf(sb_, d[mt][3], acc[mt][3])));
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+
+    if (ku == p.upt - 1) {  // tile done: post this warp's partial
+      const int e = jt % kRB;
+      if (jt >= kRB) {
+        const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / kRB) - 1) & 1u, failed);
+        if (__any_sync(0xffffffffu, !okp)) {
+          if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+          failed = true;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        part[((e * KC + warp) * MT + mt) * 32 + lane] = make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[mt][k] = 0.0f;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pfull + 8 * e);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+// 3-D map over packed words [rows, wpr] seen as (word in slice, row, slice of
+// 32 words): a box is 16 rows x z slices, each slice 16 x 128 bytes, swizzled.
+inline bool make_code_map3(CUtensorMap* map, const uint32_t* packed, int64_t rows, int64_t wpr, int z) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(wpr / 32)};
+  const cuuint64_t strides[2] = {(cuuint64_t)(wpr * 4), 128};
+  const cuuint32_t box[3] = {32, 16, (cuuint32_t)z};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(packed), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over a [rows, G] array of 16-bit scales or biases: 16-row x gpu boxes.
+inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G, int gpu) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)G * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)gpu, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Dense calls only (no ids, one matrix); cudaErrorNotSupported sends the caller
+// to the general kernels.
+template <int BITS, int GS, typename T, int MODE>
+cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
+  using C = Cfg<BITS, GS, T, MODE>;
+  if (q.ids || q.amode != 0 || q.n_pairs < 1 || q.n_pairs > C::TOKP) return cudaErrorNotSupported;
+  if (q.G % 8 != 0 || q.wpr % 32 != 0 || q.n_rows < 16 || q.G < C::GPU) return cudaErrorNotSupported;
+  if (((uintptr_t)q.packed[0] | (uintptr_t)q.scales[0] | (uintptr_t)q.biases[0]) & 15) return cudaErrorNotSupported;
+
+  Params p{};
+  p.x = q.a;
+  p.M = q.n_pairs;
+  p.K = q.K;
+  p.G = q.G;
+  p.upt = (q.G + C::GPU - 1) / C::GPU;
+  p.N = q.n_rows;
+  p.ntiles = (int)((q.n_rows + 15) / 16);
+  p.out = q.out;
+  p.out_dtype = q.out_dtype;
+  p.out_ld = q.out_ld;
+  p.d_status = q.d_status;
+  const int Gpad = p.upt * C::GPU;
+  p.tok_stride = Gpad * C::XG + 16;
+
+  // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums]
+  const size_t part = (size_t)kRB * C::KC * C::MT * 32 * 16;
+  const size_t xs = align128((size_t)p.M * p.tok_stride);
+  const size_t xsum = align128((size_t)Gpad * C::TOKP * 4 * C::NX);
+  const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
+  auto total = [&](int stages) {
+    return 1024 + (size_t)stages * C::CODE_BYTES + align128((size_t)stages * 2 * C::SB_BYTES) + align128(bars) +
+           part + xs + xsum;
+  };
+  // about 96 KB of weights in flight per SM
+  int stages = (int)((96 * 1024) / C::TX);
+  stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
+  while (stages > 2 && total(stages) > (size_t)kSmemMax) --stages;
+  if (total(stages) > (size_t)kSmemMax) return cudaErrorNotSupported;
+  p.stages = stages;
+  p.off_code = 0;
+  p.off_sb = stages * C::CODE_BYTES;
+  p.off_bar = p.off_sb + (int)align128((size_t)stages * 2 * C::SB_BYTES);
+  p.off_part = p.off_bar + (int)align128(bars);
+  p.off_xs = p.off_part + (int)part;
+  p.off_xsum = p.off_xs + (int)xs;
+  const size_t smem = total(stages);
+
+  CUtensorMap tmc, tms, tmb;
+  if (!make_code_map3(&tmc, q.packed[0], q.n_rows, q.wpr, C::Z) ||
+      !make_sb_map(&tms, q.scales[0], q.n_rows, q.G, C::GPU) || !make_sb_map(&tmb, q.biases[0], q.n_rows, q.G, C::GPU))
+    return cudaErrorNotSupported;
+
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE>;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax);
+    if (e != cudaSuccess) return e;
+    configured[dev] = 1;
+  }
+  const int grid = std::min(qmm_host::num_sms(), p.ntiles);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p, tmc, tms, tmb);
+}
+
+template <int BITS, int GS, typename T>
+cudaError_t try_stream_mt(const QgemvParams& q, int mt, cudaStream_t st) {
+  if constexpr (Share<BITS, GS, T>::kFast) {
+    if (q.n_pairs == 1) return launch_stream<BITS, GS, T, 0>(q, st);
+    return mt == 1 ? launch_stream<BITS, GS, T, 1>(q, st) : launch_stream<BITS, GS, T, 2>(q, st);
+  } else {
+    return cudaErrorNotSupported;
+  }
+}
+
+// Entry from the per-bit-width files: the streaming kernel for dense calls of
+// one matrix, cudaErrorNotSupported for everything else.
+template <int BITS>
+cudaError_t try_stream(const QgemvParams& q, int gs, int dtype, int mt, bool dual, cudaStream_t st) {
+  if (dual || q.ids) return cudaErrorNotSupported;
+  if (dtype == QMM_BF16) {
+    if (gs == 32) return try_stream_mt<BITS, 32, __nv_bfloat16>(q, mt, st);
+    if (gs == 64) return try_stream_mt<BITS, 64, __nv_bfloat16>(q, mt, st);
+    return try_stream_mt<BITS, 128, __nv_bfloat16>(q, mt, st);
+  }
+  if (gs == 32) return try_stream_mt<BITS, 32, __half>(q, mt, st);
+  if (gs == 64) return try_stream_mt<BITS, 64, __half>(q, mt, st);
+  return try_stream_mt<BITS, 128, __half>(q, mt, st);
+}
+
+}  // namespace stream
+}  // namespace qmm
