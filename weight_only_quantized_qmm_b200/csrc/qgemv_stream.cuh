@@ -55,11 +55,14 @@ struct Params {
   int32_t* d_status;
   int tok_stride;       // bytes between staged token rows of x
   int stages;           // ring depth
+  int pf;               // units prefetched into L2 ahead of the shared-memory loads
+  uint32_t magic;       // two 16-bit floats whose low bits take a code (128 + q / 1024 + q)
   int off_code, off_sb, off_bar, off_part, off_xs, off_xsum;
 };
 
-// MODE 0: one token; 1: up to 8 tokens; 2: up to 16 tokens.
-template <int BITS, int GS, typename T, int MODE>
+// MODE 0: one token; 1: up to 8 tokens; 2: up to 16 tokens.  UG: groups per
+// unit (32, or 64 when the row length allows; 16 for 32-word groups).
+template <int BITS, int GS, typename T, int MODE, int UG>
 struct Cfg {
   using S = Share<BITS, GS, T>;
   static constexpr int MT = MODE == 2 ? 2 : 1;
@@ -69,7 +72,7 @@ struct Cfg {
   static constexpr int STAGERS = (KC + 1) * 32;                   // consumers + epilogue
   static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
   static constexpr int WPG = S::kWordsPerGroup;                   // words per group per row
-  static constexpr int GPU = WPG >= 32 ? 16 : 32;                 // groups per unit
+  static constexpr int GPU = UG;                                  // groups per unit
   static constexpr int GPW = GPU / KC;                            // groups per consumer per unit
   static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
   static constexpr int CODE_BYTES = Z * 16 * 128;
@@ -80,11 +83,29 @@ struct Cfg {
   static constexpr int NX = S::kSplit ? 2 : 1;                    // per-group sums kept
   static_assert(S::kFast, "integral-lane codes only");
   static_assert(GPW >= 1 && GPW * KC == GPU, "whole groups per consumer");
-  static_assert(Z >= 1 && Z <= 256, "box depth");
+  static_assert(Z >= 1 && Z <= 16, "unit of at most 16 slices (32 KB)");
+  static_assert((kRB & (kRB - 1)) == 0, "partial ring is a power of two");
 };
 
+__device__ __forceinline__ void sts32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t a, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float ldsf(uint32_t a) { return __uint_as_float(lds32(a)); }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+               "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
                                             uint32_t bar) {
@@ -115,9 +136,51 @@ __device__ __forceinline__ void mma_first(float (&d)[4], uint32_t a0, uint32_t a
   }
 }
 
+// Codes j and j + LPW/2 of a word of LW-bit lanes as a pair of 16-bit floats
+// (MAGIC + code, exact): one shift and one lop3 ((a & b) | c).
+template <int LW, int SH>
+__device__ __forceinline__ uint32_t lane_pair(uint32_t w, uint32_t magic) {
+  constexpr uint32_t MASK = ((1u << LW) - 1u) * 0x00010001u;
+  uint32_t d;
+  if constexpr (SH == 0) {
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
+  } else {
+    asm("{\n\t.reg .b32 t;\n\tshr.u32 t, %1, %4;\n\tlop3.b32 %0, t, %2, %3, 0xEA;\n\t}"
+        : "=r"(d)
+        : "r"(w), "n"(MASK), "r"(magic), "n"(SH));
+  }
+  return d;
+}
+// All LPW/2 pairs of one word, pair j = codes (j, j + LPW/2).
+template <class S>
+__device__ __forceinline__ void word_pairs(uint32_t w, uint32_t magic, uint32_t* out) {
+  constexpr int LW = S::kLW;
+  constexpr int NP = S::kLPW / 2;
+  out[0] = lane_pair<LW, 0>(w, magic);
+  out[1] = lane_pair<LW, LW>(w, magic);
+  if constexpr (NP >= 4) {
+    out[2] = lane_pair<LW, 2 * LW>(w, magic);
+    out[3] = lane_pair<LW, 3 * LW>(w, magic);
+  }
+  if constexpr (NP >= 8) {
+    out[4] = lane_pair<LW, 4 * LW>(w, magic);
+    out[5] = lane_pair<LW, 5 * LW>(w, magic);
+    out[6] = lane_pair<LW, 6 * LW>(w, magic);
+    out[7] = lane_pair<LW, 7 * LW>(w, magic);
+  }
+}
+
 template <int BITS, class S, typename T, int MT>
 __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], const uint32_t (&rawB)[S::kRegs],
-                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4]) {
+                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4],
+                                           uint32_t magic) {
+  constexpr int NP = S::kLPW / 2;  // pairs per word
+  uint32_t pA[S::kRegs * NP], pB[S::kRegs * NP];
+#pragma unroll
+  for (int k = 0; k < S::kRegs; ++k) {
+    word_pairs<S>(rawA[k], magic, pA + k * NP);
+    word_pairs<S>(rawB[k], magic, pB + k * NP);
+  }
 #pragma unroll
   for (int q2 = 0; q2 < S::kSteps / 2; ++q2) {
     uint4 bf[MT];
@@ -126,17 +189,13 @@ __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], con
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       const int q = 2 * q2 + h2;
-      const uint32_t a0 = share_pair<BITS, S>(rawA, 2 * q);
-      const uint32_t a1 = share_pair<BITS, S>(rawB, 2 * q);
-      const uint32_t a2 = share_pair<BITS, S>(rawA, 2 * q + 1);
-      const uint32_t a3 = share_pair<BITS, S>(rawB, 2 * q + 1);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         const uint32_t b0 = h2 ? bf[mt].z : bf[mt].x, b1 = h2 ? bf[mt].w : bf[mt].y;
         if (q == 0)
-          mma_first<T>(d[mt], a0, a1, a2, a3, b0, b1);
+          mma_first<T>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
         else
-          mma16816<T>(d[mt], a0, a1, a2, a3, b0, b1);
+          mma16816<T>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
       }
     }
   }
@@ -224,11 +283,11 @@ __device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint
     if (idx % TOKP >= p.M) xsum[idx] = 0.0f;
 }
 
-template <int BITS, int GS, typename T, int MODE>
-__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE>::THREADS, 1)
+template <int BITS, int GS, typename T, int MODE, int UG>
+__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG>::THREADS, 1)
 qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
                     const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmb) {
-  using C = Cfg<BITS, GS, T, MODE>;
+  using C = Cfg<BITS, GS, T, MODE, UG>;
   using S = typename C::S;
   constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC;
   constexpr float OFF = S::kOff;
@@ -243,7 +302,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
   const uint32_t bar_empty = bar_full + 8 * kMaxStages;
   const uint32_t bar_pfull = bar_empty + 8 * kMaxStages;
   const uint32_t bar_pempty = bar_pfull + 8 * kRB;
-  float4* part = reinterpret_cast<float4*>(smem + p.off_part);
+  const uint32_t part_sa = smem_u32(smem + p.off_part);
   uint8_t* xs = smem + p.off_xs;
   float* xsum = reinterpret_cast<float*>(smem + p.off_xsum);
 
@@ -273,7 +332,21 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     if (lane == 0) {
       bool failed = false;
       int tile = tb, ku = 0, issued = 0;
+      // L2 prefetch cursor: DRAM streams into L2 ahead of the ring, so the
+      // copies into shared memory see L2 latency
+      int pt = tb, pk = 0, pi = 0;
+      auto prefetch_next = [&]() {
+        if (pi < nunits) {
+          tma_prefetch_3d(&tmc, 0, pt * 16, pk * C::Z);
+          tma_prefetch_2d(&tms, pk * GPU, pt * 16);
+          tma_prefetch_2d(&tmb, pk * GPU, pt * 16);
+          ++pi;
+          if (++pk == p.upt) { pk = 0; ++pt; }
+        }
+      };
+      for (int i = 0; i < p.pf; ++i) prefetch_next();
       for (int i = 0; i < nunits; ++i) {
+        if (p.pf > 0) prefetch_next();
         const int slot = i % STAGES;
         if (i >= STAGES && !mbar_wait(bar_empty + 8 * slot, (uint32_t)((i / STAGES) - 1) & 1u, false)) {
           failed = true;
@@ -313,19 +386,29 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
         failed = true;
       }
       if (!failed) {
-        for (int idx = lane; idx < 16 * p.M; idx += 32) {
-          const int r = idx & 15, m = idx >> 4;
-          const int mt = m >> 3, col = m & 7;
-          const int src = ((r & 7) << 2) | (col >> 1);
-          const int ci = ((r >> 3) << 1) | (col & 1);
-          float y = 0.0f;
+        if constexpr (C::ONE) {
+          // partials: [entry][consumer][16 rows] floats
+          if (lane < 16) {
+            float y = 0.0f;
 #pragma unroll
-          for (int w = 0; w < KC; ++w) {
-            const float4 v = part[((e * KC + w) * MT + mt) * 32 + src];
-            y += ci == 0 ? v.x : ci == 1 ? v.y : ci == 2 ? v.z : v.w;
+            for (int w = 0; w < KC; ++w) y += ldsf(part_sa + (uint32_t)(((e * KC + w) * 16 + lane) * 4));
+            const int64_t row = (int64_t)(tb + jt) * 16 + lane;
+            if (row < p.N) store_as(p.out, p.out_dtype, row, y);
           }
-          const int64_t row = (int64_t)(tb + jt) * 16 + r;
-          if (row < p.N) store_as(p.out, p.out_dtype, (int64_t)m * p.out_ld + row, y);
+        } else {
+          // partials: [entry][consumer][token tile][lane] float4 (the mma C fragment)
+          for (int idx = lane; idx < 16 * p.M; idx += 32) {
+            const int r = idx & 15, m = idx >> 4;
+            const int mt = m >> 3, col = m & 7;
+            const int src = ((r & 7) << 2) | (col >> 1);
+            const int ci = ((r >> 3) << 1) | (col & 1);
+            const uint32_t a0 = part_sa + (uint32_t)((((e * KC) * MT + mt) * 32 + src) * 16 + ci * 4);
+            float y = 0.0f;
+#pragma unroll
+            for (int w = 0; w < KC; ++w) y += ldsf(a0 + (uint32_t)(w * MT * 32 * 16));
+            const int64_t row = (int64_t)(tb + jt) * 16 + r;
+            if (row < p.N) store_as(p.out, p.out_dtype, (int64_t)m * p.out_ld + row, y);
+          }
         }
       }
       __syncwarp();
@@ -345,7 +428,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
              (uint32_t)(warp * GPW * C::XG);
   }
-  const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + 2 * t) * 4);
+  // per-group sums: tokens 2t, 2t + 1 (token 0 only for a single token)
+  const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 4);
   // shared offsets (within a slot) of this lane's code words, row g, per group u
   uint32_t coff[GPW];
 #pragma unroll
@@ -355,6 +439,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     const int wb = w0 & 31;
     coff[u] = (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
   }
+  const uint32_t magic = p.magic;
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's groups
   const uint32_t soff = (uint32_t)((g * GPU + warp * GPW) * 2);
 
@@ -365,17 +450,22 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
   bool failed = false;
 
+  // unit i: slot i % STAGES with phase (i / STAGES) & 1, k-unit ku of tile jt
+  int slot = 0, ku = 0, jt = 0;
+  uint32_t phase = 0;
+  uint32_t cslot = code_ring, sslot = sb_ring + soff, bfull = bar_full;
+  uint32_t xbu[MT];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
+  uint32_t su = xsum_lane;
   for (int i = 0; i < nunits; ++i) {
-    const int jt = i / p.upt, ku = i - jt * p.upt;
-    const int slot = i % STAGES;
-    const bool ok = mbar_wait(bar_full + 8 * slot, (uint32_t)(i / STAGES) & 1u, failed);
+    bool ok = mbar_try_wait(bfull, phase);
+    if (!ok) ok = mbar_wait(bfull, phase, failed);
     if (__any_sync(0xffffffffu, !ok)) {
       if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
       failed = true;
     }
     if (!failed) {
-      const uint32_t cslot = code_ring + (uint32_t)(slot * C::CODE_BYTES);
-      const uint32_t sslot = sb_ring + (uint32_t)(slot * 2 * C::SB_BYTES) + soff;
       // GPW 16-bit scales (biases) of rows g and g + 8
       uint32_t sv[2][(GPW + 1) / 2], bv[2][(GPW + 1) / 2];
 #pragma unroll
@@ -396,10 +486,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
           }
         }
       }
-      uint32_t xbu[MT];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt] + (uint32_t)(ku * GPU * C::XG);
-      const uint32_t su = xsum_lane + (uint32_t)(ku * GPU * TOKP * 4);
 #pragma unroll
       for (int u = 0; u < GPW; ++u) {
         uint32_t rA[S::kRegs], rB[S::kRegs];
@@ -421,19 +507,19 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
           rB[0] = lds32(ca + 1024);
         }
         float d[MT][4];
-        group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d);
+        group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
         const int hw = u & 1;
         const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
         const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           if constexpr (C::ONE) {
-            const float X0 = __uint_as_float(lds32(su + (uint32_t)(u * TOKP * 4) - (uint32_t)(8 * t)));
+            const float X0 = __uint_as_float(lds32(su + (uint32_t)(u * TOKP * 4)));
             if constexpr (C::NX == 1) {
               acc[0][0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], acc[0][0]));
               acc[0][2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], acc[0][2]));
             } else {
-              const float O0 = __uint_as_float(lds32(su + (uint32_t)((Gpad + u) * TOKP * 4) - (uint32_t)(8 * t)));
+              const float O0 = __uint_as_float(lds32(su + (uint32_t)((Gpad + u) * TOKP * 4)));
               acc[0][0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], acc[0][0])));
               acc[0][2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], acc[0][2])));
             }
@@ -461,10 +547,10 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar_empty + 8 * slot);
+    if (lane == 0) mbar_arrive(bfull + 8 * kMaxStages);  // the slot's `empty` barrier
 
-    if (ku == p.upt - 1) {  // tile done: post this warp's partial
-      const int e = jt % kRB;
+    if (++ku == p.upt) {  // tile done: post this warp's partial
+      const int e = jt & (kRB - 1);
       if (jt >= kRB) {
         const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / kRB) - 1) & 1u, failed);
         if (__any_sync(0xffffffffu, !okp)) {
@@ -472,14 +558,43 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
           failed = true;
         }
       }
+      if constexpr (C::ONE) {
+        if (t == 0) {
+          sts32(part_sa + (uint32_t)(((e * KC + warp) * 16 + g) * 4), acc[0][0]);
+          sts32(part_sa + (uint32_t)(((e * KC + warp) * 16 + g + 8) * 4), acc[0][2]);
+        }
+      } else {
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        part[((e * KC + warp) * MT + mt) * 32 + lane] = make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]);
+        for (int mt = 0; mt < MT; ++mt)
+          sts128(part_sa + (uint32_t)((((e * KC + warp) * MT + mt) * 32 + lane) * 16),
+                 make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[mt][k] = 0.0f;
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull + 8 * e);
+      ku = 0;
+      ++jt;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
+      su = xsum_lane;
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) xbu[mt] += (uint32_t)(GPU * C::XG);
+      su += (uint32_t)(GPU * TOKP * 4);
+    }
+    if (++slot == STAGES) {
+      slot = 0;
+      phase ^= 1u;
+      cslot = code_ring;
+      sslot = sb_ring + soff;
+      bfull = bar_full;
+    } else {
+      cslot += (uint32_t)C::CODE_BYTES;
+      sslot += (uint32_t)(2 * C::SB_BYTES);
+      bfull += 8;
     }
   }
 }
@@ -514,9 +629,9 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
 
 // Dense calls only (no ids, one matrix); cudaErrorNotSupported sends the caller
 // to the general kernels.
-template <int BITS, int GS, typename T, int MODE>
+template <int BITS, int GS, typename T, int MODE, int UG>
 cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
-  using C = Cfg<BITS, GS, T, MODE>;
+  using C = Cfg<BITS, GS, T, MODE, UG>;
   if (q.ids || q.amode != 0 || q.n_pairs < 1 || q.n_pairs > C::TOKP) return cudaErrorNotSupported;
   if (q.G % 8 != 0 || q.wpr % 32 != 0 || q.n_rows < 16 || q.G < C::GPU) return cudaErrorNotSupported;
   if (((uintptr_t)q.packed[0] | (uintptr_t)q.scales[0] | (uintptr_t)q.biases[0]) & 15) return cudaErrorNotSupported;
@@ -533,11 +648,12 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   p.out_dtype = q.out_dtype;
   p.out_ld = q.out_ld;
   p.d_status = q.d_status;
+  p.magic = C::S::kMagic;
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
   // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums]
-  const size_t part = (size_t)kRB * C::KC * C::MT * 32 * 16;
+  const size_t part = C::ONE ? (size_t)kRB * C::KC * 16 * 4 : (size_t)kRB * C::KC * C::MT * 32 * 16;
   const size_t xs = align128((size_t)p.M * p.tok_stride);
   const size_t xsum = align128((size_t)Gpad * C::TOKP * 4 * C::NX);
   const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
@@ -545,12 +661,13 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
     return 1024 + (size_t)stages * C::CODE_BYTES + align128((size_t)stages * 2 * C::SB_BYTES) + align128(bars) +
            part + xs + xsum;
   };
-  // about 96 KB of weights in flight per SM
-  int stages = (int)((96 * 1024) / C::TX);
+  // about 144 KB of weights in flight per SM
+  int stages = (int)((144 * 1024) / C::TX);
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   while (stages > 2 && total(stages) > (size_t)kSmemMax) --stages;
   if (total(stages) > (size_t)kSmemMax) return cudaErrorNotSupported;
   p.stages = stages;
+  p.pf = 0;  // L2 prefetch window (units); off: measured no faster than the ring alone
   p.off_code = 0;
   p.off_sb = stages * C::CODE_BYTES;
   p.off_bar = p.off_sb + (int)align128((size_t)stages * 2 * C::SB_BYTES);
@@ -564,7 +681,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
       !make_sb_map(&tms, q.scales[0], q.n_rows, q.G, C::GPU) || !make_sb_map(&tmb, q.biases[0], q.n_rows, q.G, C::GPU))
     return cudaErrorNotSupported;
 
-  auto k = qgemv_stream_kernel<BITS, GS, T, MODE>;
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -590,9 +707,17 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
 
 template <int BITS, int GS, typename T>
 cudaError_t try_stream_mt(const QgemvParams& q, int mt, cudaStream_t st) {
-  if constexpr (Share<BITS, GS, T>::kFast) {
-    if (q.n_pairs == 1) return launch_stream<BITS, GS, T, 0>(q, st);
-    return mt == 1 ? launch_stream<BITS, GS, T, 1>(q, st) : launch_stream<BITS, GS, T, 2>(q, st);
+  using S = Share<BITS, GS, T>;
+  if constexpr (S::kFast) {
+    constexpr int WPG = S::kWordsPerGroup;
+    constexpr int UB = WPG >= 32 ? 16 : 32;           // base unit
+    constexpr int UW = WPG <= 8 ? 64 : UB;            // wide unit: 4 groups per consumer
+    const bool wide = (q.G % UW) == 0;
+    if (q.n_pairs == 1)
+      return wide ? launch_stream<BITS, GS, T, 0, UW>(q, st) : launch_stream<BITS, GS, T, 0, UB>(q, st);
+    if (mt == 1)
+      return wide ? launch_stream<BITS, GS, T, 1, UW>(q, st) : launch_stream<BITS, GS, T, 1, UB>(q, st);
+    return launch_stream<BITS, GS, T, 2, UB>(q, st);
   } else {
     return cudaErrorNotSupported;
   }
