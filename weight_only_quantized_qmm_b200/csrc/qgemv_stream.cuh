@@ -84,6 +84,7 @@ struct Cfg {
   static_assert(S::kFast, "integral-lane codes only");
   static_assert(GPW >= 1 && GPW * KC == GPU, "whole groups per consumer");
   static_assert(Z >= 1 && Z <= 16, "unit of at most 16 slices (32 KB)");
+  static_assert(GPU * 2 == 32 || GPU * 2 == 64 || GPU * 2 == 128, "scale rows of one swizzle span");
   static_assert((kRB & (kRB - 1)) == 0, "partial ring is a power of two");
 };
 
@@ -198,6 +199,27 @@ __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], con
           mma16816<T>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
       }
     }
+  }
+}
+
+// As group_dot1 for one token column, with the x fragments in registers.
+template <int BITS, class S, typename T>
+__device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[S::kRegs], const uint32_t (&rawB)[S::kRegs],
+                                             const uint4 (&bf)[S::kSteps / 2], float (&d)[4], uint32_t magic) {
+  constexpr int NP = S::kLPW / 2;
+  uint32_t pA[S::kRegs * NP], pB[S::kRegs * NP];
+#pragma unroll
+  for (int k = 0; k < S::kRegs; ++k) {
+    word_pairs<S>(rawA[k], magic, pA + k * NP);
+    word_pairs<S>(rawB[k], magic, pB + k * NP);
+  }
+#pragma unroll
+  for (int q = 0; q < S::kSteps; ++q) {
+    const uint32_t b0 = (q & 1) ? bf[q >> 1].z : bf[q >> 1].x, b1 = (q & 1) ? bf[q >> 1].w : bf[q >> 1].y;
+    if (q == 0)
+      mma_first<T>(d, pA[0], pB[0], pA[1], pB[1], b0, b1);
+    else
+      mma16816<T>(d, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
   }
 }
 
@@ -441,7 +463,11 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
   }
   const uint32_t magic = p.magic;
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's groups
-  const uint32_t soff = (uint32_t)((g * GPU + warp * GPW) * 2);
+  // (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
+  constexpr int PITCH = GPU * 2;
+  const int sfx = PITCH == 128 ? (g & 7) : PITCH == 64 ? ((g >> 1) & 3) : ((g >> 2) & 1);
+  const int sbyte = warp * GPW * 2;
+  const uint32_t soff = (uint32_t)(g * PITCH + ((((sbyte >> 4) ^ sfx)) << 4) + (sbyte & 15));
 
   float acc[MT][4];
 #pragma unroll
@@ -458,12 +484,29 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
   uint32_t su = xsum_lane;
+  // one token: this warp's x fragments and group sums of the current k-unit,
+  // in registers (reloaded only when the k-unit changes)
+  uint4 xr[C::ONE ? GPW : 1][S::kSteps / 2];
+  float xsr[C::ONE ? GPW : 1][C::NX];
+  int xku = -1;
   for (int i = 0; i < nunits; ++i) {
     bool ok = mbar_try_wait(bfull, phase);
     if (!ok) ok = mbar_wait(bfull, phase, failed);
     if (__any_sync(0xffffffffu, !ok)) {
       if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
       failed = true;
+    }
+    if constexpr (C::ONE) {
+      if (ku != xku) {
+        xku = ku;
+#pragma unroll
+        for (int u = 0; u < GPW; ++u) {
+#pragma unroll
+          for (int q2 = 0; q2 < S::kSteps / 2; ++q2) xr[u][q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
+          xsr[u][0] = ldsf(su + (uint32_t)(u * TOKP * 4));
+          if constexpr (C::NX == 2) xsr[u][C::NX - 1] = ldsf(su + (uint32_t)((Gpad + u) * TOKP * 4));
+        }
+      }
     }
     if (!failed) {
       // GPW 16-bit scales (biases) of rows g and g + 8
@@ -507,19 +550,22 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
           rB[0] = lds32(ca + 1024);
         }
         float d[MT][4];
-        group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
+        if constexpr (C::ONE)
+          group_dot_rx<BITS, S, T>(rA, rB, xr[u], d[0], magic);
+        else
+          group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
         const int hw = u & 1;
         const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
         const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           if constexpr (C::ONE) {
-            const float X0 = __uint_as_float(lds32(su + (uint32_t)(u * TOKP * 4)));
+            const float X0 = xsr[u][0];
             if constexpr (C::NX == 1) {
               acc[0][0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], acc[0][0]));
               acc[0][2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], acc[0][2]));
             } else {
-              const float O0 = __uint_as_float(lds32(su + (uint32_t)((Gpad + u) * TOKP * 4)));
+              const float O0 = xsr[u][C::NX - 1];
               acc[0][0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], acc[0][0])));
               acc[0][2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], acc[0][2])));
             }
@@ -614,7 +660,9 @@ inline bool make_code_map3(CUtensorMap* map, const uint32_t* packed, int64_t row
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2-D map over a [rows, G] array of 16-bit scales or biases: 16-row x gpu boxes.
+// 2-D map over a [rows, G] array of 16-bit scales or biases: 16-row x gpu boxes,
+// swizzled at the box row width (32, 64 or 128 bytes) so that the eight rows a
+// warp reads at one column fall in different banks.
 inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G, int gpu) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return false;
@@ -622,8 +670,11 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
   const cuuint64_t strides[1] = {(cuuint64_t)G * 2};
   const cuuint32_t box[2] = {(cuuint32_t)gpu, 16};
   const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = gpu * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : gpu * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -661,7 +712,8 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
     return 1024 + (size_t)stages * C::CODE_BYTES + align128((size_t)stages * 2 * C::SB_BYTES) + align128(bars) +
            part + xs + xsum;
   };
-  // about 144 KB of weights in flight per SM
+  // about 144 KB of the weight stream in flight per SM (measured: deeper rings
+  // and an L2 prefetch window ahead of the ring were not faster)
   int stages = (int)((144 * 1024) / C::TX);
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   while (stages > 2 && total(stages) > (size_t)kSmemMax) --stages;
