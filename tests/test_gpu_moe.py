@@ -89,6 +89,42 @@ def test_moe_gate_up_silu_batched_many_tokens_per_expert():
     gate(out32.cpu().numpy(), ref, "batched gate_up_silu")
 
 
+@pytest.mark.parametrize("dual", [False, True])
+def test_moe_segments_split_one_expert_deterministic(dual):
+    """Rows long enough for the streaming kernel (K = 2048) and ~12 pairs per
+    expert, so an expert's pairs span several segments: every CTA must derive
+    the same pair lists (outputs complete, identical between calls, 16-bit
+    output = RNE of the fp32 output) and match the oracle."""
+    E, n_rows, n_cols, bits, gs = 8, 64, 2048, 4, 64
+    g, og = make_stack(E, n_rows, n_cols, bits, gs, 50)
+    u, ou = make_stack(E, n_rows, n_cols, bits, gs, 51)
+    m, top_k = 48, 2
+    a = wl.gen_x(m, n_cols, 52).reshape(-1)
+    ids = wl.gen_moe_ids(m, E, top_k, 53)
+    assert int(torch.bincount(ids.reshape(-1), minlength=E).max()) > 8
+
+    def call(dt):
+        if dual:
+            return api.qmm_moe_gemv_id_gate_up_silu_batched(a.to(DEV), ids.to(DEV), m, top_k, n_cols, 0,
+                                                            g, u, dt)
+        return api.qmm_moe_gemv_id_batched(a.to(DEV), ids.to(DEV), m, top_k, n_cols, 0, g, dt)
+
+    outs = [call(torch.float32) for _ in range(3)]
+    o16 = call(None)
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(outs[0], o)
+    rne_equal(o16, outs[0])
+    if dual:
+        ref, rc = oracle.moe_gate_up_silu_batched(np_storage(a), oracle.BF16, ids.numpy(), m, top_k,
+                                                  n_cols, 0, og, ou)
+    else:
+        ref, rc = oracle.moe_gemv_id_batched(np_storage(a), oracle.BF16, ids.numpy(), m, top_k,
+                                             n_cols, 0, og)
+    assert rc == oracle.ORC_OK
+    gate(outs[0].cpu().numpy(), ref, "segments split")
+
+
 def test_moe_bad_id_zero_row_and_status():
     E, n_rows, n_cols, bits, gs = 3, 32, 128, 4, 64
     st, ost = make_stack(E, n_rows, n_cols, bits, gs, 50)

@@ -271,14 +271,30 @@ __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int
       if (lane == 0) *s_nd = nd;
     }
     __syncthreads();
-    for (int i = tid; i < p.n_pairs; i += nthr) {
-      const int e = p.ids[i];
-      if (e >= 0 && e < E) {
-        s_list[s_start[e] + atomicAdd(&s_fill[e], 1)] = i;
-      } else if (blockIdx.x == 0) {
-        // bad id: zero row, report
-        for (int64_t n = 0; n < p.n_rows; ++n) store_as(p.out, p.out_dtype, (int64_t)i * p.out_ld + n, 0.0f);
-        set_status(p.d_status, QMM_ERR_BAD_EXPERT_ID);
+    // stable placement (pairs of an expert in increasing pair order), so that
+    // every CTA derives the same lists: one warp ranks 32 pairs at a time
+    if (warp == 0) {
+      for (int base = 0; base < p.n_pairs; base += 32) {
+        const int i = base + lane;
+        const int e = i < p.n_pairs ? p.ids[i] : -1;
+        const bool valid = e >= 0 && e < E;
+        const unsigned same = __match_any_sync(0xffffffffu, valid ? e : E + lane);
+        if (valid) {
+          const int rank = s_fill[e] + __popc(same & ((1u << lane) - 1u));
+          s_list[s_start[e] + rank] = i;
+        }
+        __syncwarp();
+        if (valid && lane == 31 - __clz(same)) s_fill[e] += __popc(same);
+        __syncwarp();
+      }
+    }
+    if (blockIdx.x == 0) {
+      for (int i = tid; i < p.n_pairs; i += nthr) {
+        const int e = p.ids[i];
+        if (e < 0 || e >= E) {  // bad id: zero row, report
+          for (int64_t n = 0; n < p.n_rows; ++n) store_as(p.out, p.out_dtype, (int64_t)i * p.out_ld + n, 0.0f);
+          set_status(p.d_status, QMM_ERR_BAD_EXPERT_ID);
+        }
       }
     }
     __syncthreads();

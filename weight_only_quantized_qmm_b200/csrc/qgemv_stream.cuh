@@ -1,34 +1,43 @@
-// Streaming decode GEMV for the dense case y = x . dequant(W)^T with a few
-// tokens (M <= 16): the bandwidth-bound half of the weight-only quantized
-// matmul ("Quantized matmul" / affine mode, w = q * scale + bias per group).
+// Streaming quantized GEMV for few tokens per weight row: the bandwidth-bound
+// half of the weight-only quantized matmul ("Quantized matmul", affine mode
+// w = q * scale + bias per group), for dense calls y = x . dequant(W)^T and
+// for the indirect (MoE) form out[i] = a[off(i)] . dequant(W[ids[i]])^T,
+// optionally fused as SiLU(gate) * up over two expert stacks.
 //
-// One persistent CTA per SM owns a contiguous range of 16-row tiles of W and
-// streams each tile through shared memory as units of GPU groups (all 16
-// rows).  A unit arrives with three TMA copies counted on the slot's `full`
-// mbarrier: the packed codes as one 3-D box (16 rows x Z slices of 128 bytes,
-// 128-byte swizzle; few large copies keep the copy engine off the critical
-// path), the unit's scales and its biases (16 rows x GPU 16-bit values each).
-// Warp roles:
+// Work list.  Every CTA sorts the call's pairs by expert in shared memory
+// (dense: one expert holding the M tokens) and cuts each expert's pairs into
+// segments of up to CH pairs.  A segment covers all 16-row tiles of its
+// expert's matrix; the (segment, tile) list is split into contiguous ranges,
+// one per CTA (persistent grid, one CTA per SM).
+//
+// Each tile streams through shared memory as units of GPU groups (all 16
+// rows).  A unit arrives with TMA copies counted on the slot's `full`
+// mbarrier: per matrix, the packed codes as one 3-D box (16 rows x Z slices of
+// 128 bytes, 128-byte swizzle; few large copies keep the copy engine off the
+// critical path) and the unit's scales and biases (16 rows x GPU 16-bit
+// values, swizzled at their row width).  Warp roles:
 //   * producer (1 warp, one lane) issues the copies, slot by slot;
-//   * consumers (kC warps) all read every unit, consumer w taking groups
+//   * consumers (KC warps) all read every unit, consumer w taking groups
 //     [w * GPW, (w + 1) * GPW).  Per group a consumer turns codes into 16-bit
 //     floats (OFF + q, exact), takes the partial dot with x on the tensor
-//     cores (mma.m16n8k16; rows of W as m, tokens as n), and folds it into
-//     fp32 accumulators as
+//     cores (mma.m16n8k16; rows of W as m, the segment's pairs as n), and
+//     folds it into fp32 accumulators as
 //       y += s * d + (b - OFF * s) * X,   X = sum of x over the group,
 //     which is sum_k x_k (q_k s + b) rewritten per group.  The slot is free
-//     again once all kC consumers arrived on its `empty` mbarrier;
+//     again once all KC consumers arrived on its `empty` mbarrier.  At a new
+//     segment the consumers stage its x rows (tensor-core k order, with the
+//     per-group sums);
 //   * epilogue (1 warp): when every consumer posted its partial for a tile
 //     (mbarrier `pfull`), sums them in consumer order (the result does not
-//     depend on timing) and stores the tile's outputs.
-// x is staged once per CTA in the tensor-core k order with its per-group sums.
+//     depend on timing), applies SiLU(gate) * up for the fused form and
+//     stores the tile's outputs.
 // Every wait is bounded: a timeout sets QMM_ERR_TIMEOUT, skips the remaining
 // arithmetic and still drains the copies in flight before the CTA exits.
 //
-// Launched with programmatic stream serialization: the producer streams
-// weights (which no earlier kernel writes) before griddepcontrol.wait, so a
-// call's weight traffic can start while the previous kernel drains; x and y
-// are only touched after the wait.
+// Launched with programmatic stream serialization: for dense calls the
+// producer streams weights (which no earlier kernel writes) before
+// griddepcontrol.wait, so a call's weight traffic can start while the
+// previous kernel drains; ids, x and y are only touched after the wait.
 #pragma once
 
 #include <cuda.h>
@@ -42,43 +51,36 @@ constexpr int kRB = 2;          // partial-sum ring entries (tiles)
 constexpr int kMaxStages = 8;
 
 struct Params {
-  const void* x;        // [M, K] activations (row stride K)
-  int M;                // tokens, 1..16
-  int64_t K;
-  int G;                // groups per row
+  QgemvParams q;        // the call: pairs, experts, activations, output
   int upt;              // units per tile (ceil(G / GPU))
-  int64_t N;            // rows of W
-  int ntiles;           // ceil(N / 16)
-  void* out;            // [M, N]
-  int out_dtype;
-  int64_t out_ld;
-  int32_t* d_status;
-  int tok_stride;       // bytes between staged token rows of x
+  int ntiles_e;         // 16-row tiles per expert matrix
+  int CH;               // pairs per segment
+  int tok_stride;       // bytes between staged rows of x
   int stages;           // ring depth
-  int pf;               // units prefetched into L2 ahead of the shared-memory loads
   uint32_t magic;       // two 16-bit floats whose low bits take a code (128 + q / 1024 + q)
-  int off_code, off_sb, off_bar, off_part, off_xs, off_xsum;
+  int off_code, off_sb, off_bar, off_part, off_xs, off_xsum, off_plan;
 };
 
-// MODE 0: one token; 1: up to 8 tokens; 2: up to 16 tokens.  UG: groups per
-// unit (32, or 64 when the row length allows; 16 for 32-word groups).
-template <int BITS, int GS, typename T, int MODE, int UG>
+// MODE 0: one pair per segment; 1: up to 8; 2: up to 16.  UG: groups per unit
+// (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
+// matrices per pair (2: gate and up).
+template <int BITS, int GS, typename T, int MODE, int UG, int NS>
 struct Cfg {
   using S = Share<BITS, GS, T>;
   static constexpr int MT = MODE == 2 ? 2 : 1;
   static constexpr bool ONE = MODE == 0;
   static constexpr int KC = MT == 1 ? 16 : 8;                     // consumer warps
   static constexpr int THREADS = (KC + 2) * 32;
-  static constexpr int STAGERS = (KC + 1) * 32;                   // consumers + epilogue
   static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
   static constexpr int WPG = S::kWordsPerGroup;                   // words per group per row
   static constexpr int GPU = UG;                                  // groups per unit
   static constexpr int GPW = GPU / KC;                            // groups per consumer per unit
   static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
-  static constexpr int CODE_BYTES = Z * 16 * 128;
-  static constexpr int SB_BYTES = 16 * GPU * 2;                   // scales (or biases) of a unit
-  static constexpr uint32_t TX = CODE_BYTES + 2 * SB_BYTES;
+  static constexpr int CODE_BYTES = Z * 16 * 128;                 // one matrix
+  static constexpr int SB_BYTES = 16 * GPU * 2;                   // scales (or biases) of one matrix
+  static constexpr uint32_t TX = NS * (CODE_BYTES + 2 * SB_BYTES);
   static constexpr int TOKP = 8 * MT;
+  static constexpr int CH = ONE ? 1 : TOKP;                       // pairs per segment
   static constexpr int XG = 4 * S::kVirt * (int)sizeof(T);        // staged x bytes per group
   static constexpr int NX = S::kSplit ? 2 : 1;                    // per-group sums kept
   static_assert(S::kFast, "integral-lane codes only");
@@ -244,14 +246,36 @@ __device__ __forceinline__ float half_to_f32(uint32_t v, int hi) {
   }
 }
 
-// Stage x for tokens [0, M) and groups [0, Gpad): per (token, group, quarter t)
-// the kVirt values of quarter t in slot order (the codes' mma k order), zero
-// past G; per (group, token) the fp32 sum of x over the group (and, for the
-// two-nibble 8-bit form, the sum of the slot values x').
+
+// Walk over the CTA's (segment, tile) range; segment sg belongs to the j-th
+// distinct expert when seg[j] <= sg < seg[j + 1].
+struct Walk {
+  int sg, rt, j;
+  __device__ __forceinline__ void start(int t, int ntiles_e, const int* seg, int nd) {
+    sg = t / ntiles_e;
+    rt = t - sg * ntiles_e;
+    j = 0;
+    while (j < nd - 1 && seg[j + 1] <= sg) ++j;
+  }
+  __device__ __forceinline__ void next(int ntiles_e, const int* seg, int nd) {
+    if (++rt == ntiles_e) {
+      rt = 0;
+      ++sg;
+      while (j < nd - 1 && seg[j + 1] <= sg) ++j;
+    }
+  }
+};
+
+// Stage the x rows of a segment's pairs [0, np) for groups [0, Gpad): per
+// (pair, group, quarter t) the kVirt values of quarter t in slot order (the
+// codes' mma k order), zero past G; per (group, pair) the fp32 sum of x over
+// the group (and, for the two-nibble 8-bit form, the sum of the slot values
+// x').  Pairs [np, TOKP) of the sums read as zero.
 template <class S, typename T, int TOKP, int NX, int NTHR>
-__device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint8_t* xs, float* xsum) {
+__device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, int np, int Gpad,
+                                        int tok_stride, int sid, uint8_t* xs, float* xsum) {
   constexpr int GS = S::kCodes * 4;
-  const int ntask = p.M * Gpad * 4;
+  const int ntask = np * Gpad * 4;
   for (int base = 0; base < ntask; base += NTHR) {
     const int idx = base + sid;
     const bool act = idx < ntask;
@@ -260,8 +284,8 @@ __device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint
     float sb = 0.0f, so = 0.0f;
     if (act) {
       __align__(16) T xv[S::kCodes];
-      if (gl < p.G) {
-        const T* xa = reinterpret_cast<const T*>(p.x) + (int64_t)m * p.K + (int64_t)gl * GS + tt * S::kCodes;
+      if (gl < q.G) {
+        const T* xa = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS + tt * S::kCodes;
         if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
 #pragma unroll
           for (int c = 0; c < S::kCodes * (int)sizeof(T) / 16; ++c)
@@ -277,19 +301,17 @@ __device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint
       }
       __align__(16) T outv[S::kVirt];
 #pragma unroll
-      for (int q = 0; q < S::kVirt; ++q) {
-        const int vv = S::slot_virtual(q);
+      for (int qv = 0; qv < S::kVirt; ++qv) {
+        const int vv = S::slot_virtual(qv);
         const float mult = S::virt_mult(vv);
         const float xf = to_f32(xv[S::virt_code(vv)]) * mult;
-        outv[q] = from_f32<T>(xf);
+        outv[qv] = from_f32<T>(xf);
         so += xf;
         if (mult == 1.0f) sb += xf;
       }
-      uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)m * p.tok_stride +
-                                            (size_t)(gl * 4 + tt) * S::kVirt * sizeof(T));
+      uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)m * tok_stride + (size_t)(gl * 4 + tt) * S::kVirt * sizeof(T));
 #pragma unroll
-      for (int q = 0; q < (int)(S::kVirt * sizeof(T) / 16); ++q)
-        dst[q] = reinterpret_cast<const uint4*>(outv)[q];
+      for (int qv = 0; qv < (int)(S::kVirt * sizeof(T) / 16); ++qv) dst[qv] = reinterpret_cast<const uint4*>(outv)[qv];
     }
     sb += __shfl_xor_sync(0xffffffffu, sb, 1);
     so += __shfl_xor_sync(0xffffffffu, so, 1);
@@ -300,43 +322,46 @@ __device__ __forceinline__ void stage_x(const Params& p, int Gpad, int sid, uint
       if constexpr (NX == 2) xsum[(Gpad + gl) * TOKP + m] = so;
     }
   }
-  // padding tokens [M, TOKP) of the sums read as zero
   for (int idx = sid; idx < Gpad * TOKP * NX; idx += NTHR)
-    if (idx % TOKP >= p.M) xsum[idx] = 0.0f;
+    if (idx % TOKP >= np) xsum[idx] = 0.0f;
 }
 
-template <int BITS, int GS, typename T, int MODE, int UG>
-__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG>::THREADS, 1)
-qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
-                    const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmb) {
-  using C = Cfg<BITS, GS, T, MODE, UG>;
+template <int BITS, int GS, typename T, int MODE, int UG, int NS>
+__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS>::THREADS, 1)
+qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, const __grid_constant__ CUtensorMap tms0,
+                    const __grid_constant__ CUtensorMap tmb0, const __grid_constant__ CUtensorMap tmc1,
+                    const __grid_constant__ CUtensorMap tms1, const __grid_constant__ CUtensorMap tmb1) {
+  using C = Cfg<BITS, GS, T, MODE, UG, NS>;
   using S = typename C::S;
-  constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC;
+  constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC, CH = C::CH;
   constexpr float OFF = S::kOff;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const QgemvParams& q = p.q;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int STAGES = p.stages;
   const uint32_t code_ring = smem_u32(smem + p.off_code);
   const uint32_t sb_ring = smem_u32(smem + p.off_sb);
   const uint32_t bar_full = smem_u32(smem + p.off_bar);
-  const uint32_t bar_empty = bar_full + 8 * kMaxStages;
-  const uint32_t bar_pfull = bar_empty + 8 * kMaxStages;
+  const uint32_t bar_pfull = bar_full + 16 * kMaxStages;  // after full[] and empty[]
   const uint32_t bar_pempty = bar_pfull + 8 * kRB;
   const uint32_t part_sa = smem_u32(smem + p.off_part);
   uint8_t* xs = smem + p.off_xs;
   float* xsum = reinterpret_cast<float*>(smem + p.off_xsum);
-
-  const int tb = (int)((int64_t)p.ntiles * blockIdx.x / gridDim.x);
-  const int te = (int)((int64_t)p.ntiles * (blockIdx.x + 1) / gridDim.x);
-  const int nt = te - tb;
-  const int nunits = nt * p.upt;
+  const int E = q.num_experts;
+  int* s_cnt = reinterpret_cast<int*>(smem + p.off_plan);
+  int* s_start = s_cnt + E;
+  int* s_fill = s_start + E;
+  int* s_dist = s_fill + E;
+  int* s_seg = s_dist + E;  // E + 1 entries
+  int* s_list = s_seg + E + 1;
+  __shared__ int s_nd;
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, KC);
+      mbar_init(bar_full + 8 * kMaxStages + 8 * s, KC);
     }
     for (int e = 0; e < kRB; ++e) {
       mbar_init(bar_pfull + 8 * e, KC);
@@ -344,45 +369,63 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // the ids (like x) may come from the previous kernel in the stream
+  if (q.ids) asm volatile("griddepcontrol.wait;" ::: "memory");
+  build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
+  if (tid == 0) {
+    int run = 0;
+    s_seg[0] = 0;
+    for (int j = 0; j < s_nd; ++j) {
+      run += (s_cnt[s_dist[j]] + CH - 1) / CH;
+      s_seg[j + 1] = run;
+    }
+  }
   __syncthreads();
   // the next kernel in the stream may launch now; it waits for this grid's
   // completion before it reads anything this grid writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+  const int nd = s_nd;
+  const int TT = s_seg[nd] * p.ntiles_e;
+  const int tb = (int)((int64_t)TT * blockIdx.x / gridDim.x);
+  const int te = (int)((int64_t)TT * (blockIdx.x + 1) / gridDim.x);
+  const int nt = te - tb;
+  const int nunits = nt * p.upt;
+  const int Gpad = p.upt * GPU;
+
   // ---------------------------------------------------------------- producer
   if (warp == C::PRODUCER) {
-    if (lane == 0) {
+    if (lane == 0 && nt > 0) {
       bool failed = false;
-      int tile = tb, ku = 0, issued = 0;
-      // L2 prefetch cursor: DRAM streams into L2 ahead of the ring, so the
-      // copies into shared memory see L2 latency
-      int pt = tb, pk = 0, pi = 0;
-      auto prefetch_next = [&]() {
-        if (pi < nunits) {
-          tma_prefetch_3d(&tmc, 0, pt * 16, pk * C::Z);
-          tma_prefetch_2d(&tms, pk * GPU, pt * 16);
-          tma_prefetch_2d(&tmb, pk * GPU, pt * 16);
-          ++pi;
-          if (++pk == p.upt) { pk = 0; ++pt; }
-        }
-      };
-      for (int i = 0; i < p.pf; ++i) prefetch_next();
+      int ku = 0, issued = 0;
+      Walk w;
+      w.start(tb, p.ntiles_e, s_seg, nd);
       for (int i = 0; i < nunits; ++i) {
-        if (p.pf > 0) prefetch_next();
         const int slot = i % STAGES;
-        if (i >= STAGES && !mbar_wait(bar_empty + 8 * slot, (uint32_t)((i / STAGES) - 1) & 1u, false)) {
+        if (i >= STAGES &&
+            !mbar_wait(bar_full + 8 * kMaxStages + 8 * slot, (uint32_t)((i / STAGES) - 1) & 1u, false)) {
           failed = true;
-          set_status(p.d_status, QMM_ERR_TIMEOUT);
+          set_status(q.d_status, QMM_ERR_TIMEOUT);
           break;
         }
+        const int y = s_dist[w.j] * (int)q.n_rows + w.rt * 16;  // first row in the expert stack
         const uint32_t fb = bar_full + 8 * slot;
         mbar_arrive_expect_tx(fb, C::TX);
-        tma_load_3d(code_ring + (uint32_t)(slot * C::CODE_BYTES), &tmc, 0, tile * 16, ku * C::Z, fb);
-        const uint32_t sd = sb_ring + (uint32_t)(slot * 2 * C::SB_BYTES);
-        tma_load_2d(sd, &tms, ku * GPU, tile * 16, fb);
-        tma_load_2d(sd + C::SB_BYTES, &tmb, ku * GPU, tile * 16, fb);
+        const uint32_t cd = code_ring + (uint32_t)(slot * NS * C::CODE_BYTES);
+        const uint32_t sd = sb_ring + (uint32_t)(slot * NS * 2 * C::SB_BYTES);
+        tma_load_3d(cd, &tmc0, 0, y, ku * C::Z, fb);
+        tma_load_2d(sd, &tms0, ku * GPU, y, fb);
+        tma_load_2d(sd + C::SB_BYTES, &tmb0, ku * GPU, y, fb);
+        if constexpr (NS == 2) {
+          tma_load_3d(cd + C::CODE_BYTES, &tmc1, 0, y, ku * C::Z, fb);
+          tma_load_2d(sd + 2 * C::SB_BYTES, &tms1, ku * GPU, y, fb);
+          tma_load_2d(sd + 3 * C::SB_BYTES, &tmb1, ku * GPU, y, fb);
+        }
         issued = i + 1;
-        if (++ku == p.upt) { ku = 0; ++tile; }
+        if (++ku == p.upt) {
+          ku = 0;
+          if (i + 1 < nunits) w.next(p.ntiles_e, s_seg, nd);
+        }
       }
       // no copy may still be landing when the CTA exits
       for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
@@ -390,51 +433,63 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     }
     return;
   }
-
-  // --------------------------------------------------- x staging (after the wait)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int Gpad = p.upt * GPU;
-  stage_x<S, T, TOKP, C::NX, C::STAGERS>(p, Gpad, warp < KC ? tid : tid - 32, xs, xsum);
-  asm volatile("bar.sync 1, %0;" ::"n"(C::STAGERS) : "memory");
+  if (!q.ids) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---------------------------------------------------------------- epilogue
   if (warp == C::EPILOGUE) {
     bool failed = false;
+    Walk w;
+    if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
     for (int jt = 0; jt < nt; ++jt) {
-      const int e = jt % kRB;
+      const int e = jt & (kRB - 1);
       const bool ok = mbar_wait(bar_pfull + 8 * e, (uint32_t)(jt / kRB) & 1u, failed);
       if (__any_sync(0xffffffffu, !ok)) {
-        if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+        if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
         failed = true;
       }
       if (!failed) {
+        const int ex = s_dist[w.j], chunk = w.sg - s_seg[w.j];
+        const int* pairs = s_list + s_start[ex] + chunk * CH;
+        const int np = min(CH, s_cnt[ex] - chunk * CH);
         if constexpr (C::ONE) {
-          // partials: [entry][consumer][16 rows] floats
+          // partials: [entry][consumer][matrix][16 rows] floats
           if (lane < 16) {
-            float y = 0.0f;
+            float y[NS];
 #pragma unroll
-            for (int w = 0; w < KC; ++w) y += ldsf(part_sa + (uint32_t)(((e * KC + w) * 16 + lane) * 4));
-            const int64_t row = (int64_t)(tb + jt) * 16 + lane;
-            if (row < p.N) store_as(p.out, p.out_dtype, row, y);
+            for (int ns = 0; ns < NS; ++ns) {
+              y[ns] = 0.0f;
+#pragma unroll
+              for (int wc = 0; wc < KC; ++wc)
+                y[ns] += ldsf(part_sa + (uint32_t)((((e * KC + wc) * NS + ns) * 16 + lane) * 4));
+            }
+            const float v = NS == 2 ? y[0] / (1.0f + expf(-y[0])) * y[NS - 1] : y[0];
+            const int64_t row = (int64_t)w.rt * 16 + lane;
+            if (row < q.n_rows) store_as(q.out, q.out_dtype, (int64_t)pairs[0] * q.out_ld + row, v);
           }
         } else {
-          // partials: [entry][consumer][token tile][lane] float4 (the mma C fragment)
-          for (int idx = lane; idx < 16 * p.M; idx += 32) {
+          // partials: [entry][consumer][matrix][token tile][lane] float4 (the mma C fragment)
+          for (int idx = lane; idx < 16 * np; idx += 32) {
             const int r = idx & 15, m = idx >> 4;
             const int mt = m >> 3, col = m & 7;
             const int src = ((r & 7) << 2) | (col >> 1);
             const int ci = ((r >> 3) << 1) | (col & 1);
-            const uint32_t a0 = part_sa + (uint32_t)((((e * KC) * MT + mt) * 32 + src) * 16 + ci * 4);
-            float y = 0.0f;
+            float y[NS];
 #pragma unroll
-            for (int w = 0; w < KC; ++w) y += ldsf(a0 + (uint32_t)(w * MT * 32 * 16));
-            const int64_t row = (int64_t)(tb + jt) * 16 + r;
-            if (row < p.N) store_as(p.out, p.out_dtype, (int64_t)m * p.out_ld + row, y);
+            for (int ns = 0; ns < NS; ++ns) {
+              const uint32_t a0 = part_sa + (uint32_t)(((((e * KC) * NS + ns) * MT + mt) * 32 + src) * 16 + ci * 4);
+              y[ns] = 0.0f;
+#pragma unroll
+              for (int wc = 0; wc < KC; ++wc) y[ns] += ldsf(a0 + (uint32_t)(wc * NS * MT * 32 * 16));
+            }
+            const float v = NS == 2 ? y[0] / (1.0f + expf(-y[0])) * y[NS - 1] : y[0];
+            const int64_t row = (int64_t)w.rt * 16 + r;
+            if (row < q.n_rows) store_as(q.out, q.out_dtype, (int64_t)pairs[m] * q.out_ld + row, v);
           }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pempty + 8 * e);
+      if (jt + 1 < nt) w.next(p.ntiles_e, s_seg, nd);
     }
     return;
   }
@@ -442,15 +497,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
   // --------------------------------------------------------------- consumers
   const int g = lane >> 2, t = lane & 3;
   const uint32_t xs_sa = smem_u32(xs), xsum_sa = smem_u32(xsum);
-  // this warp's groups of a unit: ug = warp * GPW + u
-  uint32_t xb[MT];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt) {
-    const int tr = (mt * 8 + g) < p.M ? mt * 8 + g : 0;  // idle columns reread token 0
-    xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
-             (uint32_t)(warp * GPW * C::XG);
-  }
-  // per-group sums: tokens 2t, 2t + 1 (token 0 only for a single token)
+  // per-group sums: pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
   const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 4);
   // shared offsets (within a slot) of this lane's code words, row g, per group u
   uint32_t coff[GPW];
@@ -462,38 +509,61 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
     coff[u] = (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
   }
   const uint32_t magic = p.magic;
-  // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's groups
-  // (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
+  // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
+  // groups (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
   constexpr int PITCH = GPU * 2;
   const int sfx = PITCH == 128 ? (g & 7) : PITCH == 64 ? ((g >> 1) & 3) : ((g >> 2) & 1);
   const int sbyte = warp * GPW * 2;
   const uint32_t soff = (uint32_t)(g * PITCH + ((((sbyte >> 4) ^ sfx)) << 4) + (sbyte & 15));
 
-  float acc[MT][4];
+  float acc[NS][MT][4];
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
+  for (int ns = 0; ns < NS; ++ns)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[mt][i] = 0.0f;
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[ns][mt][i] = 0.0f;
   bool failed = false;
 
   // unit i: slot i % STAGES with phase (i / STAGES) & 1, k-unit ku of tile jt
-  int slot = 0, ku = 0, jt = 0;
+  int slot = 0, ku = 0, jt = 0, cur_sg = -1;
   uint32_t phase = 0;
   uint32_t cslot = code_ring, sslot = sb_ring + soff, bfull = bar_full;
-  uint32_t xbu[MT];
+  uint32_t xb[MT], xbu[MT];
 #pragma unroll
-  for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
+  for (int mt = 0; mt < MT; ++mt) { xb[mt] = xs_sa; xbu[mt] = xs_sa; }
   uint32_t su = xsum_lane;
-  // one token: this warp's x fragments and group sums of the current k-unit,
-  // in registers (reloaded only when the k-unit changes)
+  // one pair: this warp's x fragments and group sums of the current k-unit,
+  // in registers (reloaded only when the k-unit or the segment changes)
   uint4 xr[C::ONE ? GPW : 1][S::kSteps / 2];
   float xsr[C::ONE ? GPW : 1][C::NX];
   int xku = -1;
+  Walk w;
+  if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
   for (int i = 0; i < nunits; ++i) {
+    if (ku == 0 && w.sg != cur_sg) {
+      // a new segment: stage the x rows of its pairs
+      asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
+      cur_sg = w.sg;
+      const int ex = s_dist[w.j], chunk = w.sg - s_seg[w.j];
+      const int np = min(CH, s_cnt[ex] - chunk * CH);
+      stage_x<S, T, TOKP, C::NX, KC * 32>(q, s_list + s_start[ex] + chunk * CH, np, Gpad, p.tok_stride, tid, xs,
+                                          xsum);
+      asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int tr = (mt * 8 + g) < np ? mt * 8 + g : 0;  // idle columns reread pair 0
+        xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
+                 (uint32_t)(warp * GPW * C::XG);
+        xbu[mt] = xb[mt];
+      }
+      su = xsum_lane;
+      xku = -1;
+    }
     bool ok = mbar_try_wait(bfull, phase);
     if (!ok) ok = mbar_wait(bfull, phase, failed);
     if (__any_sync(0xffffffffu, !ok)) {
-      if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+      if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
       failed = true;
     }
     if constexpr (C::ONE) {
@@ -509,84 +579,90 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
       }
     }
     if (!failed) {
-      // GPW 16-bit scales (biases) of rows g and g + 8
-      uint32_t sv[2][(GPW + 1) / 2], bv[2][(GPW + 1) / 2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t ra = sslot + (uint32_t)(h * 8 * GPU * 2);
-        if constexpr (GPW == 1) {
-          sv[h][0] = lds16(ra);
-          bv[h][0] = lds16(ra + C::SB_BYTES);
-        } else if constexpr (GPW == 2) {
-          sv[h][0] = lds32(ra);
-          bv[h][0] = lds32(ra + C::SB_BYTES);
-        } else {
+      for (int ns = 0; ns < NS; ++ns) {
+        const uint32_t csl = cslot + (uint32_t)(ns * C::CODE_BYTES);
+        const uint32_t ssl = sslot + (uint32_t)(ns * 2 * C::SB_BYTES);
+        // GPW 16-bit scales (biases) of rows g and g + 8
+        uint32_t sv[2][(GPW + 1) / 2], bv[2][(GPW + 1) / 2];
 #pragma unroll
-          for (int c = 0; c < GPW / 4; ++c) {
-            const uint2 s2 = lds64(ra + 8 * c), b2 = lds64(ra + C::SB_BYTES + 8 * c);
-            sv[h][2 * c] = s2.x; sv[h][2 * c + 1] = s2.y;
-            bv[h][2 * c] = b2.x; bv[h][2 * c + 1] = b2.y;
-          }
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < GPW; ++u) {
-        uint32_t rA[S::kRegs], rB[S::kRegs];
-        const uint32_t ca = cslot + coff[u];
-        if constexpr (S::kRegs >= 4) {
-          const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
-#pragma unroll
-          for (int k = 0; k < S::kRegs / 4; ++k) {
-            const uint32_t ch = (uint32_t)(((c0 ^ (uint32_t)g) + k) ^ (uint32_t)g);
-            const uint4 va = lds128(cbase + (ch << 4)), vb = lds128(cbase + 1024 + (ch << 4));
-            rA[4 * k] = va.x; rA[4 * k + 1] = va.y; rA[4 * k + 2] = va.z; rA[4 * k + 3] = va.w;
-            rB[4 * k] = vb.x; rB[4 * k + 1] = vb.y; rB[4 * k + 2] = vb.z; rB[4 * k + 3] = vb.w;
-          }
-        } else if constexpr (S::kRegs == 2) {
-          const uint2 va = lds64(ca), vb = lds64(ca + 1024);
-          rA[0] = va.x; rA[1] = va.y; rB[0] = vb.x; rB[1] = vb.y;
-        } else {
-          rA[0] = lds32(ca);
-          rB[0] = lds32(ca + 1024);
-        }
-        float d[MT][4];
-        if constexpr (C::ONE)
-          group_dot_rx<BITS, S, T>(rA, rB, xr[u], d[0], magic);
-        else
-          group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
-        const int hw = u & 1;
-        const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
-        const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          if constexpr (C::ONE) {
-            const float X0 = xsr[u][0];
-            if constexpr (C::NX == 1) {
-              acc[0][0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], acc[0][0]));
-              acc[0][2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], acc[0][2]));
-            } else {
-              const float O0 = xsr[u][C::NX - 1];
-              acc[0][0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], acc[0][0])));
-              acc[0][2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], acc[0][2])));
-            }
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t ra = ssl + (uint32_t)(h * 8 * PITCH);
+          if constexpr (GPW == 1) {
+            sv[h][0] = lds16(ra);
+            bv[h][0] = lds16(ra + C::SB_BYTES);
+          } else if constexpr (GPW == 2) {
+            sv[h][0] = lds32(ra);
+            bv[h][0] = lds32(ra + C::SB_BYTES);
           } else {
-            const uint2 xr = lds64(su + (uint32_t)((u * TOKP + mt * 8) * 4));
-            const float X0 = __uint_as_float(xr.x), X1 = __uint_as_float(xr.y);
-            if constexpr (C::NX == 1) {
-              const float ca_ = fmaf(-OFF, sa, ba), cb_ = fmaf(-OFF, sb_, bb);
-              acc[mt][0] = fmaf(ca_, X0, fmaf(sa, d[mt][0], acc[mt][0]));
-              acc[mt][1] = fmaf(ca_, X1, fmaf(sa, d[mt][1], acc[mt][1]));
-              acc[mt][2] = fmaf(cb_, X0, fmaf(sb_, d[mt][2], acc[mt][2]));
-              acc[mt][3] = fmaf(cb_, X1, fmaf(sb_, d[mt][3], acc[mt][3]));
+#pragma unroll
+            for (int c = 0; c < GPW / 4; ++c) {
+              const uint2 s2 = lds64(ra + 8 * c), b2 = lds64(ra + C::SB_BYTES + 8 * c);
+              sv[h][2 * c] = s2.x; sv[h][2 * c + 1] = s2.y;
+              bv[h][2 * c] = b2.x; bv[h][2 * c + 1] = b2.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < GPW; ++u) {
+          uint32_t rA[S::kRegs], rB[S::kRegs];
+          const uint32_t ca = csl + coff[u];
+          if constexpr (S::kRegs >= 4) {
+            const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
+#pragma unroll
+            for (int k = 0; k < S::kRegs / 4; ++k) {
+              const uint32_t ch = (uint32_t)(((c0 ^ (uint32_t)g) + k) ^ (uint32_t)g);
+              const uint4 va = lds128(cbase + (ch << 4)), vb = lds128(cbase + 1024 + (ch << 4));
+              rA[4 * k] = va.x; rA[4 * k + 1] = va.y; rA[4 * k + 2] = va.z; rA[4 * k + 3] = va.w;
+              rB[4 * k] = vb.x; rB[4 * k + 1] = vb.y; rB[4 * k + 2] = vb.z; rB[4 * k + 3] = vb.w;
+            }
+          } else if constexpr (S::kRegs == 2) {
+            const uint2 va = lds64(ca), vb = lds64(ca + 1024);
+            rA[0] = va.x; rA[1] = va.y; rB[0] = vb.x; rB[1] = vb.y;
+          } else {
+            rA[0] = lds32(ca);
+            rB[0] = lds32(ca + 1024);
+          }
+          float d[MT][4];
+          if constexpr (C::ONE)
+            group_dot_rx<BITS, S, T>(rA, rB, xr[u], d[0], magic);
+          else
+            group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
+          const int hw = u & 1;
+          const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
+          const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            float(&a_)[4] = acc[ns][mt];
+            if constexpr (C::ONE) {
+              const float X0 = xsr[u][0];
+              if constexpr (C::NX == 1) {
+                a_[0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], a_[0]));
+                a_[2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], a_[2]));
+              } else {
+                const float O0 = xsr[u][C::NX - 1];
+                a_[0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], a_[0])));
+                a_[2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], a_[2])));
+              }
             } else {
-              // bias term on sum(x), offset term on sum(x') (x' = x and 16 x)
-              const uint2 xo = lds64(su + (uint32_t)(((Gpad + u) * TOKP + mt * 8) * 4));
-              const float O0 = __uint_as_float(xo.x), O1 = __uint_as_float(xo.y);
-              const float oa = -OFF * sa, ob = -OFF * sb_;
-              acc[mt][0] = fmaf(ba, X0, fmaf(oa, O0, fmaf(sa, d[mt][0], acc[mt][0])));
-              acc[mt][1] = fmaf(ba, X1, fmaf(oa, O1, fmaf(sa, d[mt][1], acc[mt][1])));
-              acc[mt][2] = fmaf(bb, X0, fmaf(ob, O0, fmaf(sb_, d[mt][2], acc[mt][2])));
-              acc[mt][3] = fmaf(bb, X1, fmaf(ob, O1, fmaf(sb_, d[mt][3], acc[mt][3])));
+              const uint2 xr2 = lds64(su + (uint32_t)((u * TOKP + mt * 8) * 4));
+              const float X0 = __uint_as_float(xr2.x), X1 = __uint_as_float(xr2.y);
+              if constexpr (C::NX == 1) {
+                const float ca_ = fmaf(-OFF, sa, ba), cb_ = fmaf(-OFF, sb_, bb);
+                a_[0] = fmaf(ca_, X0, fmaf(sa, d[mt][0], a_[0]));
+                a_[1] = fmaf(ca_, X1, fmaf(sa, d[mt][1], a_[1]));
+                a_[2] = fmaf(cb_, X0, fmaf(sb_, d[mt][2], a_[2]));
+                a_[3] = fmaf(cb_, X1, fmaf(sb_, d[mt][3], a_[3]));
+              } else {
+                // bias term on sum(x), offset term on sum(x') (x' = x and 16 x)
+                const uint2 xo = lds64(su + (uint32_t)(((Gpad + u) * TOKP + mt * 8) * 4));
+                const float O0 = __uint_as_float(xo.x), O1 = __uint_as_float(xo.y);
+                const float oa = -OFF * sa, ob = -OFF * sb_;
+                a_[0] = fmaf(ba, X0, fmaf(oa, O0, fmaf(sa, d[mt][0], a_[0])));
+                a_[1] = fmaf(ba, X1, fmaf(oa, O1, fmaf(sa, d[mt][1], a_[1])));
+                a_[2] = fmaf(bb, X0, fmaf(ob, O0, fmaf(sb_, d[mt][2], a_[2])));
+                a_[3] = fmaf(bb, X1, fmaf(ob, O1, fmaf(sb_, d[mt][3], a_[3])));
+              }
             }
           }
         }
@@ -600,29 +676,33 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
       if (jt >= kRB) {
         const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / kRB) - 1) & 1u, failed);
         if (__any_sync(0xffffffffu, !okp)) {
-          if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+          if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
           failed = true;
         }
       }
-      if constexpr (C::ONE) {
-        if (t == 0) {
-          sts32(part_sa + (uint32_t)(((e * KC + warp) * 16 + g) * 4), acc[0][0]);
-          sts32(part_sa + (uint32_t)(((e * KC + warp) * 16 + g + 8) * 4), acc[0][2]);
+#pragma unroll
+      for (int ns = 0; ns < NS; ++ns) {
+        if constexpr (C::ONE) {
+          if (t == 0) {
+            sts32(part_sa + (uint32_t)((((e * KC + warp) * NS + ns) * 16 + g) * 4), acc[ns][0][0]);
+            sts32(part_sa + (uint32_t)((((e * KC + warp) * NS + ns) * 16 + g + 8) * 4), acc[ns][0][2]);
+          }
+        } else {
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+            sts128(part_sa + (uint32_t)(((((e * KC + warp) * NS + ns) * MT + mt) * 32 + lane) * 16),
+                   make_float4(acc[ns][mt][0], acc[ns][mt][1], acc[ns][mt][2], acc[ns][mt][3]));
         }
-      } else {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
-          sts128(part_sa + (uint32_t)((((e * KC + warp) * MT + mt) * 32 + lane) * 16),
-                 make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[ns][mt][k] = 0.0f;
       }
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[mt][k] = 0.0f;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_pfull + 8 * e);
       ku = 0;
       ++jt;
+      if (i + 1 < nunits) w.next(p.ntiles_e, s_seg, nd);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
       su = xsum_lane;
@@ -638,8 +718,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc,
       sslot = sb_ring + soff;
       bfull = bar_full;
     } else {
-      cslot += (uint32_t)C::CODE_BYTES;
-      sslot += (uint32_t)(2 * C::SB_BYTES);
+      cslot += (uint32_t)(NS * C::CODE_BYTES);
+      sslot += (uint32_t)(NS * 2 * C::SB_BYTES);
       bfull += 8;
     }
   }
@@ -674,43 +754,39 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
                                  : gpu * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Dense calls only (no ids, one matrix); cudaErrorNotSupported sends the caller
-// to the general kernels.
-template <int BITS, int GS, typename T, int MODE, int UG>
+// cudaErrorNotSupported sends the caller to the general kernels.
+template <int BITS, int GS, typename T, int MODE, int UG, int NS>
 cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
-  using C = Cfg<BITS, GS, T, MODE, UG>;
-  if (q.ids || q.amode != 0 || q.n_pairs < 1 || q.n_pairs > C::TOKP) return cudaErrorNotSupported;
-  if (q.G % 8 != 0 || q.wpr % 32 != 0 || q.n_rows < 16 || q.G < C::GPU) return cudaErrorNotSupported;
-  if (((uintptr_t)q.packed[0] | (uintptr_t)q.scales[0] | (uintptr_t)q.biases[0]) & 15) return cudaErrorNotSupported;
+  using C = Cfg<BITS, GS, T, MODE, UG, NS>;
+  const int64_t rows_total = q.n_rows * q.num_experts;
+  if (q.n_pairs < 1 || q.G % 8 != 0 || q.wpr % 32 != 0 || rows_total < 16 || q.G < C::GPU) return cudaErrorNotSupported;
+  if (rows_total + 16 >= ((int64_t)1 << 31) || (int64_t)q.n_pairs * q.K >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
+  for (int ns = 0; ns < NS; ++ns)
+    if (((uintptr_t)q.packed[ns] | (uintptr_t)q.scales[ns] | (uintptr_t)q.biases[ns]) & 15) return cudaErrorNotSupported;
 
   Params p{};
-  p.x = q.a;
-  p.M = q.n_pairs;
-  p.K = q.K;
-  p.G = q.G;
+  p.q = q;
   p.upt = (q.G + C::GPU - 1) / C::GPU;
-  p.N = q.n_rows;
-  p.ntiles = (int)((q.n_rows + 15) / 16);
-  p.out = q.out;
-  p.out_dtype = q.out_dtype;
-  p.out_ld = q.out_ld;
-  p.d_status = q.d_status;
+  p.ntiles_e = (int)((q.n_rows + 15) / 16);
+  p.CH = C::CH;
   p.magic = C::S::kMagic;
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
-  // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums]
-  const size_t part = C::ONE ? (size_t)kRB * C::KC * 16 * 4 : (size_t)kRB * C::KC * C::MT * 32 * 16;
-  const size_t xs = align128((size_t)p.M * p.tok_stride);
+  // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums | plan]
+  const size_t part = C::ONE ? (size_t)kRB * C::KC * NS * 16 * 4 : (size_t)kRB * C::KC * NS * C::MT * 32 * 16;
+  const size_t xs = align128((size_t)C::CH * p.tok_stride);
   const size_t xsum = align128((size_t)Gpad * C::TOKP * 4 * C::NX);
   const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
+  const size_t plan = align128((size_t)(5 * q.num_experts + 1 + q.n_pairs) * sizeof(int));
+  if (plan > 32 * 1024) return cudaErrorNotSupported;
   auto total = [&](int stages) {
-    return 1024 + (size_t)stages * C::CODE_BYTES + align128((size_t)stages * 2 * C::SB_BYTES) + align128(bars) +
-           part + xs + xsum;
+    return 1024 + (size_t)stages * NS * C::CODE_BYTES + align128((size_t)stages * NS * 2 * C::SB_BYTES) +
+           align128(bars) + part + xs + xsum + plan;
   };
   // about 144 KB of the weight stream in flight per SM (measured: deeper rings
   // and an L2 prefetch window ahead of the ring were not faster)
@@ -719,21 +795,24 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   while (stages > 2 && total(stages) > (size_t)kSmemMax) --stages;
   if (total(stages) > (size_t)kSmemMax) return cudaErrorNotSupported;
   p.stages = stages;
-  p.pf = 0;  // L2 prefetch window (units); off: measured no faster than the ring alone
   p.off_code = 0;
-  p.off_sb = stages * C::CODE_BYTES;
-  p.off_bar = p.off_sb + (int)align128((size_t)stages * 2 * C::SB_BYTES);
+  p.off_sb = stages * NS * C::CODE_BYTES;
+  p.off_bar = p.off_sb + (int)align128((size_t)stages * NS * 2 * C::SB_BYTES);
   p.off_part = p.off_bar + (int)align128(bars);
   p.off_xs = p.off_part + (int)part;
   p.off_xsum = p.off_xs + (int)xs;
+  p.off_plan = p.off_xsum + (int)xsum;
   const size_t smem = total(stages);
 
-  CUtensorMap tmc, tms, tmb;
-  if (!make_code_map3(&tmc, q.packed[0], q.n_rows, q.wpr, C::Z) ||
-      !make_sb_map(&tms, q.scales[0], q.n_rows, q.G, C::GPU) || !make_sb_map(&tmb, q.biases[0], q.n_rows, q.G, C::GPU))
-    return cudaErrorNotSupported;
+  CUtensorMap tm[6];
+  for (int ns = 0; ns < NS; ++ns)
+    if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z) ||
+        !make_sb_map(&tm[3 * ns + 1], q.scales[ns], rows_total, q.G, C::GPU) ||
+        !make_sb_map(&tm[3 * ns + 2], q.biases[ns], rows_total, q.G, C::GPU))
+      return cudaErrorNotSupported;
+  if (NS == 1) { tm[3] = tm[0]; tm[4] = tm[1]; tm[5] = tm[2]; }
 
-  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG>;
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -743,7 +822,9 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  const int grid = std::min(qmm_host::num_sms(), p.ntiles);
+  // dense calls have ceil(N / 16) tiles; the MoE work list is only known on
+  // the device, so those calls take one CTA per SM
+  const int grid = q.ids ? qmm_host::num_sms() : std::min(qmm_host::num_sms(), p.ntiles_e);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::THREADS);
@@ -754,40 +835,51 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, p, tmc, tms, tmb);
+  return cudaLaunchKernelEx(&cfg, k, p, tm[0], tm[1], tm[2], tm[3], tm[4], tm[5]);
 }
 
+// Instantiation for one (bits, group size, dtype): the unit width and mode.
+// Dense calls: one token -> mode 0, up to 8 -> 1, up to 16 -> 2.  MoE calls:
+// one activation row per expert is the common case for a single token, so
+// mode 0 when n_pairs <= 8, otherwise segments of up to 8 pairs (mode 1).
 template <int BITS, int GS, typename T>
-cudaError_t try_stream_mt(const QgemvParams& q, int mt, cudaStream_t st) {
+cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t st) {
   using S = Share<BITS, GS, T>;
   if constexpr (S::kFast) {
     constexpr int WPG = S::kWordsPerGroup;
-    constexpr int UB = WPG >= 32 ? 16 : 32;           // base unit
-    constexpr int UW = WPG <= 8 ? 64 : UB;            // wide unit: 4 groups per consumer
+    constexpr int UB = WPG >= 32 ? 16 : 32;  // base unit
+    constexpr int UW = WPG <= 8 ? 64 : UB;   // wide unit: 4 groups per consumer
+    if (dual) {
+      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 2>(q, st);
+      return launch_stream<BITS, GS, T, 1, UB, 2>(q, st);
+    }
+    if (q.ids) {
+      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 1>(q, st);
+      return launch_stream<BITS, GS, T, 1, UB, 1>(q, st);
+    }
     const bool wide = (q.G % UW) == 0;
     if (q.n_pairs == 1)
-      return wide ? launch_stream<BITS, GS, T, 0, UW>(q, st) : launch_stream<BITS, GS, T, 0, UB>(q, st);
+      return wide ? launch_stream<BITS, GS, T, 0, UW, 1>(q, st) : launch_stream<BITS, GS, T, 0, UB, 1>(q, st);
     if (mt == 1)
-      return wide ? launch_stream<BITS, GS, T, 1, UW>(q, st) : launch_stream<BITS, GS, T, 1, UB>(q, st);
-    return launch_stream<BITS, GS, T, 2, UB>(q, st);
+      return wide ? launch_stream<BITS, GS, T, 1, UW, 1>(q, st) : launch_stream<BITS, GS, T, 1, UB, 1>(q, st);
+    return launch_stream<BITS, GS, T, 2, UB, 1>(q, st);
   } else {
     return cudaErrorNotSupported;
   }
 }
 
-// Entry from the per-bit-width files: the streaming kernel for dense calls of
-// one matrix, cudaErrorNotSupported for everything else.
+// Entry from the per-bit-width files; cudaErrorNotSupported for shapes the
+// streaming kernel does not take.
 template <int BITS>
 cudaError_t try_stream(const QgemvParams& q, int gs, int dtype, int mt, bool dual, cudaStream_t st) {
-  if (dual || q.ids) return cudaErrorNotSupported;
   if (dtype == QMM_BF16) {
-    if (gs == 32) return try_stream_mt<BITS, 32, __nv_bfloat16>(q, mt, st);
-    if (gs == 64) return try_stream_mt<BITS, 64, __nv_bfloat16>(q, mt, st);
-    return try_stream_mt<BITS, 128, __nv_bfloat16>(q, mt, st);
+    if (gs == 32) return try_stream_t<BITS, 32, __nv_bfloat16>(q, mt, dual, st);
+    if (gs == 64) return try_stream_t<BITS, 64, __nv_bfloat16>(q, mt, dual, st);
+    return try_stream_t<BITS, 128, __nv_bfloat16>(q, mt, dual, st);
   }
-  if (gs == 32) return try_stream_mt<BITS, 32, __half>(q, mt, st);
-  if (gs == 64) return try_stream_mt<BITS, 64, __half>(q, mt, st);
-  return try_stream_mt<BITS, 128, __half>(q, mt, st);
+  if (gs == 32) return try_stream_t<BITS, 32, __half>(q, mt, dual, st);
+  if (gs == 64) return try_stream_t<BITS, 64, __half>(q, mt, dual, st);
+  return try_stream_t<BITS, 128, __half>(q, mt, dual, st);
 }
 
 }  // namespace stream
