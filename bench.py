@@ -173,7 +173,7 @@ def job_throughput(bytes_per_step: float, steps: int, world: int, ms_max: float)
 # ---------------------------------------------------------------- traffic record
 def traffic_record(name):
     """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (sha256 of the .cu file recorded in the summary)."""
+    the current kernel sources (sha256 of each file listed in the summary)."""
     path = os.path.join(ROOT, "profiles", name)
     try:
         txt = open(path).read()
@@ -184,15 +184,17 @@ def traffic_record(name):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             rec[k.strip()] = v.strip()
-    src = rec.get("source_file")
-    if not src:
+    srcs = [x.strip() for x in rec.get("source_files", "").split(",") if x.strip()]
+    shas = [x.strip() for x in rec.get("source_sha256", "").split(",") if x.strip()]
+    if not srcs or len(srcs) != len(shas):
         return None, None
-    try:
-        cur = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
-    except OSError:
-        return None, None
-    if cur != rec.get("source_sha256"):
-        return None, "stale"
+    for src, sha in zip(srcs, shas):
+        try:
+            cur = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()
+        except OSError:
+            return None, None
+        if cur != sha:
+            return None, "stale"
     return rec, "current"
 
 
@@ -357,7 +359,7 @@ def run_ours(args):
                    "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                     "peak_source": peak_src, "kernel": "qgemv_stream_kernel<4,64,bf16,1>",
+                     "peak_source": peak_src, "kernel": "qgemv_stream_kernel<4,64,bf16,0,64|32,1> (one token; 64- or 32-group units)",
                      "per_shape": per_shape},
         "e2e": e2e,
         "gpu_launches": steps * launches_per_step,

@@ -369,15 +369,28 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // the ids (like x) may come from the previous kernel in the stream
-  if (q.ids) asm volatile("griddepcontrol.wait;" ::: "memory");
-  build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
-  if (tid == 0) {
-    int run = 0;
-    s_seg[0] = 0;
-    for (int j = 0; j < s_nd; ++j) {
-      run += (s_cnt[s_dist[j]] + CH - 1) / CH;
-      s_seg[j + 1] = run;
+  if (q.ids) {
+    // the ids (like x) may come from the previous kernel in the stream
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
+    if (tid == 0) {
+      int run = 0;
+      s_seg[0] = 0;
+      for (int j = 0; j < s_nd; ++j) {
+        run += (s_cnt[s_dist[j]] + CH - 1) / CH;
+        s_seg[j + 1] = run;
+      }
+    }
+  } else {
+    // dense: one expert holding the M tokens, nothing to sort
+    if (tid < q.n_pairs) s_list[tid] = tid;
+    if (tid == 0) {
+      s_cnt[0] = q.n_pairs;
+      s_start[0] = 0;
+      s_dist[0] = 0;
+      s_nd = 1;
+      s_seg[0] = 0;
+      s_seg[1] = (q.n_pairs + CH - 1) / CH;
     }
   }
   __syncthreads();
@@ -499,15 +512,20 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   const uint32_t xs_sa = smem_u32(xs), xsum_sa = smem_u32(xsum);
   // per-group sums: pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
   const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 4);
-  // shared offsets (within a slot) of this lane's code words, row g, per group u
-  uint32_t coff[GPW];
-#pragma unroll
-  for (int u = 0; u < GPW; ++u) {
-    const int ug = warp * GPW + u;
-    const int w0 = ug * WPG + t * S::kRegs;  // first word in the unit row
+  // shared offset (within a slot) of this lane's code words, row g, for group
+  // u: coff(u).  When a warp's groups share one 128-byte slice and the group
+  // step only touches chunk bits above the lane's own, coff(u) is coff(0) with
+  // those chunk bits flipped (no per-group register).
+  constexpr bool kXorGroups = (GPW * WPG <= 32) && (32 % (GPW * WPG) == 0) && (WPG % 4 == 0) &&
+                              (S::kRegs <= 4) && ((WPG / 4) & (4 * S::kRegs / 4 - 1)) == 0;
+  auto coff_of = [&](int u) -> uint32_t {
+    const int w0 = (warp * GPW + u) * WPG + t * S::kRegs;  // first word in the unit row
     const int wb = w0 & 31;
-    coff[u] = (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
-  }
+    return (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
+  };
+  uint32_t coff[kXorGroups ? 1 : GPW];
+#pragma unroll
+  for (int u = 0; u < (kXorGroups ? 1 : GPW); ++u) coff[u] = coff_of(u);
   const uint32_t magic = p.magic;
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
   // groups (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
@@ -606,7 +624,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
         for (int u = 0; u < GPW; ++u) {
           uint32_t rA[S::kRegs], rB[S::kRegs];
-          const uint32_t ca = csl + coff[u];
+          const uint32_t ca = kXorGroups ? csl + (coff[0] ^ (uint32_t)((u * (WPG / 4)) << 4)) : csl + coff[kXorGroups ? 0 : u];
           if constexpr (S::kRegs >= 4) {
             const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
 #pragma unroll
