@@ -357,6 +357,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   int* s_seg = s_dist + E;  // E + 1 entries
   int* s_list = s_seg + E + 1;
   __shared__ int s_nd;
+  __shared__ int64_t s_xoff[16];  // activation row offsets of the staged x rows
 
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -544,7 +545,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   bool failed = false;
 
   // unit i: slot i % STAGES with phase (i / STAGES) & 1, k-unit ku of tile jt
-  int slot = 0, ku = 0, jt = 0, cur_sg = -1;
+  int slot = 0, ku = 0, jt = 0, cur_sg = -1, cur_np = -1;
   uint32_t phase = 0;
   uint32_t cslot = code_ring, sslot = sb_ring + soff, bfull = bar_full;
   uint32_t xb[MT], xbu[MT];
@@ -560,23 +561,30 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
   for (int i = 0; i < nunits; ++i) {
     if (ku == 0 && w.sg != cur_sg) {
-      // a new segment: stage the x rows of its pairs
-      asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
+      // a new segment: stage the x rows of its pairs, unless they are the rows
+      // already staged (one token routed to several experts)
       cur_sg = w.sg;
       const int ex = s_dist[w.j], chunk = w.sg - s_seg[w.j];
       const int np = min(CH, s_cnt[ex] - chunk * CH);
-      stage_x<S, T, TOKP, C::NX, KC * 32>(q, s_list + s_start[ex] + chunk * CH, np, Gpad, p.tok_stride, tid, xs,
-                                          xsum);
-      asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
+      const int* pn = s_list + s_start[ex] + chunk * CH;
+      bool same = np == cur_np;
+      for (int m = 0; m < np && same; ++m) same = pair_offset(q, pn[m]) == s_xoff[m];
+      if (!same) {
+        asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
+        stage_x<S, T, TOKP, C::NX, KC * 32>(q, pn, np, Gpad, p.tok_stride, tid, xs, xsum);
+        if (tid < np) s_xoff[tid] = pair_offset(q, pn[tid]);
+        cur_np = np;
+        asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int tr = (mt * 8 + g) < np ? mt * 8 + g : 0;  // idle columns reread pair 0
-        xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
-                 (uint32_t)(warp * GPW * C::XG);
-        xbu[mt] = xb[mt];
+        for (int mt = 0; mt < MT; ++mt) {
+          const int tr = (mt * 8 + g) < np ? mt * 8 + g : 0;  // idle columns reread pair 0
+          xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
+                   (uint32_t)(warp * GPW * C::XG);
+          xbu[mt] = xb[mt];
+        }
+        su = xsum_lane;
+        xku = -1;
       }
-      su = xsum_lane;
-      xku = -1;
     }
     bool ok = mbar_try_wait(bfull, phase);
     if (!ok) ok = mbar_wait(bfull, phase, failed);
