@@ -215,13 +215,21 @@ __device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[S::kRegs], c
     word_pairs<S>(rawA[k], magic, pA + k * NP);
     word_pairs<S>(rawB[k], magic, pB + k * NP);
   }
+  // even and odd k16 steps in two chains (half the dependent mma latency);
+  // only columns 0 (rows g, g + 8: d[0], d[2]) are merged, the others are idle
+  float e[4];
 #pragma unroll
   for (int q = 0; q < S::kSteps; ++q) {
     const uint32_t b0 = (q & 1) ? bf[q >> 1].z : bf[q >> 1].x, b1 = (q & 1) ? bf[q >> 1].w : bf[q >> 1].y;
-    if (q == 0)
-      mma_first<T>(d, pA[0], pB[0], pA[1], pB[1], b0, b1);
+    float(&acc)[4] = (q & 1) ? e : d;
+    if (q < 2)
+      mma_first<T>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
     else
-      mma16816<T>(d, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+      mma16816<T>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+  }
+  if constexpr (S::kSteps > 1) {
+    d[0] += e[0];
+    d[2] += e[2];
   }
 }
 
