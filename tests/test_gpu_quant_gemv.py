@@ -108,6 +108,37 @@ def test_gemv_ragged_shapes(N, K):
     rne_equal(y16, y32)
 
 
+# Rows the streaming kernel takes (2/4/8-bit whole-word lanes, rows of whole
+# 128-byte slices, K/gs a multiple of 8 and at least one unit): every mode
+# (one token, up to 8, up to 16), unit widths 16/32/64 groups, the two-nibble
+# 8-bit bf16 form, a ragged last row tile (N = 200) and a partly filled last
+# unit (K = 2560 at g64: 40 groups = 32 + 8).
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("gs", GROUPS)
+@pytest.mark.parametrize("M", [1, 3, 12])
+def test_gemv_streaming_kernel_shapes(bits, gs, M):
+    y32, y16, yref = _gemv_case(M, 200, 4096, bits, gs, torch.bfloat16, 600 + 10 * bits + gs + M)
+    gate(y32.cpu().numpy(), yref, f"stream b{bits} g{gs} M{M}")
+    rne_equal(y16, y32)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemv_streaming_partial_unit_fp16(M, bits):
+    y32, y16, yref = _gemv_case(M, 333, 2560, bits, 64, torch.float16, 700 + M + bits)
+    gate(y32.cpu().numpy(), yref, f"stream f16 b{bits} M{M} K=2560")
+    rne_equal(y16, y32)
+
+
+def test_gemv_streaming_deterministic():
+    """Identical calls give identical bits (fixed reduction order)."""
+    w, qw, _ = _quant_pair(14336 // 8, 4096, 4, 64, torch.bfloat16, 800)
+    x = wl.gen_x(1, 4096, 801).to(DEV)
+    ys = [api.qmm_matmul(x, qw, True, torch.float32) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+
+
 def test_gemv_long_k_chunks_x_staging():
     """M=16 with K large enough that staged x is split into several K chunks."""
     y32, y16, yref = _gemv_case(16, 64, 8192, 8, 32, torch.bfloat16, 500)

@@ -396,7 +396,7 @@ inline bool make_code_map(CUtensorMap* map, const uint32_t* packed, int64_t rows
 }
 
 template <int BITS, int GS, typename T, int MT, bool DUAL>
-cudaError_t launch_tma_one(QgemvParams prm, int64_t rows_total, cudaStream_t st) {
+cudaError_t launch_tma_impl(QgemvParams prm, int64_t rows_total, cudaStream_t st) {
   using C = TmaCfg<BITS, GS, T, MT, DUAL>;
   using S = typename C::S;
   CUtensorMap tm[2];
@@ -450,6 +450,17 @@ cudaError_t launch_tma_one(QgemvParams prm, int64_t rows_total, cudaStream_t st)
   }
   k<<<grid, kThreads, smem, st>>>(prm, tm[0], tm[1]);
   return cudaGetLastError();
+}
+
+// The swizzled box reader takes whole-word shares only (2-bit g32 shares are
+// half a word): other layouts go to the cp.async kernel.
+template <int BITS, int GS, typename T, int MT, bool DUAL>
+cudaError_t launch_tma_one(QgemvParams prm, int64_t rows_total, cudaStream_t st) {
+  if constexpr (!Share<BITS, GS, T>::kAligned) {
+    return cudaErrorNotSupported;
+  } else {
+    return launch_tma_impl<BITS, GS, T, MT, DUAL>(prm, rows_total, st);
+  }
 }
 
 }  // namespace qmm
