@@ -130,6 +130,18 @@ def test_gemv_streaming_partial_unit_fp16(M, bits):
     rne_equal(y16, y32)
 
 
+@pytest.mark.parametrize("K", [768, 1280])
+@pytest.mark.parametrize("M", [1, 6, 16])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_gemv_streaming_short_rows_cp_async_scales(K, M, dtype):
+    """K/gs = 12 or 20 groups (even, not a multiple of 8): the scale and bias
+    rows are not 16-byte strided, so they stream by 4-byte copies into 16-group
+    units, the last one partly filled."""
+    y32, y16, yref = _gemv_case(M, 150, K, 4, 64, dtype, 900 + K + M)
+    gate(y32.cpu().numpy(), yref, f"stream K={K} M{M}")
+    rne_equal(y16, y32)
+
+
 def test_gemv_streaming_deterministic():
     """Identical calls give identical bits (fixed reduction order)."""
     w, qw, _ = _quant_pair(14336 // 8, 4096, 4, 64, torch.bfloat16, 800)
