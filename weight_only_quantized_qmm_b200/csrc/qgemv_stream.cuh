@@ -64,7 +64,7 @@ struct Params {
 // MODE 0: one pair per segment; 1: up to 8; 2: up to 16.  UG: groups per unit
 // (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
 // matrices per pair (2: gate and up).
-template <int BITS, int GS, typename T, int MODE, int UG, int NS>
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
 struct Cfg {
   using S = Share<BITS, GS, T>;
   static constexpr int MT = MODE == 2 ? 2 : 1;
@@ -100,15 +100,6 @@ __device__ __forceinline__ void sts128(uint32_t a, float4 v) {
 __device__ __forceinline__ float ldsf(uint32_t a) { return __uint_as_float(lds32(a)); }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
-               "r"(z)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
-               : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
                                             uint32_t bar) {
@@ -334,12 +325,12 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     if (idx % TOKP >= np) xsum[idx] = 0.0f;
 }
 
-template <int BITS, int GS, typename T, int MODE, int UG, int NS>
-__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS>::THREADS, 1)
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
+__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS, MOE>::THREADS, 1)
 qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, const __grid_constant__ CUtensorMap tms0,
                     const __grid_constant__ CUtensorMap tmb0, const __grid_constant__ CUtensorMap tmc1,
                     const __grid_constant__ CUtensorMap tms1, const __grid_constant__ CUtensorMap tmb1) {
-  using C = Cfg<BITS, GS, T, MODE, UG, NS>;
+  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE>;
   using S = typename C::S;
   constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC, CH = C::CH;
   constexpr float OFF = S::kOff;
@@ -565,17 +556,23 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   uint4 xr[C::ONE ? GPW : 1][S::kSteps / 2];
   float xsr[C::ONE ? GPW : 1][C::NX];
   int xku = -1;
-  Walk w;
-  if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
+  Walk w;  // the work-list walk of MoE calls (a dense call is one segment)
+  if constexpr (MOE) {
+    if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
+  }
   for (int i = 0; i < nunits; ++i) {
-    if (ku == 0 && w.sg != cur_sg) {
+    if (MOE ? (ku == 0 && w.sg != cur_sg) : i == 0) {
       // a new segment: stage the x rows of its pairs, unless they are the rows
       // already staged (one token routed to several experts)
-      cur_sg = w.sg;
-      const int ex = s_dist[w.j], chunk = w.sg - s_seg[w.j];
+      int ex = 0, chunk = 0;
+      if constexpr (MOE) {
+        cur_sg = w.sg;
+        ex = s_dist[w.j];
+        chunk = w.sg - s_seg[w.j];
+      }
       const int np = min(CH, s_cnt[ex] - chunk * CH);
       const int* pn = s_list + s_start[ex] + chunk * CH;
-      bool same = np == cur_np;
+      bool same = MOE && np == cur_np;
       for (int m = 0; m < np && same; ++m) same = pair_offset(q, pn[m]) == s_xoff[m];
       if (!same) {
         asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
@@ -736,7 +733,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       if (lane == 0) mbar_arrive(bar_pfull + 8 * e);
       ku = 0;
       ++jt;
-      if (i + 1 < nunits) w.next(p.ntiles_e, s_seg, nd);
+      if constexpr (MOE) {
+        if (i + 1 < nunits) w.next(p.ntiles_e, s_seg, nd);
+      }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
       su = xsum_lane;
@@ -793,9 +792,10 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
 }
 
 // cudaErrorNotSupported sends the caller to the general kernels.
-template <int BITS, int GS, typename T, int MODE, int UG, int NS>
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
 cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
-  using C = Cfg<BITS, GS, T, MODE, UG, NS>;
+  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE>;
+  if (MOE != (q.ids != nullptr)) return cudaErrorNotSupported;
   const int64_t rows_total = q.n_rows * q.num_experts;
   if (q.n_pairs < 1 || q.G % 8 != 0 || q.wpr % 32 != 0 || rows_total < 16 || q.G < C::GPU) return cudaErrorNotSupported;
   if (rows_total + 16 >= ((int64_t)1 << 31) || (int64_t)q.n_pairs * q.K >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
@@ -846,7 +846,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
       return cudaErrorNotSupported;
   if (NS == 1) { tm[3] = tm[0]; tm[4] = tm[1]; tm[5] = tm[2]; }
 
-  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS>;
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS, MOE>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -884,19 +884,19 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
     constexpr int UB = WPG >= 32 ? 16 : 32;  // base unit
     constexpr int UW = WPG <= 8 ? 64 : UB;   // wide unit: 4 groups per consumer
     if (dual) {
-      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 2>(q, st);
-      return launch_stream<BITS, GS, T, 1, UB, 2>(q, st);
+      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 2, true>(q, st);
+      return launch_stream<BITS, GS, T, 1, UB, 2, true>(q, st);
     }
     if (q.ids) {
-      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 1>(q, st);
-      return launch_stream<BITS, GS, T, 1, UB, 1>(q, st);
+      if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 1, true>(q, st);
+      return launch_stream<BITS, GS, T, 1, UB, 1, true>(q, st);
     }
     const bool wide = (q.G % UW) == 0;
     if (q.n_pairs == 1)
-      return wide ? launch_stream<BITS, GS, T, 0, UW, 1>(q, st) : launch_stream<BITS, GS, T, 0, UB, 1>(q, st);
+      return wide ? launch_stream<BITS, GS, T, 0, UW, 1, false>(q, st) : launch_stream<BITS, GS, T, 0, UB, 1, false>(q, st);
     if (mt == 1)
-      return wide ? launch_stream<BITS, GS, T, 1, UW, 1>(q, st) : launch_stream<BITS, GS, T, 1, UB, 1>(q, st);
-    return launch_stream<BITS, GS, T, 2, UB, 1>(q, st);
+      return wide ? launch_stream<BITS, GS, T, 1, UW, 1, false>(q, st) : launch_stream<BITS, GS, T, 1, UB, 1, false>(q, st);
+    return launch_stream<BITS, GS, T, 2, UB, 1, false>(q, st);
   } else {
     return cudaErrorNotSupported;
   }
