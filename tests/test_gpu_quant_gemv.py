@@ -241,3 +241,42 @@ def test_decode_full_size_sampled(case):
     rows = rng.integers(0, case.N, 64)
     pr, sr, br = oracle.quantize(w.numpy()[rows], oracle.F32, case.group_size, case.bits, oracle.BF16)
     assert np.array_equal(p[rows], pr) and np.array_equal(s[rows], sr) and np.array_equal(b[rows], br)
+
+
+_SWEEP_W = {}
+
+
+def _sweep_weight(bits, gs, seed):
+    """8192 x 8192 weights quantized once per (bits, group size); reused over M."""
+    key = (bits, gs)
+    if key not in _SWEEP_W:
+        _SWEEP_W.clear()  # hold one matrix at a time
+        w = wl.gen_weight(8192, 8192, seed)
+        qw = api.qmm_quantize(w.to(DEV), gs, bits, torch.bfloat16)
+        torch.cuda.synchronize()
+        _SWEEP_W[key] = (w, qw, qweight_np(qw))
+    return _SWEEP_W[key]
+
+
+@pytest.mark.parametrize("case", wl.WORKLOADS.sweep, ids=lambda c: c.name)
+def test_sweep_full_size_sampled(case):
+    """Bit-width sweep at full size (N = K = 8192, b in {2,3,6,8}, gs in
+    {32,64,128}, M in {1,4,16}): all rows of the output at 128 sampled columns
+    against the oracle, 16-bit output = RNE of the fp32 output, and a spot
+    check of the quantizer."""
+    w, qw, (p, s, b) = _sweep_weight(case.bits, case.group_size, 2000 + 100 * case.bits + case.group_size)
+    x = wl.gen_x(case.M, case.K, case.seed + 1)
+    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
+    y16 = api.qmm_matmul(x.to(DEV), qw)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(case.seed)
+    cols = np.unique(np.concatenate([rng.integers(0, case.N, 126), [0, case.N - 1]]))
+    coords = [(m, int(n)) for m in range(case.M) for n in cols]
+    yref = oracle.matmul_elements(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
+                                  case.group_size, case.bits, coords)
+    ys = y32.cpu().numpy()[:, cols].reshape(-1)
+    gate(ys, yref, case.name)
+    rne_equal(y16, y32)
+    rows = rng.integers(0, case.N, 16)
+    pr, sr, br = oracle.quantize(w.numpy()[rows], oracle.F32, case.group_size, case.bits, oracle.BF16)
+    assert np.array_equal(p[rows], pr) and np.array_equal(s[rows], sr) and np.array_equal(b[rows], br)
