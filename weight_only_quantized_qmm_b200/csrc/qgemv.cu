@@ -1,6 +1,10 @@
 // Entry of the decode GEMV / MoE kernel family: picks the instantiation
-// (bits, group size, dtype, token tiles, fused gate+up).  The kernels live in
-// qgemv_impl.cuh; qgemv_b{2,3,4,6,8}.cu instantiate them per bit width.
+// (bits, group size, dtype, token tiles, fused gate+up).  qgemv_b{2,3,4,6,8}.cu
+// instantiate the kernels per bit width and try, in order: the streaming kernel
+// (qgemv_stream.cuh: 2/4/8-bit whole-word lanes, rows of whole 128-byte slices,
+// K / gs a multiple of 8), the per-warp TMA kernel (qgemv_tma.cuh: 2/4/8-bit
+// whole-word shares, 16-byte rows), and the cp.async kernel (qgemv_impl.cuh:
+// every other shape, including 3- and 6-bit codes).
 #include <algorithm>
 
 #include <cuda.h>

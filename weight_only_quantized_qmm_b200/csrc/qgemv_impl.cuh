@@ -1,5 +1,8 @@
 // Decode-shaped quantized matmul (M <= 16) and the MoE indirect-dispatch GEMV,
-// dense and fused gate+up+SiLU, in one kernel family.
+// dense and fused gate+up+SiLU, in one kernel family: the shared pieces (the
+// share layout, conversions, x staging, the expert plan) and the cp.async
+// kernel that serves every shape the streaming and TMA kernels decline
+// (3- and 6-bit codes, half-word shares, short rows).
 //
 // What is computed:
 //   dense   y[m, n]   = sum_k x[m, k] * w_hat[n, k]

@@ -5,9 +5,11 @@
 // cp.async.  Only the copy mechanism differs: the arithmetic (tensor-core
 // partial dots per group, s_g fold, bias/offset correction mma) is the same.
 //
-// Used when the rows of the packed matrix start on 16-byte boundaries
-// (K * bits / 8 % 16 == 0) and codes are 2, 4 or 8 bits wide (a group is then
-// a power-of-two number of words, so one box row holds whole groups).
+// Used for the shapes the streaming kernel (qgemv_stream.cuh) declines, when
+// the rows of the packed matrix start on 16-byte boundaries
+// (K * bits / 8 % 16 == 0) and codes are 2, 4 or 8 bits wide with whole-word
+// shares (a group is then a power-of-two number of words, so one box row
+// holds whole groups) -- e.g. the MoE down projection at K / gs = 12.
 #pragma once
 
 #include <cuda.h>
