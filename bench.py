@@ -415,29 +415,40 @@ def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
             stacks.append((api.ExpertStack.from_qweight(g, E), api.ExpertStack.from_qweight(u, E),
                            api.ExpertStack.from_qweight(d, E)))
         a = wl.gen_x(T, dm, case.seed + 3).to(dev).reshape(-1)
-        ids = wl.gen_moe_ids(T, E, k, case.seed + 4)
-        n_dist = len(np.unique(ids.numpy()))
-        ids = ids.to(dev)
+        # id sets rotate with the weight sets so that the experts a call reads
+        # are not still in L2 from the previous calls: for one token, 16
+        # disjoint sets of 8 cover all 128 experts; otherwise independent draws
+        n_ids = 16
+        if T == 1:
+            perm = torch.randperm(E, generator=torch.Generator().manual_seed(case.seed + 4)).to(torch.int32)
+            id_sets = [perm[i * k:(i + 1) * k].reshape(1, k) for i in range(E // k)][:n_ids]
+        else:
+            id_sets = [wl.gen_moe_ids(T, E, k, case.seed + 4 + 100 * i) for i in range(n_ids)]
+        n_dist = float(np.mean([len(np.unique(x.numpy())) for x in id_sets]))
+        id_sets = [x.to(dev) for x in id_sets]
         h = torch.empty(T * k, dff, dtype=torch.bfloat16, device=dev)
         o = torch.empty(T * k, dm, dtype=torch.bfloat16, device=dev)
         it = [0]
 
         def gu():
             g, u, _ = stacks[it[0] % n_sets]
+            ids = id_sets[it[0] % n_ids]
             it[0] += 1
             api.qmm_moe_gemv_id_gate_up_silu_batched(a, ids, T, k, dm, 0, g, u, out=h, stream=stream)
 
         def dn():
             _, _, d = stacks[it[0] % n_sets]
+            ids = id_sets[it[0] % n_ids]
             it[0] += 1
             api.qmm_moe_gemv_id(h.reshape(-1), ids.reshape(-1), T * k, dff, d, out=o, stream=stream)
-        t_gu = time_graph(torch, gu, stream, inner=n_sets)
-        t_dn = time_graph(torch, dn, stream, inner=n_sets)
+        t_gu = time_graph(torch, gu, stream, inner=n_ids)
+        t_dn = time_graph(torch, dn, stream, inner=n_ids)
         b_gu = n_dist * 2 * (dff * dm // 2 + dff * (dm // 64) * 4) + 2 * T * dm + 2 * T * k * dff
         b_dn = n_dist * (dm * dff // 2 + dm * (dff // 64) * 4) + 2 * T * k * dff + 2 * T * k * dm
         out[f"moe_gate_up_silu_t{T}"] = {"GB/s": round(b_gu / (t_gu * 1e-3) / 1e9, 1),
                                          "frac": round(b_gu / (t_gu * 1e-3) / 1e9 / hbm_peak, 3),
-                                         "us": round(t_gu * 1e3, 2), "distinct_experts": n_dist}
+                                         "us": round(t_gu * 1e3, 2), "distinct_experts": round(n_dist, 1),
+                                         "rotation": f"{n_sets} weight sets x {n_ids} id sets"}
         out[f"moe_down_t{T}"] = {"GB/s": round(b_dn / (t_dn * 1e-3) / 1e9, 1),
                                  "frac": round(b_dn / (t_dn * 1e-3) / 1e9 / hbm_peak, 3),
                                  "us": round(t_dn * 1e3, 2)}

@@ -235,8 +235,9 @@ __device__ __forceinline__ int64_t pair_offset(const QgemvParams& p, int pair) {
 // (a counting sort by expert id) and the list of distinct experts; dense calls
 // have one "expert" whose pairs are the M tokens.  A pair with an id outside
 // [0, E) gets a zero output row (written by CTA 0) and QMM_ERR_BAD_EXPERT_ID.
+// s_ids (n_pairs ints) holds the ids read once from global memory.
 __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int* s_start,
-                                           int* s_fill, int* s_dist, int* s_list, int* s_nd) {
+                                           int* s_fill, int* s_dist, int* s_list, int* s_ids, int* s_nd) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nthr = blockDim.x;
   const int E = p.num_experts;
@@ -249,6 +250,7 @@ __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int
     __syncthreads();
     for (int i = tid; i < p.n_pairs; i += nthr) {
       const int e = p.ids[i];
+      s_ids[i] = e;
       if (e >= 0 && e < E) atomicAdd(&s_cnt[e], 1);
     }
     __syncthreads();
@@ -279,7 +281,7 @@ __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int
     if (warp == 0) {
       for (int base = 0; base < p.n_pairs; base += 32) {
         const int i = base + lane;
-        const int e = i < p.n_pairs ? p.ids[i] : -1;
+        const int e = i < p.n_pairs ? s_ids[i] : -1;
         const bool valid = e >= 0 && e < E;
         const unsigned same = __match_any_sync(0xffffffffu, valid ? e : E + lane);
         if (valid) {
@@ -293,7 +295,7 @@ __device__ __forceinline__ void build_plan(const QgemvParams& p, int* s_cnt, int
     }
     if (blockIdx.x == 0) {
       for (int i = tid; i < p.n_pairs; i += nthr) {
-        const int e = p.ids[i];
+        const int e = s_ids[i];
         if (e < 0 || e >= E) {  // bad id: zero row, report
           for (int64_t n = 0; n < p.n_rows; ++n) store_as(p.out, p.out_dtype, (int64_t)i * p.out_ld + n, 0.0f);
           set_status(p.d_status, QMM_ERR_BAD_EXPERT_ID);
@@ -476,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1) qgemv_kernel(const QgemvParams p)
   float* part = reinterpret_cast<float*>(smem + p.off_part);   // [kWarps][16][TOKP][NS]
   const uint32_t ring_base = smem_u32(smem + p.off_ring + warp * C::RING_BYTES);
 
-  build_plan(p, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
+  build_plan(p, s_cnt, s_start, s_fill, s_dist, s_list, s_list + p.n_pairs, &s_nd);
 
   const int64_t V = (int64_t)s_nd * p.n_rows;
   const int64_t v0 = V * blockIdx.x / gridDim.x;
@@ -746,7 +748,7 @@ cudaError_t launch_one(QgemvParams prm, cudaStream_t st) {
   const int E = prm.ids ? prm.num_experts : 1;
   const int bpg_tok = GS * (S::kSplit ? 2 : 1) * (int)sizeof(T);  // staged x bytes per group per token
 
-  const size_t plan = align128((size_t)(4 * E + prm.n_pairs) * sizeof(int));
+  const size_t plan = align128((size_t)(4 * E + 2 * prm.n_pairs) * sizeof(int));
   const size_t ring = (size_t)kWarps * C::RING_BYTES;
   const size_t part = align128((size_t)kWarps * 16 * C::TOKP * C::NS * sizeof(float));
   auto chunk_bytes = [&](int kc) {

@@ -372,7 +372,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   if (q.ids) {
     // the ids (like x) may come from the previous kernel in the stream
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
+    build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, s_list + q.n_pairs, &s_nd);
     if (tid == 0) {
       int run = 0;
       s_seg[0] = 0;
@@ -816,7 +816,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   const size_t xs = align128((size_t)C::CH * p.tok_stride);
   const size_t xsum = align128((size_t)Gpad * C::TOKP * 4 * C::NX);
   const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
-  const size_t plan = align128((size_t)(5 * q.num_experts + 1 + q.n_pairs) * sizeof(int));
+  const size_t plan = align128((size_t)(5 * q.num_experts + 1 + 2 * q.n_pairs) * sizeof(int));
   if (plan > 32 * 1024) return cudaErrorNotSupported;
   auto total = [&](int stages) {
     return 1024 + (size_t)stages * NS * C::CODE_BYTES + align128((size_t)stages * NS * 2 * C::SB_BYTES) +

@@ -134,7 +134,7 @@ qgemv_tma_kernel(const QgemvParams p, const __grid_constant__ CUtensorMap tm0,
   }
   __syncwarp();
 
-  build_plan(p, s_cnt, s_start, s_fill, s_dist, s_list, &s_nd);
+  build_plan(p, s_cnt, s_start, s_fill, s_dist, s_list, s_list + p.n_pairs, &s_nd);
 
   const int64_t V = (int64_t)s_nd * p.n_rows;
   const int64_t v0 = V * blockIdx.x / gridDim.x;
@@ -415,7 +415,7 @@ cudaError_t launch_tma_impl(QgemvParams prm, int64_t rows_total, cudaStream_t st
   const size_t codes = (size_t)kWarps * C::STAGES * C::CODE_STAGE;
   const size_t sb = align128((size_t)kWarps * C::STAGES * C::SB_STAGE);
   const size_t bars = align128((size_t)kWarps * C::STAGES * 8);
-  const size_t plan = align128((size_t)(4 * E + prm.n_pairs) * sizeof(int));
+  const size_t plan = align128((size_t)(4 * E + 2 * prm.n_pairs) * sizeof(int));
   const size_t part = align128((size_t)kWarps * 16 * C::TOKP * C::NS * sizeof(float));
   auto chunk_bytes = [&](int kc) {
     const size_t ts = (size_t)kc * bpg_tok + 16;
