@@ -36,9 +36,13 @@
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronizes the host.
  *   - Host-side argument errors are returned before anything is launched.
- *     Errors found on the device (a bad expert id) are OR-ed into *d_status
- *     (a caller-zeroed device int32, may be NULL), read by the caller after
- *     the stream has synchronized.  The library never aborts.
+ *     Errors found on the device (a bad expert id; QMM_ERR_TIMEOUT when a
+ *     bounded wait inside a kernel gave up) are OR-ed into *d_status (a
+ *     caller-zeroed device int32, may be NULL), read by the caller after the
+ *     stream has synchronized.  qmm_matmul takes no status buffer: there a
+ *     device-side timeout leaves y incomplete (the prefill GEMM writes the
+ *     affected tile as NaN).  The library never aborts and never waits
+ *     without a bound.
  *   - Shapes: group_size in {32, 64, 128}; cols % group_size == 0 and
  *     cols * bits % 32 == 0 for the quantized axis.
  *   - Alignment: packed, scales, biases, x, y and out must be 16-byte
