@@ -43,12 +43,6 @@ __device__ __forceinline__ void store_as(void* base, int dtype, int64_t idx, flo
     reinterpret_cast<__half*>(base)[idx] = __float2half_rn(v);
 }
 
-__device__ __forceinline__ float load_as(const void* base, int dtype, int64_t idx) {
-  if (dtype == QMM_F32) return reinterpret_cast<const float*>(base)[idx];
-  if (dtype == QMM_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
-  return __half2float(reinterpret_cast<const __half*>(base)[idx]);
-}
-
 // ---------------------------------------------------------------- bit fields
 // Code i (compile-time after unrolling) of a register array holding an
 // LSB-first bitstream: bits [i*B, i*B+B), possibly spanning two registers.
@@ -63,28 +57,6 @@ __device__ __forceinline__ uint32_t stream_code(const uint32_t* r, int i) {
   else
     v = __funnelshift_r(r[w], r[w + 1], sh);
   return v & ((1u << B) - 1u);
-}
-
-// Non-coherent 32/64/128-bit global loads that bypass L1 allocation: the
-// packed weights are streamed exactly once per launch.
-__device__ __forceinline__ uint32_t ldg_stream_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint2 ldg_stream_u64(const uint32_t* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.b32 {%0,%1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint4 ldg_stream_u128(const uint32_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
 }
 
 __device__ __forceinline__ void set_status(int32_t* d_status, int code) {
