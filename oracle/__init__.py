@@ -33,15 +33,22 @@ _lock = threading.Lock()
 _lib = None
 
 
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+
+def compile_oracle(src: str, out: str) -> str:
+    """gcc `src` into the shared library `out` with the oracle's flags."""
+    subprocess.run(["gcc", *CFLAGS, "-o", out, src, "-lm"], check=True)
+    return out
+
+
 def build_oracle(force: bool = False) -> str:
     """Compile the oracle shared library (idempotent); returns its path."""
     with _lock:
         fresh = os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)
         if force or not fresh:
             tmp = _LIB + f".tmp{os.getpid()}"
-            cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
-                   "-shared", "-o", tmp, _SRC, "-lm"]
-            subprocess.run(cmd, check=True)
+            compile_oracle(_SRC, tmp)
             os.replace(tmp, _LIB)
     return _LIB
 
@@ -53,42 +60,46 @@ class _Stack(ctypes.Structure):
                 ("n_cols", ctypes.c_int64), ("gs", ctypes.c_int), ("bits", ctypes.c_int)]
 
 
-def lib():
+def bind(path: str) -> ctypes.CDLL:
+    """Load a compiled oracle library and declare its C signatures."""
+    L = ctypes.CDLL(path)
+    vp, i64, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_f32.restype = ctypes.c_float
+    L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+    L.orc_f16_to_f32.restype = ctypes.c_float
+    L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
+    L.orc_f32_to_bf16.restype = ctypes.c_uint16
+    L.orc_f32_to_f16.argtypes = [ctypes.c_float]
+    L.orc_f32_to_f16.restype = ctypes.c_uint16
+    L.orc_words_per_row.argtypes = [i64, c_int]
+    L.orc_words_per_row.restype = i64
+    L.orc_pack_row.argtypes = [vp, i64, c_int, vp]
+    L.orc_pack_row.restype = None
+    L.orc_code_integral.argtypes = [vp, c_int, i64]
+    L.orc_code_integral.restype = ctypes.c_uint32
+    L.orc_code_u64.argtypes = [vp, i64, c_int, i64]
+    L.orc_code_u64.restype = ctypes.c_uint32
+    L.orc_quantize.argtypes = [vp, c_int, i64, i64, c_int, c_int, c_int, vp, vp, vp, i64, i64]
+    L.orc_dequantize.argtypes = [vp, vp, vp, c_int, i64, i64, c_int, c_int, vp, c_int, i64, i64]
+    L.orc_matmul.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int, c_int, c_int,
+                             vp, i64, i64]
+    L.orc_matmul_element.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int,
+                                     c_int, c_int, i64, i64]
+    L.orc_matmul_element.restype = ctypes.c_double
+    sp = ctypes.POINTER(_Stack)
+    L.orc_moe_gemv_id.argtypes = [vp, c_int, vp, i64, i64, sp, vp, i64, i64]
+    L.orc_moe_gemv_id_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, vp, i64, i64]
+    L.orc_moe_gate_up_silu.argtypes = [vp, c_int, vp, i64, sp, sp, vp, i64, i64]
+    L.orc_moe_gate_up_silu_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, sp, vp,
+                                               i64, i64]
+    return L
+
+
+def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build_oracle())
-        vp, i64, i32, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
-        L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
-        L.orc_bf16_to_f32.restype = ctypes.c_float
-        L.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
-        L.orc_f16_to_f32.restype = ctypes.c_float
-        L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
-        L.orc_f32_to_bf16.restype = ctypes.c_uint16
-        L.orc_f32_to_f16.argtypes = [ctypes.c_float]
-        L.orc_f32_to_f16.restype = ctypes.c_uint16
-        L.orc_words_per_row.argtypes = [i64, c_int]
-        L.orc_words_per_row.restype = i64
-        L.orc_pack_row.argtypes = [vp, i64, c_int, vp]
-        L.orc_pack_row.restype = None
-        L.orc_code_integral.argtypes = [vp, c_int, i64]
-        L.orc_code_integral.restype = ctypes.c_uint32
-        L.orc_code_u64.argtypes = [vp, i64, c_int, i64]
-        L.orc_code_u64.restype = ctypes.c_uint32
-        L.orc_quantize.argtypes = [vp, c_int, i64, i64, c_int, c_int, c_int, vp, vp, vp, i64, i64]
-        L.orc_dequantize.argtypes = [vp, vp, vp, c_int, i64, i64, c_int, c_int, vp, c_int, i64, i64]
-        L.orc_matmul.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int, c_int, c_int,
-                                 vp, i64, i64]
-        L.orc_matmul_element.argtypes = [vp, c_int, i64, i64, vp, vp, vp, c_int, i64, c_int,
-                                         c_int, c_int, i64, i64]
-        L.orc_matmul_element.restype = ctypes.c_double
-        sp = ctypes.POINTER(_Stack)
-        L.orc_moe_gemv_id.argtypes = [vp, c_int, vp, i64, i64, sp, vp, i64, i64]
-        L.orc_moe_gemv_id_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, vp, i64, i64]
-        L.orc_moe_gate_up_silu.argtypes = [vp, c_int, vp, i64, sp, sp, vp, i64, i64]
-        L.orc_moe_gate_up_silu_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, sp, sp, vp,
-                                                   i64, i64]
-        _ = (i32,)
-        _lib = L
+        _lib = bind(build_oracle())
     return _lib
 
 

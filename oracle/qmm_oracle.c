@@ -26,8 +26,10 @@
  *
  * Parity pins: every function here is pinned by tests/test_oracle_pins.py
  * (exact-rational recomputation, big-integer bitstreams, library dtype
- * conversions, closed forms).  The accumulation order of the GPU kernels is
- * the only thing left "parity unpinned" (tolerance only).
+ * conversions, closed forms); tests/test_oracle_mutants.py checks that
+ * planted mistakes in a copy of this file fail those pins.  The accumulation
+ * order of the GPU kernels is the only thing left "parity unpinned"
+ * (tolerance only).
  */
 #include <float.h>
 #include <math.h>

@@ -198,6 +198,44 @@ def test_round_trip_bound_bf16_storage(bits):
     assert np.all(err <= bound * (1 + 1e-6) + 1e-9)
 
 
+def _exact_grid_distance(wv, q, s, b):
+    return abs(wv - (q * s + b))
+
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("sdt", ["bf16", "f16"])
+def test_codes_are_nearest_on_the_stored_grid(bits, sdt):
+    """Every code picks the point of its group's STORED grid {q*s + b, 0 <= q < 2^b}
+    nearest to w (exact rationals; the slack covers the two fp32 roundings of
+    (w - b)/s).  This holds only if codes are computed against the rounded
+    scale and bias, and clamped at both ends.  Group 0 of row 0 is built so
+    that its fp32 scale 1 + 2^-8 - 2^-20 rounds down to 1 in bf16: its top
+    value then sits 2^b/256 codes above the last code, past 255.5 at 8 bits."""
+    gs, rows, cols = 64, 16, 128
+    qmax = (1 << bits) - 1
+    rng = np.random.default_rng(400 + bits)
+    w = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+    scale_f = np.float32(1.0 + 2.0**-8 - 2.0**-20)
+    top = np.float32(np.float64(scale_f) * qmax)
+    w[0, :gs] = (rng.random(gs) * float(top)).astype(np.float32)
+    w[0, 0], w[0, 1] = 0.0, top
+    packed, sc, bi = oracle.quantize(w, oracle.F32, gs, bits, DT[sdt])
+    if sdt == "bf16":
+        assert widen(sc, sdt)[0, 0] == 1.0
+    for r in range(rows):
+        codes = exact.unpack_bigint(packed[r].tolist(), bits, cols)
+        for i in range(cols):
+            s = exact.storage_to_fraction(sc[r, i // gs], sdt)
+            b = exact.storage_to_fraction(bi[r, i // gs], sdt)
+            wv, q = Fraction(float(w[r, i])), codes[i]
+            d = _exact_grid_distance(wv, q, s, b)
+            slack = s * (qmax + 1) * Fraction(1, 2**22)
+            for qn in (q - 1, q + 1):
+                if 0 <= qn <= qmax:
+                    assert d <= _exact_grid_distance(wv, qn, s, b) + slack, (r, i, q)
+    assert exact.unpack_bigint(packed[0].tolist(), bits, cols)[1] == qmax
+
+
 def test_tie_rounds_half_away_from_zero():
     """{0, 6.5, 7.5, 15, 0...}: s = 1, so codes are 0, 7, 8, 15 under half-away
     (half-even would give 6 for 6.5)."""
