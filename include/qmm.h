@@ -50,6 +50,11 @@
  *     only need element alignment.
  *   - Requires a compute-capability 10.0 device (QMM_ERR_UNSUPPORTED
  *     otherwise).
+ *   - MoE calls: a_dtype must be QMM_BF16 or QMM_F16 (QMM_F32 activations
+ *     are QMM_ERR_UNSUPPORTED); at most 65536 pairs (n_selected, or
+ *     m * top_k) and 65536 experts (QMM_ERR_UNSUPPORTED above); ids and
+ *     d_status must be 4-byte aligned; a negative stride, pair count or m,
+ *     or top_k <= 0, is QMM_ERR_INVALID_ARG.
  */
 #ifndef QMM_H_
 #define QMM_H_

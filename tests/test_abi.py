@@ -115,3 +115,64 @@ def test_moe_validation(L):
     assert b(A, _lib.QMM_BF16, A, 2, 0, 0, 0, ctypes.byref(s), A, _lib.QMM_BF16, None, None) == _lib.QMM_ERR_INVALID_ARG
     bb = L.qmm_moe_gemv_id_gate_up_silu_batched
     assert bb(A, _lib.QMM_BF16, A, 0, 8, 0, 0, ctypes.byref(g), ctypes.byref(g), A, _lib.QMM_BF16, None, None) == _lib.QMM_OK
+
+
+def test_moe_limits_and_alignment(L):
+    bf, f32 = _lib.QMM_BF16, _lib.QMM_F32
+    s = stack()
+    f = L.qmm_moe_gemv_id
+    ok_args = dict(a=A, ids=A, out=A, status=None)
+
+    def call(n=2, stride=128, w=s, a_dtype=bf, out_dtype=bf, **kw):
+        args = {**ok_args, **kw}
+        return f(args["a"], a_dtype, args["ids"], n, stride, ctypes.byref(w), args["out"],
+                 out_dtype, args["status"], None)
+
+    # dtype rules: out is a_dtype or f32; fp32 activations have no MoE kernel
+    assert call(out_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
+    s32 = stack(sdtype=f32)
+    assert call(w=s32, a_dtype=f32, out_dtype=f32) == _lib.QMM_ERR_UNSUPPORTED
+    # negative counts and strides
+    assert call(n=-1) == _lib.QMM_ERR_INVALID_ARG
+    assert call(stride=-128) == _lib.QMM_ERR_INVALID_ARG
+    # size limits: 65536 pairs and 65536 experts
+    assert call(n=65537) == _lib.QMM_ERR_UNSUPPORTED
+    assert call(w=stack(E=65537)) == _lib.QMM_ERR_UNSUPPORTED
+    # pointer rules: a needs element alignment, ids and d_status 4 bytes, out 16
+    assert call(a=0) == _lib.QMM_ERR_ALIGNMENT
+    assert call(a=A + 1) == _lib.QMM_ERR_ALIGNMENT
+    assert call(ids=A + 2) == _lib.QMM_ERR_ALIGNMENT
+    assert call(ids=0) == _lib.QMM_ERR_ALIGNMENT
+    assert call(status=A + 2) == _lib.QMM_ERR_ALIGNMENT
+    assert call(out=A + 8) == _lib.QMM_ERR_ALIGNMENT
+
+
+def test_moe_batched_pair_count_cannot_overflow(L):
+    """m * top_k is checked against the 65536-pair limit without forming a
+    product that wraps (2^32 * 2^32 would wrap to 0 pairs)."""
+    s = stack()
+    g = stack()
+    b = L.qmm_moe_gemv_id_batched
+    bb = L.qmm_moe_gemv_id_gate_up_silu_batched
+    bf = _lib.QMM_BF16
+    for m, top_k, want in [(2**32, 2**32, _lib.QMM_ERR_UNSUPPORTED),
+                           (2**62, 4, _lib.QMM_ERR_UNSUPPORTED),
+                           (1000, 66, _lib.QMM_ERR_UNSUPPORTED),
+                           (0, 2**40, _lib.QMM_OK),
+                           (-1, 8, _lib.QMM_ERR_INVALID_ARG),
+                           (4, 0, _lib.QMM_ERR_INVALID_ARG)]:
+        assert b(A, bf, A, m, top_k, 0, 0, ctypes.byref(s), A, bf, None, None) == want, (m, top_k)
+        assert bb(A, bf, A, m, top_k, 0, 0, ctypes.byref(g), ctypes.byref(g), A, bf, None,
+                  None) == want, (m, top_k)
+    assert b(A, bf, A, 2, 4, -1, 0, ctypes.byref(s), A, bf, None, None) == _lib.QMM_ERR_INVALID_ARG
+    assert b(A, bf, A, 2, 4, 0, -1, ctypes.byref(s), A, bf, None, None) == _lib.QMM_ERR_INVALID_ARG
+
+
+def test_moe_gate_up_must_match(L):
+    h = L.qmm_moe_gemv_id_gate_up_silu
+    bf = _lib.QMM_BF16
+    g = stack()
+    for up in (stack(E=5), stack(cols=256), stack(bits=8), stack(gs=32),
+               stack(sdtype=_lib.QMM_F16)):
+        assert h(A, bf, A, 2, ctypes.byref(g), ctypes.byref(up), A, bf, None, None) \
+            == _lib.QMM_ERR_INVALID_ARG

@@ -42,6 +42,15 @@ static bool packable(int64_t cols, int gs, int bits) {
 }
 static bool aligned4(const void* p) { return p && ((reinterpret_cast<uintptr_t>(p) & 3u) == 0); }
 
+// Largest MoE call the kernels' per-CTA plans are sized for (pairs, experts).
+constexpr int64_t kMaxMoePairs = 65536;
+
+// m * top_k pairs of a batched MoE call; a product above kMaxMoePairs is
+// reported as kMaxMoePairs + 1 (rejected as unsupported) without overflowing.
+static int64_t batched_pairs(int64_t m, int64_t top_k) {
+  return (m > 0 && top_k > kMaxMoePairs / m) ? kMaxMoePairs + 1 : m * top_k;
+}
+
 static qmm_status check_qweight(const qmm_qweight* w) {
   if (!w) return QMM_ERR_INVALID_ARG;
   if (w->mode != QMM_MODE_AFFINE) return QMM_ERR_UNSUPPORTED;
@@ -183,7 +192,7 @@ static qmm_status moe_common(const void* a, qmm_dtype a_dtype, const int32_t* id
   if (n_pairs < 0 || stride < 0 || outer < 0 || inner < 0) return QMM_ERR_INVALID_ARG;
   if (n_pairs == 0) return QMM_OK;
   if (a_dtype == QMM_F32) return QMM_ERR_UNSUPPORTED;  // tensor-core path only
-  if (n_pairs > 65536 || w0->num_experts > 65536) return QMM_ERR_UNSUPPORTED;
+  if (n_pairs > kMaxMoePairs || w0->num_experts > kMaxMoePairs) return QMM_ERR_UNSUPPORTED;
   if (!a || (reinterpret_cast<uintptr_t>(a) & 1u)) return QMM_ERR_ALIGNMENT;
   if (!aligned4(ids) || !aligned16(out)) return QMM_ERR_ALIGNMENT;
   if (d_status && !aligned4(d_status)) return QMM_ERR_ALIGNMENT;
@@ -209,7 +218,7 @@ qmm_status qmm_moe_gemv_id_batched(const void* a, qmm_dtype a_dtype, const int32
                                    int64_t inner_stride, const qmm_expert_stack* w, void* out,
                                    qmm_dtype out_dtype, int32_t* d_status, void* stream) {
   if (m < 0 || top_k <= 0) return QMM_ERR_INVALID_ARG;
-  return moe_common(a, a_dtype, ids, m * top_k, w, nullptr, out, out_dtype, d_status, stream, 2,
+  return moe_common(a, a_dtype, ids, batched_pairs(m, top_k), w, nullptr, out, out_dtype, d_status, stream, 2,
                     0, outer_stride, inner_stride, top_k);
 }
 
@@ -231,7 +240,7 @@ qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype
                                                 void* stream) {
   if (!up) return QMM_ERR_INVALID_ARG;
   if (m < 0 || top_k <= 0) return QMM_ERR_INVALID_ARG;
-  return moe_common(a, a_dtype, ids, m * top_k, gate, up, silu_out, out_dtype, d_status, stream,
+  return moe_common(a, a_dtype, ids, batched_pairs(m, top_k), gate, up, silu_out, out_dtype, d_status, stream,
                     2, 0, outer_stride, inner_stride, top_k);
 }
 
