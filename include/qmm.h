@@ -51,10 +51,16 @@
  *   - Requires a compute-capability 10.0 device (QMM_ERR_UNSUPPORTED
  *     otherwise).
  *   - MoE calls: a_dtype must be QMM_BF16 or QMM_F16 (QMM_F32 activations
- *     are QMM_ERR_UNSUPPORTED); at most 65536 pairs (n_selected, or
- *     m * top_k) and 65536 experts (QMM_ERR_UNSUPPORTED above); ids and
- *     d_status must be 4-byte aligned; a negative stride, pair count or m,
- *     or top_k <= 0, is QMM_ERR_INVALID_ARG.
+ *     are QMM_ERR_UNSUPPORTED); ids and d_status must be 4-byte aligned; a
+ *     negative stride, pair count or m, or top_k <= 0, is
+ *     QMM_ERR_INVALID_ARG.  These are decode-size kernels: every CTA keeps
+ *     the call's expert plan (two ints per pair, four or five per expert) in
+ *     shared memory beside its pipeline buffers, so the pair count
+ *     (n_selected, or m * top_k) that fits depends on num_experts and the
+ *     kernel.  At 128 experts that is about 3,800 pairs for the fused
+ *     gate/up calls and about 6,800 for the single ones.  A larger call, or
+ *     one with more than 65536 pairs or experts, returns
+ *     QMM_ERR_UNSUPPORTED before anything is launched.
  */
 #ifndef QMM_H_
 #define QMM_H_
