@@ -138,29 +138,50 @@ const char* qmm_status_string(int status);
 /* QMM_OK when the current CUDA device is compute capability 10.0. */
 qmm_status qmm_device_check(void);
 
-/* Dense -> (packed, scales, biases).  w: [rows, cols] in w_dtype.  Output
- * scales/biases in s_dtype.  Bit-exact with the oracle's definition (see the
- * quantizer paragraph above).  rows == 0 is a no-op. */
+/* Dense -> (packed, scales, biases): the quantize step that "ollama
+ * x/create/client/quantize.go" (loadAndQuantizeArray) calls, with the
+ * per-group min/max rule of the quantizer paragraph above.
+ * w: [rows, cols] row-major in w_dtype (f32, f16 or bf16).  packed:
+ * [rows, cols*bits/32] uint32; scales, biases: [rows, cols/group_size] in
+ * s_dtype.  Bit-exact, whatever the launch shape.  rows == 0 is a no-op.
+ * Errors: INVALID_ARG for bits, group_size or cols outside the shape rules
+ * or rows < 0; DTYPE for an unknown dtype; ALIGNMENT for a null or
+ * under-aligned pointer; UNSUPPORTED on a device that is not compute
+ * capability 10.0; CUDA when the launch fails. */
 qmm_status qmm_quantize(const void* w, qmm_dtype w_dtype, int64_t rows, int64_t cols,
                         int group_size, int bits, qmm_dtype s_dtype, uint32_t* packed,
                         void* scales, void* biases, void* stream);
 
-/* out[r][i] = fmaf(q, scale, bias) stored in out_dtype (one RNE rounding
- * for f16/bf16).  out: [w->rows, w->cols] row-major. */
+/* Standalone dequantization ("emily 0.5.1 lib/emily/quantization.ex",
+ * dequantize_defn/1): out[r][i] = fmaf(q, scale, bias), stored in out_dtype
+ * with one RNE rounding for f16/bf16 and none for f32.  out: [w->rows,
+ * w->cols] row-major.  Bit-exact.  w->rows == 0 is a no-op.
+ * Errors: INVALID_ARG (shape rules, null w), UNSUPPORTED (mode other than
+ * affine, or the device), DTYPE, ALIGNMENT, CUDA. */
 qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, void* stream);
 
-/* y[M, N] = x[M, K] . dequant(W)^T  (transpose = 1: W is [N, K], w->rows = N,
+/* Quantized matmul ("emily 0.5.1 lib/emily/quantization.ex",
+ * quantized_matmul/2):
+ * y[M, N] = x[M, K] . dequant(W)^T  (transpose = 1: W is [N, K], w->rows = N,
  *                                    w->cols = K)
  * y[M, N] = x[M, K] . dequant(W)    (transpose = 0: W is [K, N] quantized
  *                                    along N, w->rows = K, w->cols = N)
  * x_dtype must equal w->sdtype; y_dtype is x_dtype or QMM_F32 (same
- * arithmetic, different final store).  Accumulation is fp32.  M == 0 is a
- * no-op.  bf16/f16 with transpose = 1 use the tensor-core kernels. */
+ * arithmetic, different final store).  x: [M, K] row-major; y: [M, N]
+ * row-major.  Accumulation is fp32.  M == 0 is a no-op.  bf16/f16 with
+ * transpose = 1 use the tensor-core kernels (M <= 16: the streaming GEMV;
+ * M > 16: the tcgen05 GEMM).
+ * Errors: INVALID_ARG (shape rules, K != the weight's input dimension,
+ * transpose not 0/1, M < 0), UNSUPPORTED (mode other than affine, or a
+ * device that is not compute capability 10.0), DTYPE (x_dtype !=
+ * w->sdtype, or y_dtype neither x_dtype nor f32), ALIGNMENT, CUDA. */
 qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
                       const qmm_qweight* w, int transpose, void* y, qmm_dtype y_dtype,
                       void* stream);
 
-/* out[i, :] = a[i*src1_stride : i*src1_stride + n_cols] . dequant(W[ids[i]])^T,
+/* MoE indirect GEMV ("ferrum-kernels 0.7.7 src/stacked_expert.rs",
+ * gemv_moe_id):
+ * out[i, :] = a[i*src1_stride : i*src1_stride + n_cols] . dequant(W[ids[i]])^T,
  * i in [0, n_selected).  ids: device int32[n_selected].  out: [n_selected,
  * n_rows] in out_dtype (a_dtype or QMM_F32).  A pair whose id is outside
  * [0, num_experts) gets a zero row and sets QMM_ERR_BAD_EXPERT_ID in
@@ -169,7 +190,8 @@ qmm_status qmm_moe_gemv_id(const void* a, qmm_dtype a_dtype, const int32_t* ids,
                            int64_t n_selected, int64_t src1_stride, const qmm_expert_stack* w,
                            void* out, qmm_dtype out_dtype, int32_t* d_status, void* stream);
 
-/* Batched form: ids is [m, top_k] row-major; pair p in [0, m*top_k) reads
+/* Batched form (same page, gemv_moe_id_batched): ids is [m, top_k]
+ * row-major; pair p in [0, m*top_k) reads
  * a[(p/top_k)*outer_stride + (p%top_k)*inner_stride : ... + n_cols] and
  * writes out[p, :]. */
 qmm_status qmm_moe_gemv_id_batched(const void* a, qmm_dtype a_dtype, const int32_t* ids,
@@ -177,7 +199,8 @@ qmm_status qmm_moe_gemv_id_batched(const void* a, qmm_dtype a_dtype, const int32
                                    int64_t inner_stride, const qmm_expert_stack* w, void* out,
                                    qmm_dtype out_dtype, int32_t* d_status, void* stream);
 
-/* silu_out[i, :] = SiLU(a . gate_e^T) * (a . up_e^T), e = ids[i], with
+/* Fused gate/up (same page, gemv_moe_id_gate_up_silu):
+ * silu_out[i, :] = SiLU(a . gate_e^T) * (a . up_e^T), e = ids[i], with
  * SiLU(g) = g / (1 + exp(-g)); every pair reads a[0 : n_cols] (the call has
  * no stride).  gate and up must have identical shapes and parameters
  * (QMM_ERR_INVALID_ARG otherwise).  Gate and up are computed in one pass. */
@@ -186,7 +209,9 @@ qmm_status qmm_moe_gemv_id_gate_up_silu(const void* a, qmm_dtype a_dtype, const 
                                         const qmm_expert_stack* up, void* silu_out,
                                         qmm_dtype out_dtype, int32_t* d_status, void* stream);
 
-/* Batched fused form: pair offsets as in qmm_moe_gemv_id_batched. */
+/* Batched fused form (same page, gemv_moe_id_gate_up_silu_batched): pair
+ * offsets as in qmm_moe_gemv_id_batched.  The MoE errors for all four calls
+ * are listed in the conventions above. */
 qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype,
                                                 const int32_t* ids, int64_t m, int64_t top_k,
                                                 int64_t outer_stride, int64_t inner_stride,
