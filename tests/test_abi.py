@@ -176,3 +176,23 @@ def test_moe_gate_up_must_match(L):
                stack(sdtype=_lib.QMM_F16)):
         assert h(A, bf, A, 2, ctypes.byref(g), ctypes.byref(up), A, bf, None, None) \
             == _lib.QMM_ERR_INVALID_ARG
+
+
+def _sources(root, exts):
+    for dirpath, dirnames, files in os.walk(root):
+        dirnames[:] = [d for d in dirnames if not d.startswith((".", "_build", "__pycache__"))]
+        for f in files:
+            if f.endswith(exts):
+                yield os.path.join(dirpath, f)
+
+
+def test_product_and_oracle_share_no_code():
+    """The product package never loads the oracle, and the oracle never
+    includes, imports or links anything of the product."""
+    pkg = os.path.join(ROOT, "weight_only_quantized_qmm_b200")
+    bad_in_pkg = re.compile(r"^\s*(import|from)\s+oracle\b|liboracle|qmm_oracle\.c", re.M)
+    for path in _sources(pkg, (".py", ".cu", ".cuh", ".h", ".cpp")):
+        assert not bad_in_pkg.search(open(path).read()), path
+    bad_in_oracle = re.compile(r"weight_only_quantized_qmm_b200|libqmm|#include\s+\"|qmm\.h")
+    for path in _sources(os.path.join(ROOT, "oracle"), (".py", ".c", ".h")):
+        assert not bad_in_oracle.search(open(path).read()), path
