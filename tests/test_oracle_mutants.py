@@ -124,6 +124,23 @@ MUTANTS = [
      "        out[i * st->n_rows + n] = 0.0;\n        rc = ORC_ERR_ID;",
      "        out[i * st->n_rows + n] = 0.0;",
      [P(pins.test_moe_bad_id_reports_and_zero_fills)]),
+    ("batched bad expert id not reported",
+     "        out[p * st->n_rows + n] = 0.0;\n        rc = ORC_ERR_ID;",
+     "        out[p * st->n_rows + n] = 0.0;",
+     [P(pins.test_moe_bad_id_reports_and_zero_fills)]),
+    ("fused bad expert id not reported",
+     "        out[i * gate->n_rows + n] = 0.0;\n        rc = ORC_ERR_ID;",
+     "        out[i * gate->n_rows + n] = 0.0;",
+     [P(pins.test_moe_bad_id_reports_and_zero_fills)]),
+    ("fused batched offset swaps outer and inner",
+     "int64_t off = (p / top_k) * outer + (p % top_k) * inner;\n    for (int64_t n = 0; n < gate->n_rows; ++n) {",
+     "int64_t off = (p % top_k) * outer + (p / top_k) * inner;\n    for (int64_t n = 0; n < gate->n_rows; ++n) {",
+     [P(pins.test_moe_gate_up_silu_closed_form)]),
+    # the single-element form used by the sampled full-size checks
+    ("sampled element drops the first term",
+     "  for (int64_t k = 0; k < K; ++k) {\n    float wv = transpose",
+     "  for (int64_t k = 1; k < K; ++k) {\n    float wv = transpose",
+     [P(pins.test_matmul_brute_force_exact, bits=4, transpose=True)]),
 ]
 
 

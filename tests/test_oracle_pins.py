@@ -460,3 +460,14 @@ def test_moe_bad_id_reports_and_zero_fills():
     out, rc = oracle.moe_gemv_id(a, oracle.BF16, np.array([0, 7, -1], np.int32), 3, 0, st)
     assert rc == oracle.ORC_ERR_ID
     assert np.all(out[1] == 0) and np.all(out[2] == 0) and np.any(out[0] != 0)
+    # the same rule in the batched and fused forms
+    ids2 = np.array([[0, 3], [-2, 1]], np.int32)
+    ob, rc = oracle.moe_gemv_id_batched(a, oracle.BF16, ids2, 2, 2, 0, 0, st)
+    assert rc == oracle.ORC_ERR_ID
+    assert np.all(ob[1] == 0) and np.all(ob[2] == 0) and np.any(ob[0] != 0) and np.any(ob[3] != 0)
+    og, rc = oracle.moe_gate_up_silu(a, oracle.BF16, np.array([3, 2], np.int32), 2, st, st)
+    assert rc == oracle.ORC_ERR_ID
+    assert np.all(og[0] == 0) and np.any(og[1] != 0)
+    ogb, rc = oracle.moe_gate_up_silu_batched(a, oracle.BF16, ids2, 2, 2, 0, 0, st, st)
+    assert rc == oracle.ORC_ERR_ID
+    assert np.all(ogb[1] == 0) and np.all(ogb[2] == 0) and np.any(ogb[0] != 0)
