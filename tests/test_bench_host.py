@@ -96,3 +96,21 @@ def test_clock_sampler_without_nvml_reports_unavailable(monkeypatch):
     with cs:
         pass
     assert cs.summary()["reasons"] == ["unavailable"]
+
+
+def test_gpu_arm_fails_loudly_without_a_gpu():
+    """With no GPU the bench's own arm exits non-zero and prints no result
+    line: there is no CPU path that could stand in for the kernels."""
+    import os
+    import subprocess
+    import sys
+
+    import pytest
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--steps", "3",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0
+    assert '"metric"' not in r.stdout
