@@ -196,3 +196,20 @@ def test_product_and_oracle_share_no_code():
     bad_in_oracle = re.compile(r"weight_only_quantized_qmm_b200|libqmm|#include\s+\"|qmm\.h")
     for path in _sources(os.path.join(ROOT, "oracle"), (".py", ".c", ".h")):
         assert not bad_in_oracle.search(open(path).read()), path
+
+
+def test_binding_refuses_host_tensors():
+    """The Python binding passes device addresses only: a CPU tensor raises
+    before anything reaches the library (no CPU path exists)."""
+    import torch
+
+    from weight_only_quantized_qmm_b200 import api
+
+    with pytest.raises(ValueError, match="CUDA"):
+        api.qmm_quantize(torch.zeros(16, 64), 32, 4)
+    qw = api.QWeight(torch.zeros(16, 8, dtype=torch.int32), torch.zeros(16, 2),
+                     torch.zeros(16, 2), 16, 64, 32, 4)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.qmm_matmul(torch.zeros(1, 64), qw)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.qmm_dequantize(qw)

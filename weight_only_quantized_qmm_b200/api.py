@@ -27,7 +27,13 @@ def dtype_code(dt: torch.dtype) -> int:
 
 
 def _ptr(t) -> int:
-    return 0 if t is None else int(t.data_ptr())
+    """Device address of a CUDA tensor (0 for None).  A host tensor is
+    refused: the kernels would dereference its address on the GPU."""
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"qmm: tensor arguments must be CUDA tensors, got one on {t.device}")
+    return int(t.data_ptr())
 
 
 def _stream(stream=None) -> int:
