@@ -10,11 +10,20 @@ group 64, bf16 activations, scales and biases).  `value` is the algorithmic
 bytes of those three calls (packed codes + scales + biases + x + y) summed over
 all steps of all ranks, divided by the timed device time (max over ranks).
 
-Timing: W warm-up steps, then K steps bracketed by barrier +
-cuda.synchronize, CUDA events on the launching stream.  The steps are
-replayed from a CUDA graph (host launch overhead is larger than the kernels)
-and rotate over weight copies larger than L2.  Under torchrun each rank runs
-the same workload on its own GPU (independent replicas, weak scaling).
+Timing: W warm-up steps, then timed trials of exactly K steps each, every
+trial behind an L2 flush and bracketed by barrier + cuda.synchronize, CUDA
+events on the launching stream; trials repeat for --clock-window seconds so
+that the NVML clock sampler sees the load, and the median trial is reported.
+The steps are replayed from CUDA graphs (host launch overhead is larger than
+the kernels) and rotate over weight copies larger than 3x L2.  Under torchrun
+each rank runs the same workload on its own GPU (independent replicas, weak
+scaling); the time is the max over ranks.
+
+Secondary lines (rank 0): every other workload -- the 36-config bit-width
+sweep, the MoE gate+up+SiLU and down GEMVs at T = 1, 16, 64 and the six
+prefill GEMMs -- with the fraction of the measured and the datasheet peaks.
+The oracle's CPU baseline is timed single-threaded (reported) and on all
+affinity cores (beside it).
 
 --impl reference times the CPU oracle (oracle/) on the same workload and
 metric, on a bounded sample per step; rank 0 only.
@@ -199,6 +208,20 @@ def traffic_record(name):
 
 
 # ---------------------------------------------------------------- our arm
+HBM_DATASHEET_GBS = 8000.0      # B200 HBM3e, datasheet
+BF16_DATASHEET_TFLOPS = 2250.0  # B200 dense bf16, datasheet
+
+
+def copies_for(nbytes: int) -> int:
+    """weight copies whose rotation reads more than 3x the L2 between reuses"""
+    return max(2, int(np.ceil(3 * L2_BYTES / nbytes)))
+
+
+def clone_qw(api, qw):
+    return api.QWeight(qw.packed.clone(), qw.scales.clone(), qw.biases.clone(), qw.rows, qw.cols,
+                       qw.group_size, qw.bits)
+
+
 def build_decode(torch, api, wl, n_sets, dev):
     cases = wl.WORKLOADS.decode
     sets = []
@@ -212,14 +235,35 @@ def build_decode(torch, api, wl, n_sets, dev):
     for s in range(n_sets):
         cur = []
         for c, qw, x in base:
-            q2 = qw if s == 0 else api.QWeight(qw.packed.clone(), qw.scales.clone(),
-                                               qw.biases.clone(), qw.rows, qw.cols,
-                                               qw.group_size, qw.bits)
+            q2 = qw if s == 0 else clone_qw(api, qw)
             y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
             cur.append((c, q2, x, y))
         sets.append(cur)
     torch.cuda.synchronize()
     return sets
+
+
+class L2Flush:
+    """Writes a buffer twice the size of L2 (between timed trials)."""
+
+    def __init__(self, torch, dev):
+        self.buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+        self.n = 0
+
+    def __call__(self):
+        self.n += 1
+        self.buf.fill_(float(self.n))
+
+
+def capture(torch, fn, n, stream):
+    """a CUDA graph of fn(0), ..., fn(n - 1) on `stream` (None when n == 0)"""
+    if n == 0:
+        return None
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(n):
+            fn(s)
+    return g
 
 
 def run_ours(args):
@@ -235,67 +279,92 @@ def run_ours(args):
 
     cases = wl.WORKLOADS.decode
     step_bytes = sum(decode_bytes(c.M, c.N, c.K, c.bits, c.group_size) for c in cases)
-    n_sets = max(2, int(np.ceil(3 * L2_BYTES / step_bytes)))  # rotate > 3x L2 of weights
+    n_sets = copies_for(step_bytes)  # the step's weights rotate over > 3x L2
     sets = build_decode(torch, api, wl, n_sets, dev)
-
     stream = torch.cuda.Stream(device=dev)
     launches_per_step = len(cases)
+    flush = L2Flush(torch, dev)
 
     def one_step(s):
         for c, qw, x, y in sets[s % n_sets]:
             api.qmm_matmul(x, qw, True, out=y, stream=stream)
 
-    # capture G steps (one full rotation, repeated) into one graph
-    G = n_sets * max(1, 48 // n_sets)
+    K = args.steps
+    W = max(args.warmup, 3)
     with torch.cuda.stream(stream):
-        for s in range(max(args.warmup, 3)):  # eager warm-up (also configures the kernels)
+        for s in range(W):  # eager warm-up steps (also configure the kernels)
             one_step(s)
     torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for s in range(G):
-            one_step(s)
-    torch.cuda.synchronize()
-    reps = max(1, args.steps // G)
-    steps = reps * G
-    # warm-up replays (W steps at least); graphs replay on the current stream
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, -(-args.warmup // G))):
-            graph.replay()
+    # exactly K steps per timed trial: `reps` replays of a one-rotation graph
+    # (n_sets steps) and one graph of the remaining K mod n_sets steps
+    reps, rem = divmod(K, n_sets)
+    g_full = capture(torch, one_step, n_sets if reps else 0, stream)
+    g_rem = capture(torch, one_step, rem, stream)
     torch.cuda.synchronize()
 
+    def replay_k():
+        for _ in range(reps):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    with torch.cuda.stream(stream):  # warm-up replays
+        replay_k()
+    torch.cuda.synchronize()
+
+    # timed trials: each trial is exactly K steps behind an L2 flush, bracketed
+    # by barrier + synchronize; trials repeat until the clock sampler has seen
+    # at least `clock_window` seconds of them; the reported time is the median
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(dev.index)
-    barrier(world)
-    torch.cuda.synchronize()
-    with sampler, torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(reps):
-            graph.replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    ms = max_over_ranks(world, ms)
-    ms_step = ms / steps
-    value = job_throughput(step_bytes, steps, world, ms)
+    sampler = ClockSampler(dev.index, period_s=0.01)
+    trial_ms = []
+    with sampler:
+        t_start = time.perf_counter()
+        while True:
+            with torch.cuda.stream(stream):
+                flush()
+            torch.cuda.synchronize()
+            barrier(world)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(stream):
+                ev0.record(stream)
+                replay_k()
+                ev1.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+            trial_ms.append(ev0.elapsed_time(ev1))
+            done = (time.perf_counter() - t_start >= args.clock_window and len(trial_ms) >= 3) \
+                or len(trial_ms) >= 20000
+            # every rank takes the same number of trials
+            if world > 1:
+                done = max_over_ranks(world, 1.0 if done else 0.0) > 0.5
+            if done:
+                break
+    ms = max_over_ranks(world, statistics.median(trial_ms))
+    ms_step = ms / K
+    value = job_throughput(step_bytes, K, world, ms)
 
-    # per-shape launch durations: one graph per shape (rotating its weight
-    # copies), timed from outside, so no event sits between two kernels
+    # per-shape launch durations: one graph per shape rotating its own copies
+    # (> 3x L2 each), timed from outside, so no event sits between two kernels
     per_shape = {}
     tot_b, tot_ms = 0.0, 0.0
     for i, c in enumerate(cases):
-        def shape_fn(i=i):
-            for s in range(n_sets):
-                _, qw, x, y = sets[s][i]
-                api.qmm_matmul(x, qw, True, out=y, stream=stream)
-        d = time_graph(torch, shape_fn, stream, reps=10, inner=max(1, 48 // n_sets)) / n_sets
         b = decode_bytes(c.M, c.N, c.K, c.bits, c.group_size)
+        n_i = copies_for(b)
+        qws = [sets[s][i][1] if s < n_sets else clone_qw(api, sets[0][i][1]) for s in range(n_i)]
+        _, _, x, y = sets[0][i]
+
+        def shape_fn(qws=qws, x=x, y=y):
+            for qw in qws:
+                api.qmm_matmul(x, qw, True, out=y, stream=stream)
+        d = time_graph(torch, shape_fn, stream, reps=10, inner=1) / n_i
         per_shape[c.name] = {"us": round(d * 1e3, 3), "GB/s": round(b / (d * 1e-3) / 1e9, 1),
-                             "frac": round(b / (d * 1e-3) / 1e9 / hbm_peak, 3)}
+                             "frac": round(b / (d * 1e-3) / 1e9 / hbm_peak, 3),
+                             "copies": n_i}
         tot_b += b
         tot_ms += d
+        del qws
     achieved = tot_b / (tot_ms * 1e-3) / 1e9
     rec, state = traffic_record("qgemv_decode_m1.txt")
     traffic = None
@@ -307,36 +376,34 @@ def run_ours(args):
 
     # end to end through the public API with host buffers (pinned), per step:
     # H2D of x, the three calls, D2H of y, synchronize
-    e2e = None
-    if rank == 0 or world > 1:
-        xs_h = [x.cpu().pin_memory() for (_, _, x, _) in sets[0]]
-        ys_h = [torch.empty(c.M, c.N, dtype=torch.bfloat16).pin_memory() for c in cases]
-        h2d = sum(t.numel() * t.element_size() for t in xs_h)
-        d2h = sum(t.numel() * t.element_size() for t in ys_h)
-        n_e2e = min(2000, max(50, args.steps // 10))
+    xs_h = [x.cpu().pin_memory() for (_, _, x, _) in sets[0]]
+    ys_h = [torch.empty(c.M, c.N, dtype=torch.bfloat16).pin_memory() for c in cases]
+    h2d = sum(t.numel() * t.element_size() for t in xs_h)
+    d2h = sum(t.numel() * t.element_size() for t in ys_h)
+    n_e2e = min(2000, max(50, 10 * K))
 
-        def e2e_step(s):
-            for i, (c, qw, x, y) in enumerate(sets[s % n_sets]):
-                x.copy_(xs_h[i], non_blocking=True)
-                api.qmm_matmul(x, qw, True, out=y)
-                ys_h[i].copy_(y, non_blocking=True)
-            torch.cuda.current_stream().synchronize()
-        for s in range(10):
-            e2e_step(s)
-        barrier(world)
-        t0 = time.perf_counter()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for s in range(n_e2e):
-            e2e_step(s)
-        e1.record()
-        torch.cuda.synchronize()
-        ms_e2e = max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3)
-        ms_e2e = max_over_ranks(world, ms_e2e)
-        e2e = {"value": round(step_bytes * n_e2e * world / (ms_e2e * 1e-3) / 1e9, 2),
-               "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(ms_e2e / n_e2e, 4), "steps": n_e2e}
+    def e2e_step(s):
+        for i, (c, qw, x, y) in enumerate(sets[s % n_sets]):
+            x.copy_(xs_h[i], non_blocking=True)
+            api.qmm_matmul(x, qw, True, out=y)
+            ys_h[i].copy_(y, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    for s in range(10):
+        e2e_step(s)
+    barrier(world)
+    t0 = time.perf_counter()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(n_e2e):
+        e2e_step(s)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_e2e = max(e0.elapsed_time(e1), (time.perf_counter() - t0) * 1e3)
+    ms_e2e = max_over_ranks(world, ms_e2e)
+    e2e = {"value": round(step_bytes * n_e2e * world / (ms_e2e * 1e-3) / 1e9, 2),
+           "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(ms_e2e / n_e2e, 4), "steps": n_e2e}
 
     secondary = {}
     if not args.no_secondary and rank == 0:
@@ -349,33 +416,41 @@ def run_ours(args):
     clocks = sampler.summary()
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 6),
+        "steps": K, "warmup": W, "ms_per_step": round(ms_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded: W=0.02*randn quantized 4-bit g64, x=randn->bf16)",
         "config": {"workload": "decode GEMV M=1, 4-bit affine g64, bf16 x/scales/biases; "
                                "N x K = 4096x4096 + 14336x4096 + 4096x14336 per step",
                    "global_batch": world, "M": 1, "bits": 4, "group_size": 64,
-                   "l2": f"rotates {n_sets} weight copies ({n_sets * step_bytes / 1e6:.0f} MB) > L2 126 MB",
-                   "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
+                   "l2": f"L2 flushed (256 MB write) before every trial; within a trial the steps "
+                         f"rotate {n_sets} weight copies ({n_sets * step_bytes / 1e6:.0f} MB > 3x L2)",
+                   "launch": "CUDA graph replay", "parallelism": f"replicas x{world}",
+                   "trials": len(trial_ms),
+                   "trial_ms": {"median": round(statistics.median(trial_ms), 5),
+                                "min": round(min(trial_ms), 5), "max": round(max(trial_ms), 5)}},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak,
                      "unit": "GB/s", "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
-                     "peak_source": peak_src, "kernel": "qgemv_stream_kernel<4,64,bf16,0,64|32,1> (one token; 64- or 32-group units)",
+                     "peak_source": peak_src,
+                     "frac_of_datasheet_8000": round(achieved / HBM_DATASHEET_GBS, 4),
+                     "kernel": "qgemv_stream_kernel (decode GEMV, one token)",
                      "per_shape": per_shape},
         "e2e": e2e,
-        "gpu_launches": steps * launches_per_step,
+        "gpu_launches": K * launches_per_step,
         "clocks": clocks,
         "cpu_baseline": cpu,
         "secondary": secondary,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
+    del g_full, g_rem
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 
 
 def time_graph(torch, fn, stream, reps=20, inner=4):
+    """median per-call device time (ms) of fn, replayed from a CUDA graph of
+    `inner` calls"""
     with torch.cuda.stream(stream):
         fn()
         fn()
@@ -401,10 +476,28 @@ def time_graph(torch, fn, stream, reps=20, inner=4):
     return statistics.median(times)
 
 
+def _gbs(nbytes, ms, hbm_peak):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"GB/s": round(gbs, 1), "frac": round(gbs / hbm_peak, 3),
+            "frac_of_datasheet_8000": round(gbs / HBM_DATASHEET_GBS, 3), "us": round(ms * 1e3, 3)}
+
+
 def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
     out = {}
-    # MoE decode: fused gate+up+SiLU then down, T = 1 and 16, top-8 of 128
-    for case in wl.WORKLOADS.moe[:2]:
+    for name, fn in (("moe", secondary_moe), ("sweep", secondary_sweep),
+                     ("prefill", secondary_prefill)):
+        try:
+            out[name] = fn(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust)
+        except Exception as e:  # pragma: no cover
+            out[name + "_error"] = str(e)[:300]
+        torch.cuda.empty_cache()
+    return out
+
+
+def secondary_moe(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    """MoE decode: fused gate+up+SiLU then down, T = 1, 16, 64, top-8 of 128"""
+    out = {}
+    for case in wl.WORKLOADS.moe:
         E, dff, dm, T, k = case.num_experts, case.d_ff, case.d_model, case.tokens, case.top_k
         n_sets = 3
         stacks = []
@@ -445,39 +538,55 @@ def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
         t_dn = time_graph(torch, dn, stream, inner=n_ids)
         b_gu = n_dist * 2 * (dff * dm // 2 + dff * (dm // 64) * 4) + 2 * T * dm + 2 * T * k * dff
         b_dn = n_dist * (dm * dff // 2 + dm * (dff // 64) * 4) + 2 * T * k * dff + 2 * T * k * dm
-        out[f"moe_gate_up_silu_t{T}"] = {"GB/s": round(b_gu / (t_gu * 1e-3) / 1e9, 1),
-                                         "frac": round(b_gu / (t_gu * 1e-3) / 1e9 / hbm_peak, 3),
-                                         "us": round(t_gu * 1e3, 2), "distinct_experts": round(n_dist, 1),
-                                         "rotation": f"{n_sets} weight sets x {n_ids} id sets"}
-        out[f"moe_down_t{T}"] = {"GB/s": round(b_dn / (t_dn * 1e-3) / 1e9, 1),
-                                 "frac": round(b_dn / (t_dn * 1e-3) / 1e9 / hbm_peak, 3),
-                                 "us": round(t_dn * 1e3, 2)}
+        out[f"moe_gate_up_silu_t{T}"] = dict(_gbs(b_gu, t_gu, hbm_peak), distinct_experts=round(n_dist, 1),
+                                             rotation=f"{n_sets} weight sets x {n_ids} id sets")
+        out[f"moe_down_t{T}"] = _gbs(b_dn, t_dn, hbm_peak)
         del stacks
-    # prefill GEMM M=2048, 14336x4096 (when the tensor-core GEMM path is built)
-    try:
-        c = [p for p in wl.WORKLOADS.prefill if p.M == 2048 and p.N == 14336][0]
-        qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), 64, 4, torch.bfloat16)
-        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
-        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
-        if _has_tc_gemm():
-            t = time_graph(torch, lambda: api.qmm_matmul(x, qw, True, out=y, stream=stream), stream,
-                           reps=10, inner=5)
-            tf = 2 * c.M * c.N * c.K / (t * 1e-3) / 1e12
-            out["prefill_gemm_m2048_14336x4096"] = {"TFLOP/s": round(tf, 1),
-                                                    "frac_of_measured_burst": round(tf / bf16_peak, 3),
-                                                    "frac_of_2250_dense": round(tf / 2250.0, 3),
-                                                    "us": round(t * 1e3, 1)}
-    except Exception as e:  # pragma: no cover
-        out["prefill_error"] = str(e)[:200]
     return out
 
 
-# the prefill line is timed once the tensor-core GEMM serves M > 16
-PREFILL_READY = True
+def secondary_sweep(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    """bit-width sweep: N = K = 8192, bits x group size x M, weights rotating
+    over copies > 3x L2"""
+    out = {}
+    by_w = {}
+    for c in wl.WORKLOADS.sweep:
+        by_w.setdefault((c.bits, c.group_size), []).append(c)
+    for (bits, gs), cs in by_w.items():
+        qw = api.qmm_quantize(wl.gen_weight(8192, 8192, 2000 + 100 * bits + gs).to(dev), gs, bits,
+                              torch.bfloat16)
+        wbytes = 8192 * 8192 * bits // 8 + 8192 * (8192 // gs) * 4
+        qws = [qw] + [clone_qw(api, qw) for _ in range(copies_for(wbytes) - 1)]
+        for c in cs:
+            x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+            y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+
+            def fn(x=x, y=y):
+                for q in qws:
+                    api.qmm_matmul(x, q, True, out=y, stream=stream)
+            t = time_graph(torch, fn, stream, reps=10, inner=1) / len(qws)
+            out[c.name] = _gbs(decode_bytes(c.M, c.N, c.K, c.bits, c.group_size), t, hbm_peak)
+        del qws, qw
+        torch.cuda.empty_cache()
+    return out
 
 
-def _has_tc_gemm():
-    return PREFILL_READY
+def secondary_prefill(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    """prefill GEMMs (tensor-bound): TFLOP/s against the measured burst and the
+    datasheet dense bf16 peak"""
+    out = {}
+    for c in wl.WORKLOADS.prefill:
+        qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), 64, 4, torch.bfloat16)
+        x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+        y = torch.empty(c.M, c.N, dtype=torch.bfloat16, device=dev)
+        t = time_graph(torch, lambda: api.qmm_matmul(x, qw, True, out=y, stream=stream), stream,
+                       reps=10, inner=3)
+        tf = 2 * c.M * c.N * c.K / (t * 1e-3) / 1e12
+        out[c.name] = {"TFLOP/s": round(tf, 1), "frac_of_measured_burst": round(tf / bf16_peak, 3),
+                       "frac_of_datasheet_2250": round(tf / BF16_DATASHEET_TFLOPS, 3),
+                       "us": round(t * 1e3, 1)}
+        del qw, x, y
+    return out
 
 
 # ---------------------------------------------------------------- oracle arms
@@ -509,25 +618,36 @@ def _oracle_step(oracle, ins, threads, frac):
     return nbytes
 
 
-def cpu_baseline(wl, seconds):
-    import oracle
-    ins = _oracle_decode_inputs(wl, oracle)
-    threads = cpu_threads()
-    frac = 1.0
+def _time_oracle(oracle, ins, threads, seconds):
+    """bytes/s of the oracle over repeated sampled decode steps for ~seconds"""
     t0 = time.perf_counter()
-    nb = _oracle_step(oracle, ins, threads, 0.05)
+    _oracle_step(oracle, ins, threads, 0.01)
     dt = time.perf_counter() - t0
-    frac = min(1.0, max(0.01, 0.05 * (seconds / 3) / max(dt, 1e-3)))
-    total_b, t0 = 0.0, time.perf_counter()
-    reps = 0
+    # size the sample so one pass takes about a tenth of the budget
+    frac = min(1.0, max(0.002, 0.01 * (seconds / 10) / max(dt, 1e-4)))
+    total_b, reps, t0 = 0.0, 0, time.perf_counter()
     while time.perf_counter() - t0 < seconds and reps < 1000:
         total_b += _oracle_step(oracle, ins, threads, frac)
         reps += 1
     dt = time.perf_counter() - t0
-    return {"value": round(total_b / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"{reps} passes over the first {frac:.1%} of output rows of the 3 decode "
-                      f"GEMVs (M=1), fp64 oracle, {threads} threads, {dt:.1f} s"}
+    return total_b / dt / 1e9, frac, reps, dt
+
+
+def cpu_baseline(wl, seconds):
+    """The oracle as it stands on the host's cores, on a bounded sample of the
+    decode step: single-threaded (the reported baseline) and over every
+    affinity core beside it."""
+    import oracle
+    ins = _oracle_decode_inputs(wl, oracle)
+    threads = cpu_threads()
+    v1, f1, r1, d1 = _time_oracle(oracle, ins, 1, seconds / 2)
+    vn, fn, rn, dn = _time_oracle(oracle, ins, threads, seconds / 2)
+    return {"value": round(v1, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{r1} passes over the first {f1:.2%} of output rows of the 3 decode GEMVs "
+                      f"(M=1), fp64 oracle, 1 thread, {d1:.1f} s",
+            "all_cores": {"value": round(vn, 5), "unit": "GB/s", "cores": threads,
+                          "sample": f"{rn} passes over the first {fn:.2%} of output rows, "
+                                    f"{threads} threads, {dn:.1f} s"}}
 
 
 def run_reference(args):
@@ -612,7 +732,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=16.0,
+                    help="oracle CPU baseline budget (half single-thread, half all cores)")
+    ap.add_argument("--clock-window", type=float, default=0.3,
+                    help="seconds of repeated K-step trials the clock sampler sees")
     ap.add_argument("--profile", default=None,
                     help="run a few launches of one named case (e.g. decode_14336x4096) for ncu")
     ap.add_argument("--profile-launches", type=int, default=3)
@@ -622,7 +745,7 @@ def main():
         return
     args.steps_given = args.steps is not None
     if args.steps is None:
-        args.steps = 20000
+        args.steps = 200
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -220,6 +220,24 @@ qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype
                                                 qmm_dtype out_dtype, int32_t* d_status,
                                                 void* stream);
 
+/* Diagnostic of the bounded device-side waits (not a step of the method).
+ * Every TMA-fed kernel here waits on shared-memory mbarriers with a poll
+ * limit and reports QMM_ERR_TIMEOUT instead of hanging when a wait gives up.
+ * This call runs one tiny kernel that waits on a barrier nothing arrives on:
+ *   d_result[0] = 1 if a wait on the already-completed phase returned at once,
+ *   d_result[1] = 1 if the wait on the pending phase completed (expected 0:
+ *                 it gives up after `spins` polls and ORs QMM_ERR_TIMEOUT into
+ *                 *d_status),
+ *   d_result[2] = 1 if the abortable wait completed with the abort flag
+ *                 raised (expected 0).
+ * d_result: device int32[3]; d_status: device int32, caller-zeroed; both
+ * 4-byte aligned and required.  spins in [1, 2^22] (QMM_ERR_INVALID_ARG
+ * otherwise).  Touches no memory but these two buffers and its own shared
+ * memory; no copy is ever in flight.  Errors: INVALID_ARG, ALIGNMENT,
+ * UNSUPPORTED (device), CUDA. */
+qmm_status qmm_selftest_bounded_wait(uint32_t spins, int32_t* d_result, int32_t* d_status,
+                                     void* stream);
+
 #ifdef __cplusplus
 }
 #endif

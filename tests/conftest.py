@@ -27,3 +27,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # worst observed parity ratios, when QMM_PARITY_REPORT names a file
+    try:
+        from tests.helpers import write_report
+    except Exception:  # pragma: no cover
+        return
+    write_report()

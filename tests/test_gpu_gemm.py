@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle
-from tests.helpers import ORC, gate, np_storage, qweight_np, rne_equal
+from tests.helpers import ORC, Guarded, gate, np_storage, qweight_np, rne_equal
 from weight_only_quantized_qmm_b200 import api
 from weight_only_quantized_qmm_b200 import workloads as wl
 
@@ -15,13 +15,15 @@ DTS = {torch.bfloat16: "bf16", torch.float16: "f16"}
 
 
 def _case(M, N, K, bits, gs, dtype, seed):
+    """fp32 and 16-bit outputs in poisoned buffers with guard bands."""
     w = wl.gen_weight(N, K, seed)
     qw = api.qmm_quantize(w.to(DEV), gs, bits, dtype)
     x = wl.gen_x(M, K, seed + 1, DTS[dtype])
-    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
-    y16 = api.qmm_matmul(x.to(DEV), qw, True, dtype)
+    g32, g16 = Guarded((M, N), torch.float32), Guarded((M, N), dtype)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g32.out)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g16.out)
     torch.cuda.synchronize()
-    return x, qw, y32, y16
+    return x, qw, g32.check("y32"), g16.check("y16")
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 6, 8])
@@ -62,20 +64,38 @@ def test_gemm_weight_operand_equals_bf16_dequant():
         assert torch.equal(y[i].cpu(), deq[:, 5 * i].cpu())
 
 
+def _tile_cover(n, tile, per_tile, rng):
+    """per_tile distinct indices in every tile of `tile` along [0, n), always
+    including the first and last index of each tile"""
+    out = []
+    for t0 in range(0, n, tile):
+        t1 = min(n, t0 + tile)
+        pick = {t0, t1 - 1}
+        while len(pick) < min(per_tile, t1 - t0):
+            pick.add(int(rng.integers(t0, t1)))
+        out.extend(sorted(pick))
+    return np.array(out)
+
+
 @pytest.mark.parametrize("case", wl.WORKLOADS.prefill, ids=lambda c: c.name)
-def test_prefill_full_size_sampled(case):
+def test_prefill_full_size(case):
+    """Every (256-token, 128-row) output tile of the GEMM is checked: all N
+    columns of 3 tokens in every 256-token tile, and all M tokens of 3
+    weight rows in every 128-row tile, against the oracle; the whole 16-bit
+    output equals RNE of the fp32 output; every output written, guard bands
+    intact (poisoned buffers)."""
     x, qw, y32, y16 = _case(case.M, case.N, case.K, case.bits, case.group_size, torch.bfloat16,
                             case.seed)
     p, s, b = qweight_np(qw)
     rng = np.random.default_rng(case.seed)
-    ms = np.concatenate([rng.integers(0, case.M, 300), [0, case.M - 1]])
-    ns = np.concatenate([rng.integers(0, case.N, 300), [case.N - 1, 0]])
-    coords = list(zip(ms.tolist(), ns.tolist()))
-    yref = oracle.matmul_elements(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
-                                  case.group_size, case.bits, coords)
-    got = y32.cpu().numpy()[ms, ns]
-    gate(got, yref, case.name)
-    # bf16 output: the same kernel's fp32 result rounded once
-    idx = torch.tensor(ms), torch.tensor(ns)
-    assert torch.equal(y16.cpu()[idx].view(torch.int16), y32.cpu()[idx].to(torch.bfloat16).view(torch.int16))
-    assert torch.isfinite(y16).all()
+    xs = np_storage(x)
+    y = y32.cpu().numpy()
+    toks = _tile_cover(case.M, 256, 3, rng)
+    ref_t = oracle.matmul(xs[toks], oracle.BF16, p, s, b, oracle.BF16, case.N, case.group_size,
+                          case.bits)
+    gate(y[toks], ref_t, case.name + " token rows")
+    rows = _tile_cover(case.N, 128, 3, rng)
+    ref_r = oracle.matmul(xs, oracle.BF16, p[rows], s[rows], b[rows], oracle.BF16, len(rows),
+                          case.group_size, case.bits)
+    gate(y[:, rows], ref_r, case.name + " weight rows")
+    rne_equal(y16, y32)

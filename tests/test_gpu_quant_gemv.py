@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import oracle
-from tests.helpers import ORC, gate, np_storage, packed_np, qweight_np, rne_equal
+from tests.helpers import ORC, Guarded, gate, np_storage, packed_np, qweight_np, rne_equal
 from weight_only_quantized_qmm_b200 import api
 from weight_only_quantized_qmm_b200 import workloads as wl
 
@@ -60,20 +60,26 @@ def test_quantize_degenerate_groups():
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16, torch.float16])
 def test_dequantize_bit_exact(bits, gs, out_dtype):
     _, qw, (p_ref, s_ref, b_ref) = _quant_pair(19, 2 * gs, bits, gs, torch.bfloat16, 40 + bits)
-    out = api.qmm_dequantize(qw, out_dtype)
+    g = Guarded((19, 2 * gs), out_dtype)
+    api.qmm_dequantize(qw, out=g.out)
     torch.cuda.synchronize()
+    out = g.check("dequant")
     ref = oracle.dequantize(p_ref, s_ref, b_ref, oracle.BF16, 2 * gs, gs, bits, ORC[out_dtype])
     assert np.array_equal(np_storage(out), ref)
 
 
 # ------------------------------------------------------------------ decode GEMV (M <= 16)
 def _gemv_case(M, N, K, bits, gs, dtype, seed):
+    """fp32 and 16-bit outputs of one call each, in poisoned buffers with guard
+    bands (every output written, nothing past the end touched)."""
     w, qw, (p, s, b) = _quant_pair(N, K, bits, gs, dtype, seed)
     x = wl.gen_x(M, K, seed + 1, {torch.bfloat16: "bf16", torch.float16: "f16",
                                   torch.float32: "f32"}[dtype])
-    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
-    y16 = api.qmm_matmul(x.to(DEV), qw, True, dtype)
+    g32, g16 = Guarded((M, N), torch.float32), Guarded((M, N), dtype)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g32.out)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g16.out)
     torch.cuda.synchronize()
+    y32, y16 = g32.check("y32"), g16.check("y16")
     yref = oracle.matmul(np_storage(x), ORC[dtype], p, s, b, ORC[dtype], N, gs, bits)
     return y32, y16, yref
 
@@ -219,28 +225,27 @@ def test_zero_rows_is_noop():
     assert tuple(y.shape) == (0, 64)
 
 
-# ------------------------------------------------------------------ full-size decode, sampled
+# ------------------------------------------------------------------ full-size decode and sweep
+# Every output element of every full-size call is compared with the oracle;
+# outputs sit in poisoned buffers with guard bands; the quantizer is checked
+# bit for bit on every row.
 @pytest.mark.parametrize("case", wl.WORKLOADS.decode, ids=lambda c: c.name)
-def test_decode_full_size_sampled(case):
+def test_decode_full_size(case):
     w = wl.gen_weight(case.N, case.K, case.seed)
     x = wl.gen_x(case.M, case.K, case.seed + 1)
     qw = api.qmm_quantize(w.to(DEV), case.group_size, case.bits, torch.bfloat16)
-    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
-    y16 = api.qmm_matmul(x.to(DEV), qw)
+    g32, g16 = Guarded((case.M, case.N), torch.float32), Guarded((case.M, case.N), torch.bfloat16)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g32.out)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g16.out)
     torch.cuda.synchronize()
+    y32, y16 = g32.check(case.name), g16.check(case.name)
     p, s, b = qweight_np(qw)
-    rng = np.random.default_rng(case.seed)
-    cols = np.unique(np.concatenate([rng.integers(0, case.N, 384), [0, case.N - 1]]))
-    coords = [(0, int(n)) for n in cols]
-    yref = oracle.matmul_elements(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
-                                  case.group_size, case.bits, coords)
-    ys = y32.cpu().numpy()[0, cols]
-    gate(ys, yref, case.name)
+    pr, sr, br = oracle.quantize(w.numpy(), oracle.F32, case.group_size, case.bits, oracle.BF16)
+    assert np.array_equal(p, pr) and np.array_equal(s, sr) and np.array_equal(b, br)
+    yref = oracle.matmul(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
+                         case.group_size, case.bits)
+    gate(y32.cpu().numpy(), yref, case.name)
     rne_equal(y16, y32)
-    # the quantizer itself is exact at full size: spot-check 64 rows
-    rows = rng.integers(0, case.N, 64)
-    pr, sr, br = oracle.quantize(w.numpy()[rows], oracle.F32, case.group_size, case.bits, oracle.BF16)
-    assert np.array_equal(p[rows], pr) and np.array_equal(s[rows], sr) and np.array_equal(b[rows], br)
 
 
 _SWEEP_W = {}
@@ -254,29 +259,54 @@ def _sweep_weight(bits, gs, seed):
         w = wl.gen_weight(8192, 8192, seed)
         qw = api.qmm_quantize(w.to(DEV), gs, bits, torch.bfloat16)
         torch.cuda.synchronize()
-        _SWEEP_W[key] = (w, qw, qweight_np(qw))
+        p, s, b = qweight_np(qw)
+        pr, sr, br = oracle.quantize(w.numpy(), oracle.F32, gs, bits, oracle.BF16)
+        assert np.array_equal(p, pr) and np.array_equal(s, sr) and np.array_equal(b, br)
+        _SWEEP_W[key] = (w, qw, (p, s, b))
     return _SWEEP_W[key]
 
 
 @pytest.mark.parametrize("case", wl.WORKLOADS.sweep, ids=lambda c: c.name)
-def test_sweep_full_size_sampled(case):
+def test_sweep_full_size(case):
     """Bit-width sweep at full size (N = K = 8192, b in {2,3,6,8}, gs in
-    {32,64,128}, M in {1,4,16}): all rows of the output at 128 sampled columns
-    against the oracle, 16-bit output = RNE of the fp32 output, and a spot
-    check of the quantizer."""
+    {32,64,128}, M in {1,4,16}): every output against the oracle, 16-bit
+    output = RNE of the fp32 output, quantizer bit-exact on every row."""
     w, qw, (p, s, b) = _sweep_weight(case.bits, case.group_size, 2000 + 100 * case.bits + case.group_size)
     x = wl.gen_x(case.M, case.K, case.seed + 1)
-    y32 = api.qmm_matmul(x.to(DEV), qw, True, torch.float32)
-    y16 = api.qmm_matmul(x.to(DEV), qw)
+    g32, g16 = Guarded((case.M, case.N), torch.float32), Guarded((case.M, case.N), torch.bfloat16)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g32.out)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g16.out)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(case.seed)
-    cols = np.unique(np.concatenate([rng.integers(0, case.N, 126), [0, case.N - 1]]))
-    coords = [(m, int(n)) for m in range(case.M) for n in cols]
-    yref = oracle.matmul_elements(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
-                                  case.group_size, case.bits, coords)
-    ys = y32.cpu().numpy()[:, cols].reshape(-1)
-    gate(ys, yref, case.name)
+    y32, y16 = g32.check(case.name), g16.check(case.name)
+    yref = oracle.matmul(np_storage(x), oracle.BF16, p, s, b, oracle.BF16, case.N,
+                         case.group_size, case.bits)
+    gate(y32.cpu().numpy(), yref, case.name)
     rne_equal(y16, y32)
-    rows = rng.integers(0, case.N, 16)
-    pr, sr, br = oracle.quantize(w.numpy()[rows], oracle.F32, case.group_size, case.bits, oracle.BF16)
-    assert np.array_equal(p[rows], pr) and np.array_equal(s[rows], sr) and np.array_equal(b[rows], br)
+
+
+@pytest.mark.parametrize("M", [1, 4, 32])
+def test_quantize_then_matmul_back_to_back(M):
+    """The weights are rewritten by qmm_quantize immediately before qmm_matmul
+    on the same stream, with no synchronization in between: the matmul must
+    see the new weights (its kernels read nothing before the previous kernel
+    in the stream has completed)."""
+    from weight_only_quantized_qmm_b200 import _lib
+    N, K = 4096, 4096
+    w1 = wl.gen_weight(N, K, 950).to(DEV)
+    w2 = wl.gen_weight(N, K, 951).to(DEV)
+    x = wl.gen_x(M, K, 952).to(DEV)
+    qw = api.qmm_quantize(w1, 64, 4, torch.bfloat16)
+    api.qmm_matmul(x, qw, True, torch.float32)
+    torch.cuda.synchronize()
+    L = _lib.load()
+    st = int(torch.cuda.current_stream().cuda_stream)
+    y = torch.empty(M, N, dtype=torch.float32, device=DEV)
+    rc = L.qmm_quantize(w2.data_ptr(), _lib.QMM_F32, N, K, 64, 4, _lib.QMM_BF16, qw.packed.data_ptr(),
+                        qw.scales.data_ptr(), qw.biases.data_ptr(), st)
+    assert rc == 0
+    api.qmm_matmul(x, qw, True, out=y)
+    torch.cuda.synchronize()
+    p, s, b = oracle.quantize(w2.cpu().numpy(), oracle.F32, 64, 4, oracle.BF16)
+    assert np.array_equal(packed_np(qw.packed), p)
+    yref = oracle.matmul(np_storage(x.cpu()), oracle.BF16, p, s, b, oracle.BF16, N, 64, 4)
+    gate(y.cpu().numpy(), yref, f"quantize->matmul M{M}")

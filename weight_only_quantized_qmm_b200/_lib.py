@@ -29,7 +29,7 @@ EXPORTS = (
     "qmm_packed_words_per_row", "qmm_groups_per_row", "qmm_status_string", "qmm_device_check",
     "qmm_quantize", "qmm_dequantize", "qmm_matmul", "qmm_moe_gemv_id",
     "qmm_moe_gemv_id_batched", "qmm_moe_gemv_id_gate_up_silu",
-    "qmm_moe_gemv_id_gate_up_silu_batched",
+    "qmm_moe_gemv_id_gate_up_silu_batched", "qmm_selftest_bounded_wait",
 )
 
 
@@ -89,6 +89,8 @@ def load() -> ctypes.CDLL:
     L.qmm_moe_gemv_id_gate_up_silu_batched.argtypes = [vp, c_int, vp, i64, i64, i64, i64, stp,
                                                        stp, vp, c_int, vp, vp]
     L.qmm_moe_gemv_id_gate_up_silu_batched.restype = c_int
+    L.qmm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp, vp, vp]
+    L.qmm_selftest_bounded_wait.restype = c_int
     _lib = L
     return L
 

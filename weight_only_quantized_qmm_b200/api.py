@@ -36,6 +36,54 @@ def _ptr(t) -> int:
     return int(t.data_ptr())
 
 
+def _need(t, what: str, numel: int, dtypes=None) -> None:
+    """Refuse a tensor the kernels would read or write out of bounds: it must
+    hold at least `numel` elements (of one of `dtypes` when given) and be
+    contiguous.  Raises ValueError before any call into the library."""
+    if t is None:
+        raise ValueError(f"qmm: {what} is required")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"qmm: {what} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"qmm: {what} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"qmm: {what} holds {t.numel()} elements, the call needs {numel}")
+
+
+def _on_device(**named) -> None:
+    """Every given tensor is a CUDA tensor on the current device (where the
+    library launches).  Raises ValueError otherwise."""
+    cur = None
+    for what, t in named.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"qmm: {what} must be a CUDA tensor, got one on {t.device}")
+        if cur is None:
+            cur = torch.cuda.current_device()
+        if t.device.index != cur:
+            raise ValueError(f"qmm: {what} is on {t.device}, but the current device is cuda:{cur} "
+                             "(the call runs there)")
+
+
+def _words(cols: int, bits: int) -> int:
+    wpr = qmm_packed_words_per_row(cols, bits)
+    if wpr < 0:
+        check("qmm", _lib.QMM_ERR_INVALID_ARG)
+    return wpr
+
+
+def _groups(cols: int, group_size: int) -> int:
+    G = qmm_groups_per_row(cols, group_size)
+    if G < 0:
+        check("qmm", _lib.QMM_ERR_INVALID_ARG)
+    return G
+
+
+_PACKED = (torch.int32,)
+_FLOAT = (torch.float32, torch.float16, torch.bfloat16)
+
+
 def _stream(stream=None) -> int:
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(s.cuda_stream)
@@ -54,6 +102,16 @@ class QWeight:
     bits: int
     mode: int = QMM_MODE_AFFINE
 
+    def validate(self) -> dict:
+        """packed, scales and biases hold rows x (words | groups) elements;
+        returns them by name for the device check."""
+        n = self.rows
+        _need(self.packed, "packed", n * _words(self.cols, self.bits), _PACKED)
+        G = _groups(self.cols, self.group_size)
+        _need(self.scales, "scales", n * G, _FLOAT)
+        _need(self.biases, "biases", n * G, (self.scales.dtype,))
+        return {"packed": self.packed, "scales": self.scales, "biases": self.biases}
+
     def c(self) -> QWeightC:
         return QWeightC(_ptr(self.packed), _ptr(self.scales), _ptr(self.biases),
                         dtype_code(self.scales.dtype), self.rows, self.cols, self.group_size,
@@ -71,6 +129,17 @@ class ExpertStack:
     n_cols: int
     group_size: int
     bits: int
+
+    def validate(self, role: str = "") -> dict:
+        """packed, scales and biases hold num_experts x n_rows x (words |
+        groups) elements; returns them by name for the device check."""
+        n = self.num_experts * self.n_rows
+        _need(self.packed, role + "packed", n * _words(self.n_cols, self.bits), _PACKED)
+        G = _groups(self.n_cols, self.group_size)
+        _need(self.scales, role + "scales", n * G, _FLOAT)
+        _need(self.biases, role + "biases", n * G, (self.scales.dtype,))
+        return {role + "packed": self.packed, role + "scales": self.scales,
+                role + "biases": self.biases}
 
     def c(self) -> ExpertStackC:
         return ExpertStackC(_ptr(self.packed), _ptr(self.scales), _ptr(self.biases),
@@ -101,20 +170,43 @@ def qmm_device_check() -> int:
     return int(_lib.load().qmm_device_check())
 
 
+def qmm_selftest_bounded_wait(spins: int, d_result: torch.Tensor, d_status: torch.Tensor,
+                              stream=None) -> None:
+    """Run the bounded-wait diagnostic kernel (see include/qmm.h)."""
+    _need(d_result, "d_result", 3, (torch.int32,))
+    _need(d_status, "d_status", 1, (torch.int32,))
+    _on_device(d_result=d_result, d_status=d_status)
+    rc = _lib.load().qmm_selftest_bounded_wait(int(spins), _ptr(d_result), _ptr(d_status),
+                                               _stream(stream))
+    check("qmm_selftest_bounded_wait", rc)
+
+
 # ------------------------------------------------------------------ calls
+def _last_pair_end(n_pairs: int, top_k: int, outer: int, inner: int, n_cols: int) -> int:
+    """Elements of `a` the last pair reads up to (batched pair offsets)."""
+    if n_pairs == 0:
+        return 0
+    last = n_pairs - 1
+    return (last // top_k) * outer + (last % top_k) * inner + n_cols
+
+
 def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4,
                  s_dtype: torch.dtype | None = None, stream=None) -> QWeight:
     """Dense [rows, cols] -> QWeight (scales/biases in s_dtype, default w.dtype)."""
+    if w.dim() != 2:
+        raise ValueError(f"qmm_quantize: w must be 2-D, got shape {tuple(w.shape)}")
     rows, cols = w.shape
     s_dtype = s_dtype or w.dtype
     wpr = qmm_packed_words_per_row(cols, bits)
     G = qmm_groups_per_row(cols, group_size)
     if wpr < 0 or G < 0:
         check("qmm_quantize", _lib.QMM_ERR_INVALID_ARG)
+    w = w.contiguous()
+    _need(w, "w", rows * cols, _FLOAT)
+    _on_device(w=w)
     packed = torch.empty(rows, wpr, dtype=torch.int32, device=w.device)
     scales = torch.empty(rows, G, dtype=s_dtype, device=w.device)
     biases = torch.empty(rows, G, dtype=s_dtype, device=w.device)
-    w = w.contiguous()
     rc = _lib.load().qmm_quantize(_ptr(w), dtype_code(w.dtype), rows, cols, group_size, bits,
                                   dtype_code(s_dtype), _ptr(packed), _ptr(scales), _ptr(biases),
                                   _stream(stream))
@@ -124,8 +216,11 @@ def qmm_quantize(w: torch.Tensor, group_size: int = 64, bits: int = 4,
 
 def qmm_dequantize(qw: QWeight, out_dtype: torch.dtype = torch.float32, out=None,
                    stream=None) -> torch.Tensor:
+    ws = qw.validate()
     if out is None:
         out = torch.empty(qw.rows, qw.cols, dtype=out_dtype, device=qw.packed.device)
+    _need(out, "out", qw.rows * qw.cols, _FLOAT)
+    _on_device(out=out, **ws)
     c = qw.c()
     rc = _lib.load().qmm_dequantize(ctypes.byref(c), _ptr(out), dtype_code(out.dtype),
                                     _stream(stream))
@@ -141,8 +236,14 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
     x2 = x.reshape(-1, K).contiguous()
     M = x2.shape[0]
     N = qw.rows if transpose else qw.cols
+    _need(x2, "x", M * K, _FLOAT)
+    ws = qw.validate()
     if out is None:
-        out = torch.empty(M, N, dtype=y_dtype or x.dtype, device=x.device)
+        out = torch.empty(M, N, dtype=y_dtype or x.dtype, device=x2.device)
+    _need(out, "out", M * N, _FLOAT)
+    if out.numel() != M * N:
+        raise ValueError(f"qmm_matmul: out holds {out.numel()} elements, expected {M}x{N}")
+    _on_device(x=x2, out=out, **ws)
     c = qw.c()
     rc = _lib.load().qmm_matmul(_ptr(x2), dtype_code(x2.dtype), M, K, ctypes.byref(c),
                                 int(bool(transpose)), _ptr(out), dtype_code(out.dtype),
@@ -151,11 +252,24 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
     return out.reshape(*lead, N)
 
 
+def _moe_checks(a, ids, n_pairs, top_k, outer, inner, stacks, out, n_out_rows, d_status):
+    _need(a, "a", _last_pair_end(n_pairs, top_k, outer, inner, stacks[0].n_cols), _FLOAT)
+    named = {}
+    for role, st in zip(("", "up."), stacks):
+        named.update(st.validate(role))
+    _need(ids, "ids", n_pairs, (torch.int32,))
+    _need(out, "out", n_pairs * n_out_rows, _FLOAT)
+    if d_status is not None:
+        _need(d_status, "d_status", 1, (torch.int32,))
+    _on_device(a=a, ids=ids, out=out, d_status=d_status, **named)
+
+
 def qmm_moe_gemv_id(a: torch.Tensor, ids: torch.Tensor, n_selected: int, src1_stride: int,
                     w: ExpertStack, out_dtype: torch.dtype | None = None, out=None,
                     d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(n_selected, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    _moe_checks(a, ids, n_selected, 1, src1_stride, 0, (w,), out, w.n_rows, d_status)
     c = w.c()
     rc = _lib.load().qmm_moe_gemv_id(_ptr(a), dtype_code(a.dtype), _ptr(ids), n_selected,
                                      src1_stride, ctypes.byref(c), _ptr(out),
@@ -170,6 +284,9 @@ def qmm_moe_gemv_id_batched(a: torch.Tensor, ids: torch.Tensor, m: int, top_k: i
                             d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(m * top_k, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    if top_k > 0:
+        _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (w,), out, w.n_rows,
+                    d_status)
     c = w.c()
     rc = _lib.load().qmm_moe_gemv_id_batched(_ptr(a), dtype_code(a.dtype), _ptr(ids), m, top_k,
                                              outer_stride, inner_stride, ctypes.byref(c),
@@ -186,6 +303,7 @@ def qmm_moe_gemv_id_gate_up_silu(a: torch.Tensor, ids: torch.Tensor, n_selected:
                                  stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(n_selected, gate.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    _moe_checks(a, ids, n_selected, 1, 0, 0, (gate, up), out, gate.n_rows, d_status)
     cg, cu = gate.c(), up.c()
     rc = _lib.load().qmm_moe_gemv_id_gate_up_silu(_ptr(a), dtype_code(a.dtype), _ptr(ids),
                                                   n_selected, ctypes.byref(cg), ctypes.byref(cu),
@@ -203,6 +321,9 @@ def qmm_moe_gemv_id_gate_up_silu_batched(a: torch.Tensor, ids: torch.Tensor, m: 
                                          stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(m * top_k, gate.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    if top_k > 0:
+        _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (gate, up), out,
+                    gate.n_rows, d_status)
     cg, cu = gate.c(), up.c()
     rc = _lib.load().qmm_moe_gemv_id_gate_up_silu_batched(
         _ptr(a), dtype_code(a.dtype), _ptr(ids), m, top_k, outer_stride, inner_stride,

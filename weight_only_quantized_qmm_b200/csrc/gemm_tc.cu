@@ -23,6 +23,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "mbarrier.cuh"
 
 namespace qmm {
 
@@ -43,33 +44,10 @@ constexpr uint32_t kSpins = 1u << 22;
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void bar_init(uint32_t b, uint32_t n) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(n));
-}
-__device__ __forceinline__ void bar_arrive(uint32_t b) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
-}
-__device__ __forceinline__ void bar_expect(uint32_t b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(b),
-               "r"(bytes)
-               : "memory");
-}
 // Bounded wait on an mbarrier phase.  Gives up (returns false) after kSpins
 // polls, or as soon as another role of the CTA has raised the abort flag.
 __device__ __forceinline__ bool bar_wait(uint32_t b, uint32_t parity, const int* abort_flag) {
-  for (uint32_t i = 0; i < gemm::kSpins; ++i) {
-    if ((i & 1023u) == 1023u && *reinterpret_cast<const volatile int*>(abort_flag)) return false;
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(b), "r"(parity)
-        : "memory");
-    if (done) return true;
-  }
-  return false;
+  return mbar_wait_abortable(b, parity, gemm::kSpins, abort_flag);
 }
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* m, int c0, int c1,
                                        uint32_t b) {
@@ -220,11 +198,11 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      bar_init(full0 + 8 * s, 1);
-      bar_init(afull0 + 8 * s, 4);
-      bar_init(empty0 + 8 * s, 1);
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(afull0 + 8 * s, 4);
+      mbar_init(empty0 + 8 * s, 1);
     }
-    bar_init(accf, 1);
+    mbar_init(accf, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -240,12 +218,18 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      int issued = 0;
       for (int i = 0; i < nk; ++i) {
         const int s = i % kStages, u = i / kStages;
         if (i >= kStages && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) { *abort_flag = 1; break; }
-        bar_expect(full0 + 8 * s, kXStage);
+        mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
         tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, m0, full0 + 8 * s);
+        issued = i + 1;
       }
+      // no copy may still be landing when the CTA exits: the last copy of every
+      // slot is waited for with the full bound, also after an abort
+      for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+        mbar_wait_n(full0 + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u, gemm::kSpins);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -350,12 +334,15 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
       __syncwarp();
-      if (lane == 0) bar_arrive(afull0 + 8 * s);
+      if (lane == 0) mbar_arrive(afull0 + 8 * s);
     }
     }
 
     // ---------------- epilogue: TMEM -> registers -> smem transpose -> y ----------------
-    const bool ok = bar_wait(accf, 0, abort_flag) && !*reinterpret_cast<volatile int*>(abort_flag);
+    // the MMA warp commits accf on every path (also after an abort), so this
+    // wait ignores the abort flag: TMEM is read and released only once every
+    // issued MMA has completed
+    const bool ok = mbar_wait_n(accf, 0, gemm::kSpins) && !*reinterpret_cast<volatile int*>(abort_flag);
     tc_fence_after();
     const bool f32out = p.y_dtype == QMM_F32;
     // staging tile [256 tokens][128 rows] in the (now idle) pipeline buffers

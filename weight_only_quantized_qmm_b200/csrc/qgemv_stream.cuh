@@ -34,10 +34,11 @@
 // Every wait is bounded: a timeout sets QMM_ERR_TIMEOUT, skips the remaining
 // arithmetic and still drains the copies in flight before the CTA exits.
 //
-// Launched with programmatic stream serialization: for dense calls the
-// producer streams weights (which no earlier kernel writes) before
-// griddepcontrol.wait, so a call's weight traffic can start while the
-// previous kernel drains; ids, x and y are only touched after the wait.
+// Launched with programmatic stream serialization: the CTA's set-up (barrier
+// initialisation, shared-memory carve-up) overlaps the previous kernel's
+// tail; every global read (weights, ids, x) comes after griddepcontrol.wait,
+// so whatever the previous kernel in the stream wrote -- weights included --
+// is visible.
 #pragma once
 
 #include <cuda.h>
@@ -98,9 +99,6 @@ __device__ __forceinline__ void sts128(uint32_t a, float4 v) {
                : "memory");
 }
 __device__ __forceinline__ float ldsf(uint32_t a) { return __uint_as_float(lds32(a)); }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
                                             uint32_t bar) {
   asm volatile(
@@ -369,9 +367,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // weights, ids and x may all come from the previous kernel in the stream
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (q.ids) {
-    // the ids (like x) may come from the previous kernel in the stream
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, s_list + q.n_pairs, &s_nd);
     if (tid == 0) {
       int run = 0;
@@ -409,7 +407,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   // ---------------------------------------------------------------- producer
   if (warp == C::PRODUCER) {
     if (lane == 0 && nt > 0) {
-      bool failed = false;
       int ku = 0, issued = 0;
       Walk w;
       w.start(tb, p.ntiles_e, s_seg, nd);
@@ -417,7 +414,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         const int slot = i % STAGES;
         if (i >= STAGES &&
             !mbar_wait(bar_full + 8 * kMaxStages + 8 * slot, (uint32_t)((i / STAGES) - 1) & 1u, false)) {
-          failed = true;
           set_status(q.d_status, QMM_ERR_TIMEOUT);
           break;
         }
@@ -440,13 +436,13 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           if (i + 1 < nunits) w.next(p.ntiles_e, s_seg, nd);
         }
       }
-      // no copy may still be landing when the CTA exits
+      // no copy may still be landing when the CTA exits: wait (full bound,
+      // even after a failure) for the last copies of every slot
       for (int i = issued > STAGES ? issued - STAGES : 0; i < issued; ++i)
-        if (!mbar_wait(bar_full + 8 * (i % STAGES), (uint32_t)(i / STAGES) & 1u, failed)) failed = true;
+        mbar_wait_n(bar_full + 8 * (i % STAGES), (uint32_t)(i / STAGES) & 1u, kMbarSpins);
     }
     return;
   }
-  if (!q.ids) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // ---------------------------------------------------------------- epilogue
   if (warp == C::EPILOGUE) {

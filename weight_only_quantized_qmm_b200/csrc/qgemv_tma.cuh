@@ -14,40 +14,17 @@
 
 #include <cuda.h>
 
+#include "mbarrier.cuh"
 #include "qgemv_impl.cuh"
 
 namespace qmm {
 
 // ------------------------------------------------------------------ mbarrier / TMA
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-// Bounded wait on a phase of an mbarrier: gives up after kMbarSpins polls
-// (each try_wait may suspend the thread for a while) and returns false.
-constexpr uint32_t kMbarSpins = 1u << 20;
-// After a first failure the warp only polls briefly (`failed`), so a broken
-// copy cannot stretch the kernel by one full timeout per remaining stage.
+// In a pipeline loop, after a first failure the warp only polls briefly
+// (`failed`), so a broken copy cannot stretch the kernel by one full timeout
+// per remaining stage; draining copies already issued uses the full bound.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool failed) {
-  const uint32_t spins = failed ? 1024u : kMbarSpins;
-  for (uint32_t i = 0; i < spins; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+  return mbar_wait_n(bar, parity, failed ? 1024u : kMbarSpins);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
@@ -213,8 +190,11 @@ qgemv_tma_kernel(const QgemvParams p, const __grid_constant__ CUtensorMap tm0,
             ssrc[i] = sok[i] ? reinterpret_cast<const uint32_t*>(arrp) + (e0 >> 1) + jw : safe_src;
           }
 
+          // stages of this chunk whose copies were issued; none after a failure
+          int n_issued = 0;
           auto issue = [&](int st) {
-            if (st < nst) {
+            if (st < nst && !failed) {
+              n_issued = st + 1;
               const uint32_t k = (used + (uint32_t)st) % STAGES;
               const int g0 = gbeg + st * SG;
               const int nu = min(SG, gend - g0);
@@ -264,10 +244,14 @@ qgemv_tma_kernel(const QgemvParams p, const __grid_constant__ CUtensorMap tm0,
             issue(st + STAGES - 1);
             const uint32_t k = (used + (uint32_t)st) % STAGES;
             const uint32_t parity = ((used + (uint32_t)st) / STAGES) & 1u;
-            // every issued stage is waited on (bounded), so nothing is in flight at exit
-            if (!mbar_wait(bar_base + 8 * k, parity, failed) && !failed) {
-              failed = true;
-              if (lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+            // every issued stage is waited on with the full bound (also after a
+            // failure), so no copy is in flight at exit; `failed` is warp-uniform
+            if (st < n_issued) {
+              const bool ok = mbar_wait(bar_base + 8 * k, parity, false);
+              if (__any_sync(0xffffffffu, !ok)) {
+                if (!failed && lane == 0) set_status(p.d_status, QMM_ERR_TIMEOUT);
+                failed = true;
+              }
             }
             cp_async_wait<STAGES - 1>();
             __syncwarp();
