@@ -696,7 +696,19 @@ def run_profile(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     name = args.profile
-    if name.startswith("decode"):
+    if name == "decode_all":
+        # one launch of each decode shape per repetition (per-shape DRAM traffic)
+        fns = []
+        for c in wl.WORKLOADS.decode:
+            qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), c.group_size, c.bits,
+                                  torch.bfloat16)
+            x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
+            fns.append(lambda x=x, qw=qw: api.qmm_matmul(x, qw))
+
+        def fn():
+            for f in fns:
+                f()
+    elif name.startswith("decode"):
         c = [d for d in wl.WORKLOADS.decode if d.name == name][0]
         qw = api.qmm_quantize(wl.gen_weight(c.N, c.K, c.seed).to(dev), c.group_size, c.bits,
                               torch.bfloat16)

@@ -236,6 +236,31 @@ def matmul(x, x_dtype: int, packed, scales, biases, s_dtype: int, N: int, group_
     return y
 
 
+def widen_f64(x, x_dtype: int) -> np.ndarray:
+    """Storage-form activations (float32, or the uint16 bit patterns of f16 /
+    bf16) as float64: exact widening, element by element by definition
+    (bf16 = the high half of an fp32; f16 = IEEE binary16)."""
+    x = np.ascontiguousarray(x)
+    if x_dtype == BF16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    if x_dtype == F16:
+        return x.view(np.float16).astype(np.float64)
+    return x.astype(np.float64)
+
+
+def matmul_dense(x, x_dtype: int, packed, scales, biases, s_dtype: int, N: int, group_size: int,
+                 bits: int, n_threads=None) -> np.ndarray:
+    """fp64 y[M, N] = x . dequant(W)^T for whole-output checks of large
+    calls: the weights are dequantized by this oracle (fmaf, bit-exact) and
+    widened to fp64, then the product is one library fp64 matrix multiply
+    (numpy).  Same definition as matmul(); only the summation order differs,
+    so the two agree within K * 2^-53 * sum |x| |w| per element."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    w = dequantize(packed, scales, biases, s_dtype, K, group_size, bits, F32, n_threads)
+    return widen_f64(x, x_dtype) @ w.astype(np.float64).T
+
+
 def matmul_elements(x, x_dtype: int, packed, scales, biases, s_dtype: int, N: int,
                     group_size: int, bits: int, coords, transpose: bool = True,
                     n_threads=None) -> np.ndarray:

@@ -79,22 +79,26 @@ def _tile_cover(n, tile, per_tile, rng):
 
 @pytest.mark.parametrize("case", wl.WORKLOADS.prefill, ids=lambda c: c.name)
 def test_prefill_full_size(case):
-    """Every (256-token, 128-row) output tile of the GEMM is checked: all N
-    columns of 3 tokens in every 256-token tile, and all M tokens of 3
-    weight rows in every 128-row tile, against the oracle; the whole 16-bit
-    output equals RNE of the fp32 output; every output written, guard bands
-    intact (poisoned buffers)."""
+    """Every output of the GEMM against the oracle's dequantized weights in an
+    fp64 library GEMM (oracle.matmul_dense); in addition the plain oracle
+    loops check 2 tokens of every 256-token tile and 2 weight rows of every
+    128-row tile; the whole 16-bit output equals RNE of the fp32 output;
+    every output written, guard bands intact (poisoned buffers)."""
     x, qw, y32, y16 = _case(case.M, case.N, case.K, case.bits, case.group_size, torch.bfloat16,
                             case.seed)
     p, s, b = qweight_np(qw)
-    rng = np.random.default_rng(case.seed)
     xs = np_storage(x)
     y = y32.cpu().numpy()
-    toks = _tile_cover(case.M, 256, 3, rng)
+    ref = oracle.matmul_dense(xs, oracle.BF16, p, s, b, oracle.BF16, case.N, case.group_size,
+                              case.bits)
+    gate(y, ref, case.name + " all outputs")
+    del ref
+    rng = np.random.default_rng(case.seed)
+    toks = _tile_cover(case.M, 256, 2, rng)
     ref_t = oracle.matmul(xs[toks], oracle.BF16, p, s, b, oracle.BF16, case.N, case.group_size,
                           case.bits)
     gate(y[toks], ref_t, case.name + " token rows")
-    rows = _tile_cover(case.N, 128, 3, rng)
+    rows = _tile_cover(case.N, 128, 2, rng)
     ref_r = oracle.matmul(xs, oracle.BF16, p[rows], s[rows], b[rows], oracle.BF16, len(rows),
                           case.group_size, case.bits)
     gate(y[:, rows], ref_r, case.name + " weight rows")

@@ -310,3 +310,30 @@ def test_quantize_then_matmul_back_to_back(M):
     assert np.array_equal(packed_np(qw.packed), p)
     yref = oracle.matmul(np_storage(x.cpu()), oracle.BF16, p, s, b, oracle.BF16, N, 64, 4)
     gate(y.cpu().numpy(), yref, f"quantize->matmul M{M}")
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_gemv_activation_dynamic_range(bits, M, dtype):
+    """Activations whose magnitude changes by many orders from group to group
+    (and inside a group), all-zero groups and single-spike groups: the decode
+    kernels carry x per group with its own power-of-two range, so every group
+    keeps its precision whatever its neighbours' magnitude."""
+    N, K, gs = 192, 4096, 64
+    w, qw, (p, s, b) = _quant_pair(N, K, bits, gs, dtype, 1300 + bits + M)
+    g = torch.Generator().manual_seed(1301 + M)
+    lim = 30 if dtype == torch.bfloat16 else 4  # f16 holds about 1e-4 .. 6e4 at full precision
+    mag = 10.0 ** torch.randint(-lim, lim + 1, (M, K // gs), generator=g).double()
+    x = (torch.randn(M, K, generator=g, dtype=torch.float64) * mag.repeat_interleave(gs, dim=1))
+    x[:, 3 * gs:4 * gs] = 0.0                       # an all-zero group
+    x[:, 5 * gs:6 * gs] = 0.0
+    x[:, 5 * gs + 17] = 3.0                         # a single spike
+    x[0, 7 * gs:8 * gs] *= torch.logspace(-3, 3, gs, dtype=torch.float64)  # range inside a group
+    x = x.to(dtype)
+    g32 = Guarded((M, N), torch.float32)
+    api.qmm_matmul(x.to(DEV), qw, True, out=g32.out)
+    torch.cuda.synchronize()
+    y = g32.check("y32")
+    yref = oracle.matmul(np_storage(x), ORC[dtype], p, s, b, ORC[dtype], N, gs, bits)
+    gate(y.cpu().numpy(), yref, f"dynamic range b{bits} M{M}")

@@ -471,3 +471,38 @@ def test_moe_bad_id_reports_and_zero_fills():
     ogb, rc = oracle.moe_gate_up_silu_batched(a, oracle.BF16, ids2, 2, 2, 0, 0, st, st)
     assert rc == oracle.ORC_ERR_ID
     assert np.all(ogb[1] == 0) and np.all(ogb[2] == 0) and np.any(ogb[0] != 0)
+
+
+@pytest.mark.parametrize("x_dtype", [oracle.BF16, oracle.F16, oracle.F32])
+def test_widen_f64_matches_the_scalar_conversions(x_dtype):
+    """the vector widening used by matmul_dense equals the C conversions"""
+    rng = np.random.default_rng(7)
+    if x_dtype == oracle.F32:
+        x = rng.standard_normal(64).astype(np.float32)
+        ref = x.astype(np.float64)
+    else:
+        x = rng.integers(0, 1 << 16, 256, dtype=np.uint16)
+        x = x[(x & 0x7C00) != 0x7C00] if x_dtype == oracle.F16 else x[(x & 0x7F80) != 0x7F80]
+        conv = oracle.bf16_to_f32 if x_dtype == oracle.BF16 else oracle.f16_to_f32
+        ref = np.array([conv(int(h)) for h in x], dtype=np.float64)
+    assert np.array_equal(oracle.widen_f64(x, x_dtype), ref)
+
+
+@pytest.mark.parametrize("bits", [3, 4, 8])
+def test_matmul_dense_agrees_with_matmul(bits):
+    """the library-GEMM form and the plain loops compute the same sums: they
+    differ only by summation order, within K * 2^-53 * sum |x| |w|"""
+    N, K, M, gs = 48, 256, 7, 64
+    w = wl.gen_weight(N, K, 30 + bits).numpy()
+    p, s, b = oracle.quantize(w, oracle.F32, gs, bits, oracle.BF16)
+    x = wl.storage_numpy(wl.gen_x(M, K, 31))
+    y1 = oracle.matmul(x, oracle.BF16, p, s, b, oracle.BF16, N, gs, bits)
+    y2 = oracle.matmul_dense(x, oracle.BF16, p, s, b, oracle.BF16, N, gs, bits)
+    wd = oracle.dequantize(p, s, b, oracle.BF16, K, gs, bits, oracle.F32).astype(np.float64)
+    bound = K * 2.0 ** -52 * (np.abs(oracle.widen_f64(x, oracle.BF16)) @ np.abs(wd).T)
+    assert np.all(np.abs(y1 - y2) <= bound)
+    # a dropped term would show: zeroing one weight column changes y2 beyond the bound
+    p2 = p.copy()
+    p2[:, 0] = 0
+    y3 = oracle.matmul_dense(x, oracle.BF16, p2, s, b, oracle.BF16, N, gs, bits)
+    assert np.any(np.abs(y3 - y1) > bound)

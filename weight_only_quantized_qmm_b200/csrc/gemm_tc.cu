@@ -32,11 +32,11 @@ constexpr int kBM = 128;                 // weight rows per CTA (UMMA M)
 constexpr int kBN = 256;                 // tokens per CTA (UMMA N)
 constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row of 16-bit values
 constexpr int kStages = 4;
-constexpr int kThreads = 192;            // 6 warps
+constexpr int kThreads = 320;            // 10 warps
 constexpr int kXStage = kBN * kBK * 2;   // 32 KB
 constexpr int kAStage = kBM * kBK * 2;   // 16 KB
 constexpr int kTileBytes = kStages * (kXStage + kAStage);
-constexpr int kSmem = 1024 + kTileBytes + 256;  // + alignment slack + barriers
+constexpr int kSmem = 1024 + kTileBytes + 256;  // + alignment slack + barriers (17 used)
 constexpr uint32_t kSpins = 1u << 22;
 }  // namespace gemm
 
@@ -178,6 +178,27 @@ __device__ __forceinline__ void codes_to_pairs(const uint32_t (&w)[2 * B], uint3
   }
 }
 
+// The CTA's tiles, in order: tile = blockIdx.x + lt * gridDim.x.  Weight-row
+// tiles vary slowest, so the CTAs running at the same time share their x
+// tiles and weight rows through L2.
+struct TileOf {
+  int n0, m0;
+};
+__device__ __forceinline__ TileOf tile_of(int lt, int m_tiles) {
+  const int t = blockIdx.x + lt * gridDim.x;
+  return TileOf{(t / m_tiles) * gemm::kBM, (t % m_tiles) * gemm::kBN};
+}
+
+// Persistent: every CTA walks its tiles (static round robin over the grid).
+// Warp roles:
+//   warp 0      TMA producer of the x tiles (one stage = 256 tokens x 64 k)
+//   warp 1      TMEM owner (512 columns: two 128 x 256 fp32 accumulators)
+//               and MMA issuer; the accumulator alternates per tile, so the
+//               epilogue of one tile runs under the main loop of the next
+//   warps 2..5  dequantize the weight tile of each stage into the A buffer
+//   warps 6..9  epilogue: tcgen05.ld of the finished accumulator, release it,
+//               store y directly from registers (per instruction, a warp
+//               writes 32 consecutive weight rows of one token)
 template <int B, int GS, typename T>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
 qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
@@ -188,13 +209,18 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   uint8_t* as = smem + kStages * kXStage;             // [kStages][128 x 128 B]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTileBytes);
   const uint32_t full0 = su32(bars), afull0 = full0 + 8 * kStages, empty0 = afull0 + 8 * kStages;
-  const uint32_t accf = empty0 + 8 * kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 1);
+  const uint32_t accf0 = empty0 + 8 * kStages;      // [2] accumulator complete
+  const uint32_t tfree0 = accf0 + 16;               // [2] accumulator read out by the epilogue
+  const uint32_t drain = tfree0 + 16;               // every issued MMA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 5);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBM, m0 = blockIdx.y * kBN;
   const int nk = (p.K + kBK - 1) / kBK;
+  const int m_tiles = (p.M + kBN - 1) / kBN;
+  const int n_tiles = (p.N + kBM - 1) / kBM;
+  const int T_all = m_tiles * n_tiles;
+  const int my_tiles = blockIdx.x < T_all ? (T_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -202,29 +228,43 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
       mbar_init(afull0 + 8 * s, 4);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(accf, 1);
+    mbar_init(accf0, 1);
+    mbar_init(accf0 + 8, 1);
+    mbar_init(tfree0, 4);
+    mbar_init(tfree0 + 8, 4);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {  // 256 TMEM columns for the 128 x 256 fp32 accumulator
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(su32(tmem_slot)));
+  if (warp == 1) {  // 512 TMEM columns: accumulators at columns 0 and 256
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(su32(tmem_slot)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // x and the weights may come from the previous kernel in the stream
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % kStages, u = i / kStages;
-        if (i >= kStages && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
-        tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, m0, full0 + 8 * s);
-        issued = i + 1;
+      int j = 0, issued = 0;
+      bool stop = false;
+      for (int lt = 0; lt < my_tiles && !stop; ++lt) {
+        const TileOf tl = tile_of(lt, m_tiles);
+        for (int i = 0; i < nk; ++i, ++j) {
+          const int s = j % kStages, u = j / kStages;
+          if (j >= kStages && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
+          tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, tl.m0, full0 + 8 * s);
+          issued = j + 1;
+        }
       }
       // no copy may still be landing when the CTA exits: the last copy of every
       // slot is waited for with the full bound, also after an abort
@@ -235,151 +275,164 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = mma_idesc<T>();
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % kStages, u = i / kStages;
-        if (!bar_wait(full0 + 8 * s, u & 1, abort_flag) || !bar_wait(afull0 + 8 * s, u & 1, abort_flag)) {
+      int j = 0;
+      bool stop = false;
+      for (int lt = 0; lt < my_tiles && !stop; ++lt) {
+        const int b = lt & 1;
+        // accumulator b is free once the epilogue has read out tile lt - 2
+        if (lt >= 2 && !bar_wait(tfree0 + 8 * b, ((lt >> 1) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = su32(as + s * kAStage), b0 = su32(xs + s * kXStage);
+        const uint32_t acc = tmem + (uint32_t)(b * kBN);
+        for (int i = 0; i < nk; ++i, ++j) {
+          const int s = j % kStages, u = j / kStages;
+          if (!bar_wait(full0 + 8 * s, u & 1, abort_flag) || !bar_wait(afull0 + 8 * s, u & 1, abort_flag)) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = su32(as + s * kAStage), b0 = su32(xs + s * kXStage);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_f16(tmem, sw128_desc(a0 + 32 * kk), sw128_desc(b0 + 32 * kk), idesc,
-                  (i | kk) != 0 ? 1u : 0u);
-        mma_commit(empty0 + 8 * s);  // frees the stage once these MMAs have read it
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            mma_f16(acc, sw128_desc(a0 + 32 * kk), sw128_desc(b0 + 32 * kk), idesc, (i | kk) != 0 ? 1u : 0u);
+          mma_commit(empty0 + 8 * s);  // frees the stage once these MMAs have read it
+        }
+        mma_commit(accf0 + 8 * b);  // accumulator b complete (also after an abort)
       }
-      mma_commit(accf);  // accumulator complete
+      // TMEM is released only once every issued MMA has completed
+      mma_commit(drain);
+      mbar_wait_n(drain, 0, gemm::kSpins);
     }
-  } else {
-    // ---------------- dequant (warps 2..5), then epilogue ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r = q * 32 + lane;  // weight row of the tile owned by this thread
-    const int n = n0 + r;
-    const bool nval = n < p.N;
-    const uint32_t* row = p.packed + (int64_t)(nval ? n : 0) * p.wpr;
-    const T* srow = reinterpret_cast<const T*>(p.scales) + (int64_t)(nval ? n : 0) * p.G;
-    const T* brow = reinterpret_cast<const T*>(p.biases) + (int64_t)(nval ? n : 0) * p.G;
+  } else if (warp < 6) {
+    // ---------------- dequant (warps 2..5) ----------------
+    const int r = (warp & 3) * 32 + lane;  // weight row of the tile owned by this thread
     constexpr int NGS = (kBK + GS - 1) / GS;  // groups touched by a stage (1 or 2)
     constexpr uint32_t OFF2 = std::is_same<T, __half>::value ? 0x64006400u : 0x43004300u;
     constexpr bool kF32Path = (B == 8) && !std::is_same<T, __half>::value;
+    const int total = my_tiles * nk;
 
     // codes and scales/biases are prefetched kAhead stages ahead into a register
-    // ring (compile-time indices: the stage loop is unrolled by kAhead)
+    // ring (compile-time indices: the stage loop is unrolled by kAhead); stage j
+    // is k-stage j % nk of the CTA's tile j / nk
     constexpr int kAhead = 3;
     uint32_t rw[kAhead][2 * B];
     T rs[kAhead][NGS], rb[kAhead][NGS];
-    auto load = [&](int i, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
+    auto load = [&](int j, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
+      const bool in = j < total;
+      const int lt = in ? j / nk : 0, i = in ? j - lt * nk : 0;
+      const int n = tile_of(lt, m_tiles).n0 + r;
+      const bool nval = in && n < p.N;
+      const uint32_t* row = p.packed + (int64_t)(nval ? n : 0) * p.wpr;
+      const T* srow = reinterpret_cast<const T*>(p.scales) + (int64_t)(nval ? n : 0) * p.G;
+      const T* brow = reinterpret_cast<const T*>(p.biases) + (int64_t)(nval ? n : 0) * p.G;
       const int k0 = i * kBK;
-      load_codes<B>(row, k0 * B / 32, p.wpr, nval && i < nk, w);
+      load_codes<B>(row, k0 * B / 32, p.wpr, nval, w);
 #pragma unroll
-      for (int j = 0; j < NGS; ++j) {
-        const int gidx = (k0 + j * GS) / GS;
-        const bool ok = nval && i < nk && gidx < p.G;
-        sv[j] = ok ? srow[gidx] : from_f32<T>(0.0f);
-        bv[j] = ok ? brow[gidx] : from_f32<T>(0.0f);
+      for (int jj = 0; jj < NGS; ++jj) {
+        const int gidx = (k0 + jj * GS) / GS;
+        const bool ok = nval && gidx < p.G;
+        sv[jj] = ok ? srow[gidx] : from_f32<T>(0.0f);
+        bv[jj] = ok ? brow[gidx] : from_f32<T>(0.0f);
       }
     };
 #pragma unroll
     for (int a = 0; a < kAhead; ++a) load(a, rw[a], rs[a], rb[a]);
-    for (int i0 = 0; i0 < nk; i0 += kAhead) {
+    for (int j0 = 0; j0 < total; j0 += kAhead) {
 #pragma unroll
-    for (int a = 0; a < kAhead; ++a) {
-      const int i = i0 + a;
-      if (i >= nk) break;
-      const int s = i % kStages, u = i / kStages;
-      uint32_t cw[2 * B];
-      T cs[NGS], cb[NGS];
+      for (int a = 0; a < kAhead; ++a) {
+        const int j = j0 + a;
+        if (j >= total) break;
+        const int s = j % kStages, u = j / kStages;
+        uint32_t cw[2 * B];
+        T cs[NGS], cb[NGS];
 #pragma unroll
-      for (int j = 0; j < 2 * B; ++j) cw[j] = rw[a][j];
+        for (int q = 0; q < 2 * B; ++q) cw[q] = rw[a][q];
 #pragma unroll
-      for (int j = 0; j < NGS; ++j) { cs[j] = rs[a][j]; cb[j] = rb[a][j]; }
-      load(i + kAhead, rw[a], rs[a], rb[a]);  // refill this ring slot kAhead stages ahead
-      // the A buffer of this stage is free once the MMAs of stage i - kStages are done
-      if (u > 0 && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) *abort_flag = 1;
-      uint32_t pr[32];
-      float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
-      if constexpr (kF32Path) {
-        sf0 = to_f32(cs[0]); bf0 = to_f32(cb[0]);
-        sf1 = to_f32(cs[NGS - 1]); bf1 = to_f32(cb[NGS - 1]);
-      } else {
-        codes_to_pairs<B, T>(cw, pr);
+        for (int q = 0; q < NGS; ++q) { cs[q] = rs[a][q]; cb[q] = rb[a][q]; }
+        load(j + kAhead, rw[a], rs[a], rb[a]);  // refill this ring slot kAhead stages ahead
+        // the A buffer of this stage is free once the MMAs of stage j - kStages are done
+        if (u > 0 && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) *abort_flag = 1;
+        uint32_t pr[32];
+        float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
+        if constexpr (kF32Path) {
+          sf0 = to_f32(cs[0]); bf0 = to_f32(cb[0]);
+          sf1 = to_f32(cs[NGS - 1]); bf1 = to_f32(cb[NGS - 1]);
+        } else {
+          codes_to_pairs<B, T>(cw, pr);
+        }
+        const uint32_t s2a = (uint32_t)bits16(cs[0]) * 0x00010001u;
+        const uint32_t b2a = (uint32_t)bits16(cb[0]) * 0x00010001u;
+        const uint32_t s2b = (uint32_t)bits16(cs[NGS - 1]) * 0x00010001u;
+        const uint32_t b2b = (uint32_t)bits16(cb[NGS - 1]) * 0x00010001u;
+        uint8_t* arow = as + s * kAStage + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = pairs 4c..4c+3 = codes 8c..8c+7
+          uint4 v;
+          uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int pi = 4 * c + e;
+            const bool second = NGS > 1 && (2 * pi) >= GS;
+            if constexpr (kF32Path) {
+              // 8-bit codes do not fit the bf16 magic: q exact in fp32, fmaf, one bf16 rounding
+              const float q0 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi)) - 8388608.0f;
+              const float q1 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi + 1)) - 8388608.0f;
+              const float sv = second ? sf1 : sf0, bv = second ? bf1 : bf0;
+              const __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(q0, sv, bv), fmaf(q1, sv, bv));
+              vv[e] = *reinterpret_cast<const uint32_t*>(&h);
+            } else {
+              const uint32_t qv = h2_sub<T>(pr[pi], OFF2);  // exact q
+              vv[e] = h2_fma<T>(qv, second ? s2b : s2a, second ? b2b : b2a);
+            }
+          }
+          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+        __syncwarp();
+        if (lane == 0) mbar_arrive(afull0 + 8 * s);
       }
-      const uint32_t s2a = (uint32_t)bits16(cs[0]) * 0x00010001u;
-      const uint32_t b2a = (uint32_t)bits16(cb[0]) * 0x00010001u;
-      const uint32_t s2b = (uint32_t)bits16(cs[NGS - 1]) * 0x00010001u;
-      const uint32_t b2b = (uint32_t)bits16(cb[NGS - 1]) * 0x00010001u;
-      uint8_t* arow = as + s * kAStage + r * 128;
+    }
+  } else {
+    // ---------------- epilogue (warps 6..9): TMEM -> registers -> y ----------------
+    const int qq = warp & 3;          // TMEM lane quarter this warp may access
+    const int r = qq * 32 + lane;     // weight row of the tile
+    const bool f32out = p.y_dtype == QMM_F32;
+    bool failed = false;
+    for (int lt = 0; lt < my_tiles; ++lt) {
+      const TileOf tl = tile_of(lt, m_tiles);
+      const int b = lt & 1;
+      const int n = tl.n0 + r;
+      if (!failed) {
+        // the MMA warp commits accf on every path it takes; a raised abort flag
+        // ends the wait early, and the tile (and all later ones) is written as NaN
+        failed = !bar_wait(accf0 + 8 * b, (lt >> 1) & 1, abort_flag) ||
+                 *reinterpret_cast<volatile int*>(abort_flag);
+        failed = __any_sync(0xffffffffu, failed);
+      }
+      tc_fence_after();
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t v[32];
+        if (!failed) tmem_ld32(tmem + ((uint32_t)(qq * 32) << 16) + (uint32_t)(b * kBN + c * 32), v);
+        if (n < p.N) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = pairs 4c..4c+3 = codes 8c..8c+7
-        uint4 v;
-        uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int pi = 4 * c + e;
-          const bool second = NGS > 1 && (2 * pi) >= GS;
-          if constexpr (kF32Path) {
-            // 8-bit codes do not fit the bf16 magic: q exact in fp32, fmaf, one bf16 rounding
-            const float q0 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi)) - 8388608.0f;
-            const float q1 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi + 1)) - 8388608.0f;
-            const float sv = second ? sf1 : sf0, bv = second ? bf1 : bf0;
-            const __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(q0, sv, bv), fmaf(q1, sv, bv));
-            vv[e] = *reinterpret_cast<const uint32_t*>(&h);
-          } else {
-            const uint32_t qv = h2_sub<T>(pr[pi], OFF2);  // exact q
-            vv[e] = h2_fma<T>(qv, second ? s2b : s2a, second ? b2b : b2a);
+          for (int jj = 0; jj < 32; ++jj) {
+            const int m = tl.m0 + c * 32 + jj;
+            if (m < p.M) {
+              const float f = failed ? __int_as_float(0x7fc00000) : __uint_as_float(v[jj]);
+              if (f32out)
+                reinterpret_cast<float*>(p.y)[(int64_t)m * p.N + n] = f;
+              else
+                reinterpret_cast<T*>(p.y)[(int64_t)m * p.N + n] = from_f32<T>(f);
+            }
           }
         }
-        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = v;
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(afull0 + 8 * s);
-    }
-    }
-
-    // ---------------- epilogue: TMEM -> registers -> smem transpose -> y ----------------
-    // the MMA warp commits accf on every path (also after an abort), so this
-    // wait ignores the abort flag: TMEM is read and released only once every
-    // issued MMA has completed
-    const bool ok = mbar_wait_n(accf, 0, gemm::kSpins) && !*reinterpret_cast<volatile int*>(abort_flag);
-    tc_fence_after();
-    const bool f32out = p.y_dtype == QMM_F32;
-    // staging tile [256 tokens][128 rows] in the (now idle) pipeline buffers
-    uint8_t* stg = smem;
-    const int esz = f32out ? 4 : 2;
-    for (int c = 0; c < kBN / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c * 32), v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int tok = c * 32 + j;
-        const float f = ok ? __uint_as_float(v[j]) : __int_as_float(0x7fc00000);
-        if (f32out)
-          *reinterpret_cast<float*>(stg + ((size_t)tok * kBM + r) * 4) = f;
-        else
-          *reinterpret_cast<T*>(stg + ((size_t)tok * kBM + r) * 2) = from_f32<T>(f);
-      }
-    }
-    tc_fence_before();
-    asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps
-    // coalesced stores: 16 bytes per thread per step along each token row
-    const int row_bytes = kBM * esz;
-    const int chunks = kBN * row_bytes / 16;
-    const int et = threadIdx.x - 64;
-    for (int ci = et; ci < chunks; ci += 128) {
-      const int tok = ci / (row_bytes / 16);
-      const int col = (ci % (row_bytes / 16)) * (16 / esz);  // first weight row of the chunk
-      const int m = m0 + tok, nn = n0 + col;
-      if (m >= p.M || nn >= p.N) continue;
-      const uint8_t* src = stg + (size_t)tok * row_bytes + (size_t)col * esz;
-      uint8_t* dst = reinterpret_cast<uint8_t*>(p.y) + ((int64_t)m * p.N + nn) * esz;
-      const int nvalid = min(16 / esz, p.N - nn);
-      if (nvalid == 16 / esz && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-      } else {
-        for (int e = 0; e < nvalid * esz; ++e) dst[e] = src[e];
-      }
+      if (lane == 0 && !failed) mbar_arrive(tfree0 + 8 * b);
     }
   }
 
@@ -387,7 +440,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
   }
 }
 
@@ -410,9 +463,19 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, 
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  dim3 grid((prm.N + gemm::kBM - 1) / gemm::kBM, (prm.M + gemm::kBN - 1) / gemm::kBN);
-  k<<<grid, gemm::kThreads, gemm::kSmem, st>>>(prm, tmx);
-  return cudaGetLastError();
+  // persistent: one CTA per SM (or per tile when there are fewer tiles)
+  const int tiles = ((prm.N + gemm::kBM - 1) / gemm::kBM) * ((prm.M + gemm::kBN - 1) / gemm::kBN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(tiles, qmm_host::num_sms()));
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = gemm::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, prm, tmx);
 }
 
 template <typename T>

@@ -18,15 +18,22 @@
 // values, swizzled at their row width).  Warp roles:
 //   * producer (1 warp, one lane) issues the copies, slot by slot;
 //   * consumers (KC warps) all read every unit, consumer w taking groups
-//     [w * GPW, (w + 1) * GPW).  Per group a consumer turns codes into 16-bit
-//     floats (OFF + q, exact), takes the partial dot with x on the tensor
-//     cores (mma.m16n8k16; rows of W as m, the segment's pairs as n), and
-//     folds it into fp32 accumulators as
-//       y += s * d + (b - OFF * s) * X,   X = sum of x over the group,
+//     [w * GPW, (w + 1) * GPW).  Per group a consumer turns codes into f16
+//     pairs with one lop3 (or prmt) each -- a code q sitting at bit p of a
+//     16-bit half becomes 1024 + q * 2^p exactly -- takes the partial dot with
+//     x on the tensor cores (mma.m16n8k16 f16; rows of W as m, the segment's
+//     pairs as n) and folds it into fp32 accumulators.  x is staged per
+//     (group, pair) in f16 as x * 2^(e - p), with 2^e a power of two that puts
+//     the group's largest |x| in [2^14, 2^15) (exact for 16-bit activations
+//     but for values below 2^-24 of the group maximum) and 2^-p undoing the
+//     code's bit offset, so the mma yields
+//       D = 2^e * (sum_k q_k x_k) + 1024 * sum_k x''_k   (x'' the staged values)
+//     and per row
+//       y += s * (2^-e * D - 1024 * 2^-e * sum x'') + b * sum_k x_k,
 //     which is sum_k x_k (q_k s + b) rewritten per group.  The slot is free
 //     again once all KC consumers arrived on its `empty` mbarrier.  At a new
 //     segment the consumers stage its x rows (tensor-core k order, with the
-//     per-group sums);
+//     per-group records {2^-e, -1024 * 2^-e * sum x'', sum x});
 //   * epilogue (1 warp): when every consumer posted its partial for a tile
 //     (mbarrier `pfull`), sums them in consumer order (the result does not
 //     depend on timing), applies SiLU(gate) * up for the fused form and
@@ -35,10 +42,11 @@
 // arithmetic and still drains the copies in flight before the CTA exits.
 //
 // Launched with programmatic stream serialization: the CTA's set-up (barrier
-// initialisation, shared-memory carve-up) overlaps the previous kernel's
-// tail; every global read (weights, ids, x) comes after griddepcontrol.wait,
-// so whatever the previous kernel in the stream wrote -- weights included --
-// is visible.
+// initialisation, shared-memory carve-up and, for dense calls, L2 prefetches
+// of its first weight units) overlaps the previous kernel's tail; every read
+// into shared memory or registers (weights, ids, x) comes after
+// griddepcontrol.wait, so whatever the previous kernel in the stream wrote --
+// weights included -- is visible.
 #pragma once
 
 #include <cuda.h>
@@ -58,8 +66,38 @@ struct Params {
   int CH;               // pairs per segment
   int tok_stride;       // bytes between staged rows of x
   int stages;           // ring depth
-  uint32_t magic;       // two 16-bit floats whose low bits take a code (128 + q / 1024 + q)
   int off_code, off_sb, off_bar, off_part, off_xs, off_xsum, off_plan;
+};
+
+// Layout of one thread's quarter of a group for the f16 lane arithmetic:
+// kCodes consecutive codes in kRegs packed words; each word yields kOPW f16
+// pairs, pair j holding codes j and j + kOPW of the word, both at bit offset
+// pos(j) inside their 16-bit half (a code at bit p reads as 1024 + q * 2^p).
+//   8-bit: pairs (0,2) (1,3), offset 0 (byte permutes, no mask);
+//   4-bit: pairs (0,4) (1,5) (2,6) (3,7), offsets 0, 4, 0, 4 (the last two
+//          from the word shifted right by 8);
+//   2-bit: pairs (j, j+8), offsets 0, 2, 4, 6, 8 for j < 5 and 0, 2, 4 for
+//          j = 5..7 (from the word shifted right by 10).
+template <int BITS, int GS>
+struct Lanes {
+  static constexpr int kLPW = 32 / BITS;            // codes per packed word
+  static constexpr int kOPW = kLPW / 2;             // f16 pairs per word
+  static constexpr int kCodes = GS / 4;             // codes of a thread's quarter
+  static constexpr int kRegs = kCodes * BITS / 32;  // packed words of a quarter
+  static constexpr int kOuts = kCodes / 2;          // f16 pairs of a quarter
+  static constexpr int kSteps = kCodes / 4;         // m16n8k16 steps per group
+  static constexpr int kWordsPerGroup = GS * BITS / 32;
+  static constexpr bool kOk = (BITS == 2 || BITS == 4 || BITS == 8) && (kCodes * BITS) % 32 == 0;
+  static constexpr uint32_t kMagic = 0x64006400u;   // f16 1024.0 in both halves
+  static constexpr float kOff = 1024.0f;
+  __host__ __device__ static constexpr int pos(int j) {
+    return BITS == 8 ? 0 : BITS == 4 ? (j & 1) * 4 : (j < 5 ? 2 * j : 2 * (j - 5));
+  }
+  // pair o of the quarter -> code index (within the quarter) of its low and
+  // high half
+  __host__ __device__ static constexpr int lo_code(int o) { return (o / kOPW) * kLPW + o % kOPW; }
+  __host__ __device__ static constexpr int hi_code(int o) { return lo_code(o) + kOPW; }
+  __host__ __device__ static constexpr int lo_pos(int o) { return pos(o % kOPW); }
 };
 
 // MODE 0: one pair per segment; 1: up to 8; 2: up to 16.  UG: groups per unit
@@ -67,13 +105,13 @@ struct Params {
 // matrices per pair (2: gate and up).
 template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
 struct Cfg {
-  using S = Share<BITS, GS, T>;
+  using L = Lanes<BITS, GS>;
   static constexpr int MT = MODE == 2 ? 2 : 1;
   static constexpr bool ONE = MODE == 0;
   static constexpr int KC = MT == 1 ? 16 : 8;                     // consumer warps
   static constexpr int THREADS = (KC + 2) * 32;
   static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
-  static constexpr int WPG = S::kWordsPerGroup;                   // words per group per row
+  static constexpr int WPG = L::kWordsPerGroup;                   // words per group per row
   static constexpr int GPU = UG;                                  // groups per unit
   static constexpr int GPW = GPU / KC;                            // groups per consumer per unit
   static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
@@ -82,9 +120,8 @@ struct Cfg {
   static constexpr uint32_t TX = NS * (CODE_BYTES + 2 * SB_BYTES);
   static constexpr int TOKP = 8 * MT;
   static constexpr int CH = ONE ? 1 : TOKP;                       // pairs per segment
-  static constexpr int XG = 4 * S::kVirt * (int)sizeof(T);        // staged x bytes per group
-  static constexpr int NX = S::kSplit ? 2 : 1;                    // per-group sums kept
-  static_assert(S::kFast, "integral-lane codes only");
+  static constexpr int XG = 4 * L::kCodes * 2;                    // staged f16 x bytes per group
+  static_assert(L::kOk, "integral-lane codes only");
   static_assert(GPW >= 1 && GPW * KC == GPU, "whole groups per consumer");
   static_assert(Z >= 1 && Z <= 16, "unit of at most 16 slices (32 KB)");
   static_assert(GPU * 2 == 32 || GPU * 2 == 64 || GPU * 2 == 128, "scale rows of one swizzle span");
@@ -107,74 +144,81 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// d = sum over the k16 steps of (OFF + v) * x' for 16 rows x 8 columns; the
-// first step starts from a zero accumulator.
-template <typename T>
-__device__ __forceinline__ void mma_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                          uint32_t b0, uint32_t b1) {
-  const float z = 0.0f;
-  if constexpr (std::is_same<T, __half>::value) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
-  } else {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%10,%10,%10};"
-        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
-  }
+// L2 prefetches of one box of a tensor map (no shared memory, no barrier)
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int x, int y, int z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y),
+               "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
 }
 
-// Codes j and j + LPW/2 of a word of LW-bit lanes as a pair of 16-bit floats
-// (MAGIC + code, exact): one shift and one lop3 ((a & b) | c).
-template <int LW, int SH>
-__device__ __forceinline__ uint32_t lane_pair(uint32_t w, uint32_t magic) {
-  constexpr uint32_t MASK = ((1u << LW) - 1u) * 0x00010001u;
+// d = A . B for one m16n8k16 f16 step, starting from a zero accumulator.
+__device__ __forceinline__ void mma_f16_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  const float z = 0.0f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(z));
+}
+
+// (w & MASK) | 1024.0 in both f16 halves: one lop3
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t mask_magic(uint32_t w) {
   uint32_t d;
-  if constexpr (SH == 0) {
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(magic));
-  } else {
-    asm("{\n\t.reg .b32 t;\n\tshr.u32 t, %1, %4;\n\tlop3.b32 %0, t, %2, %3, 0xEA;\n\t}"
-        : "=r"(d)
-        : "r"(w), "n"(MASK), "r"(magic), "n"(SH));
-  }
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "n"(0x64006400u));
   return d;
 }
-// All LPW/2 pairs of one word, pair j = codes (j, j + LPW/2).
-template <class S>
-__device__ __forceinline__ void word_pairs(uint32_t w, uint32_t magic, uint32_t* out) {
-  constexpr int LW = S::kLW;
-  constexpr int NP = S::kLPW / 2;
-  out[0] = lane_pair<LW, 0>(w, magic);
-  out[1] = lane_pair<LW, LW>(w, magic);
-  if constexpr (NP >= 4) {
-    out[2] = lane_pair<LW, 2 * LW>(w, magic);
-    out[3] = lane_pair<LW, 3 * LW>(w, magic);
-  }
-  if constexpr (NP >= 8) {
-    out[4] = lane_pair<LW, 4 * LW>(w, magic);
-    out[5] = lane_pair<LW, 5 * LW>(w, magic);
-    out[6] = lane_pair<LW, 6 * LW>(w, magic);
-    out[7] = lane_pair<LW, 7 * LW>(w, magic);
+// bytes (a.SEL0, 0x64, a.SEL2, 0x64): two 8-bit codes as 1024 + q in f16
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t byte_magic(uint32_t w) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(w), "r"(0x64646464u), "n"(SEL));
+  return d;
+}
+
+// The kOPW f16 pairs of one packed word (pair j = codes j, j + kOPW; see Lanes).
+template <int BITS>
+__device__ __forceinline__ void word_pairs16(uint32_t w, uint32_t* o) {
+  if constexpr (BITS == 8) {
+    o[0] = byte_magic<0x4240u>(w);
+    o[1] = byte_magic<0x4341u>(w);
+  } else if constexpr (BITS == 4) {
+    o[0] = mask_magic<0x000F000Fu>(w);
+    o[1] = mask_magic<0x00F000F0u>(w);
+    const uint32_t t = w >> 8;
+    o[2] = mask_magic<0x000F000Fu>(t);
+    o[3] = mask_magic<0x00F000F0u>(t);
+  } else {
+    o[0] = mask_magic<0x00030003u>(w);
+    o[1] = mask_magic<0x000C000Cu>(w);
+    o[2] = mask_magic<0x00300030u>(w);
+    o[3] = mask_magic<0x00C000C0u>(w);
+    o[4] = mask_magic<0x03000300u>(w);
+    const uint32_t t = w >> 10;
+    o[5] = mask_magic<0x00030003u>(t);
+    o[6] = mask_magic<0x000C000Cu>(t);
+    o[7] = mask_magic<0x00300030u>(t);
   }
 }
 
-template <int BITS, class S, typename T, int MT>
-__device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], const uint32_t (&rawB)[S::kRegs],
-                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4],
-                                           uint32_t magic) {
-  constexpr int NP = S::kLPW / 2;  // pairs per word
-  uint32_t pA[S::kRegs * NP], pB[S::kRegs * NP];
+// Tensor-core partial dot of one group for 16 rows x 8 (per token tile)
+// columns: d = sum over the group's k16 steps of (1024 + q 2^p) * x''.
+template <class L, int MT>
+__device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[L::kRegs], const uint32_t (&rawB)[L::kRegs],
+                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4]) {
+  uint32_t pA[L::kOuts], pB[L::kOuts];
 #pragma unroll
-  for (int k = 0; k < S::kRegs; ++k) {
-    word_pairs<S>(rawA[k], magic, pA + k * NP);
-    word_pairs<S>(rawB[k], magic, pB + k * NP);
+  for (int k = 0; k < L::kRegs; ++k) {
+    word_pairs16<32 / L::kLPW>(rawA[k], pA + k * L::kOPW);
+    word_pairs16<32 / L::kLPW>(rawB[k], pB + k * L::kOPW);
   }
 #pragma unroll
-  for (int q2 = 0; q2 < S::kSteps / 2; ++q2) {
+  for (int q2 = 0; q2 < L::kSteps / 2; ++q2) {
     uint4 bf[MT];
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) bf[mt] = lds128(xb[mt] + xo + q2 * 16);
@@ -185,38 +229,37 @@ __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[S::kRegs], con
       for (int mt = 0; mt < MT; ++mt) {
         const uint32_t b0 = h2 ? bf[mt].z : bf[mt].x, b1 = h2 ? bf[mt].w : bf[mt].y;
         if (q == 0)
-          mma_first<T>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+          mma_f16_first(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
         else
-          mma16816<T>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+          mma16816<__half>(d[mt], pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
       }
     }
   }
 }
 
 // As group_dot1 for one token column, with the x fragments in registers.
-template <int BITS, class S, typename T>
-__device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[S::kRegs], const uint32_t (&rawB)[S::kRegs],
-                                             const uint4 (&bf)[S::kSteps / 2], float (&d)[4], uint32_t magic) {
-  constexpr int NP = S::kLPW / 2;
-  uint32_t pA[S::kRegs * NP], pB[S::kRegs * NP];
+template <class L>
+__device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[L::kRegs], const uint32_t (&rawB)[L::kRegs],
+                                             const uint4 (&bf)[L::kSteps / 2], float (&d)[4]) {
+  uint32_t pA[L::kOuts], pB[L::kOuts];
 #pragma unroll
-  for (int k = 0; k < S::kRegs; ++k) {
-    word_pairs<S>(rawA[k], magic, pA + k * NP);
-    word_pairs<S>(rawB[k], magic, pB + k * NP);
+  for (int k = 0; k < L::kRegs; ++k) {
+    word_pairs16<32 / L::kLPW>(rawA[k], pA + k * L::kOPW);
+    word_pairs16<32 / L::kLPW>(rawB[k], pB + k * L::kOPW);
   }
   // even and odd k16 steps in two chains (half the dependent mma latency);
-  // only columns 0 (rows g, g + 8: d[0], d[2]) are merged, the others are idle
+  // only column 0 (rows g, g + 8: d[0], d[2]) is merged, the others are idle
   float e[4];
 #pragma unroll
-  for (int q = 0; q < S::kSteps; ++q) {
+  for (int q = 0; q < L::kSteps; ++q) {
     const uint32_t b0 = (q & 1) ? bf[q >> 1].z : bf[q >> 1].x, b1 = (q & 1) ? bf[q >> 1].w : bf[q >> 1].y;
     float(&acc)[4] = (q & 1) ? e : d;
     if (q < 2)
-      mma_first<T>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+      mma_f16_first(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
     else
-      mma16816<T>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+      mma16816<__half>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
   }
-  if constexpr (S::kSteps > 1) {
+  if constexpr (L::kSteps > 1) {
     d[0] += e[0];
     d[2] += e[2];
   }
@@ -263,64 +306,81 @@ struct Walk {
   }
 };
 
+// 2^e as a float for e in [-126, 127]
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
 // Stage the x rows of a segment's pairs [0, np) for groups [0, Gpad): per
-// (pair, group, quarter t) the kVirt values of quarter t in slot order (the
-// codes' mma k order), zero past G; per (group, pair) the fp32 sum of x over
-// the group (and, for the two-nibble 8-bit form, the sum of the slot values
-// x').  Pairs [np, TOKP) of the sums read as zero.
-template <class S, typename T, int TOKP, int NX, int NTHR>
+// (pair, group, quarter t) the quarter's kCodes values as f16 pairs in the
+// order of the code pairs (Lanes), each x_k * 2^(e - p_k), with 2^e chosen per
+// (pair, group) so that the group's largest |x| lands in [2^14, 2^15); per
+// (group, pair) the record {2^-e, -1024 * 2^-e * sum of the staged values (as
+// rounded), sum of x, 0}.  Groups past G stage zeros; records of pairs
+// [np, TOKP) read as zero.
+template <class L, typename T, int TOKP, int NTHR>
 __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, int np, int Gpad,
-                                        int tok_stride, int sid, uint8_t* xs, float* xsum) {
-  constexpr int GS = S::kCodes * 4;
+                                        int tok_stride, int sid, uint8_t* xs, float4* rec) {
+  constexpr int GS = L::kCodes * 4;
   const int ntask = np * Gpad * 4;
   for (int base = 0; base < ntask; base += NTHR) {
     const int idx = base + sid;
     const bool act = idx < ntask;
     const int tt = idx & 3, gq = idx >> 2;
     const int m = act ? gq / Gpad : 0, gl = act ? gq - m * Gpad : 0;
-    float sb = 0.0f, so = 0.0f;
-    if (act) {
-      __align__(16) T xv[S::kCodes];
-      if (gl < q.G) {
-        const T* xa = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS + tt * S::kCodes;
-        if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
+    __align__(16) T xv[L::kCodes];
+    if (act && gl < q.G) {
+      const T* xa = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS + tt * L::kCodes;
+      if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
 #pragma unroll
-          for (int c = 0; c < S::kCodes * (int)sizeof(T) / 16; ++c)
-            reinterpret_cast<uint4*>(xv)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
-        } else {
-#pragma unroll
-          for (int c = 0; c < S::kCodes; ++c) xv[c] = xa[c];
-        }
+        for (int c = 0; c < L::kCodes * (int)sizeof(T) / 16; ++c)
+          reinterpret_cast<uint4*>(xv)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
       } else {
 #pragma unroll
-        for (int c = 0; c < S::kCodes * (int)sizeof(T) / 16; ++c)
-          reinterpret_cast<uint4*>(xv)[c] = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < L::kCodes; ++c) xv[c] = xa[c];
       }
-      __align__(16) T outv[S::kVirt];
+    } else {
 #pragma unroll
-      for (int qv = 0; qv < S::kVirt; ++qv) {
-        const int vv = S::slot_virtual(qv);
-        const float mult = S::virt_mult(vv);
-        const float xf = to_f32(xv[S::virt_code(vv)]) * mult;
-        outv[qv] = from_f32<T>(xf);
-        so += xf;
-        if (mult == 1.0f) sb += xf;
-      }
-      uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)m * tok_stride + (size_t)(gl * 4 + tt) * S::kVirt * sizeof(T));
-#pragma unroll
-      for (int qv = 0; qv < (int)(S::kVirt * sizeof(T) / 16); ++qv) dst[qv] = reinterpret_cast<const uint4*>(outv)[qv];
+      for (int c = 0; c < L::kCodes * (int)sizeof(T) / 16; ++c)
+        reinterpret_cast<uint4*>(xv)[c] = make_uint4(0u, 0u, 0u, 0u);
     }
-    sb += __shfl_xor_sync(0xffffffffu, sb, 1);
-    so += __shfl_xor_sync(0xffffffffu, so, 1);
-    sb += __shfl_xor_sync(0xffffffffu, sb, 2);
-    so += __shfl_xor_sync(0xffffffffu, so, 2);
+    // the group's largest magnitude (the four quarters sit in one quad)
+    float mx = 0.0f;
+#pragma unroll
+    for (int c = 0; c < L::kCodes; ++c) mx = fmaxf(mx, fabsf(to_f32(xv[c])));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    // e = 14 - floor(log2(mx)), kept inside the normal fp32 range
+    int e = 0;
+    if (mx > 0.0f) {
+      const int E = ((__float_as_int(mx) >> 23) & 0xFF) - 127;
+      e = min(max(14 - E, -100), 126);
+    }
+    float sx = 0.0f, ss = 0.0f;
+    __align__(16) uint32_t outv[L::kOuts];
+#pragma unroll
+    for (int o = 0; o < L::kOuts; ++o) {
+      const float sc = exp2i(e - L::lo_pos(o));
+      const float xl = to_f32(xv[L::lo_code(o)]), xh = to_f32(xv[L::hi_code(o)]);
+      const __half hl = __float2half_rn(xl * sc), hh = __float2half_rn(xh * sc);
+      ss += __half2float(hl) + __half2float(hh);
+      sx += xl + xh;
+      outv[o] = (uint32_t)__half_as_ushort(hl) | ((uint32_t)__half_as_ushort(hh) << 16);
+    }
+    if (act) {
+      uint4* dst = reinterpret_cast<uint4*>(xs + (int64_t)m * tok_stride + (size_t)(gl * 4 + tt) * L::kCodes * 2);
+#pragma unroll
+      for (int c = 0; c < L::kOuts / 4; ++c) dst[c] = reinterpret_cast<const uint4*>(outv)[c];
+    }
+    sx += __shfl_xor_sync(0xffffffffu, sx, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    sx += __shfl_xor_sync(0xffffffffu, sx, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     if (act && tt == 0) {
-      xsum[gl * TOKP + m] = sb;
-      if constexpr (NX == 2) xsum[(Gpad + gl) * TOKP + m] = so;
+      const float c = exp2i(-e);
+      rec[gl * TOKP + m] = make_float4(c, -L::kOff * c * ss, sx, 0.0f);
     }
   }
-  for (int idx = sid; idx < Gpad * TOKP * NX; idx += NTHR)
-    if (idx % TOKP >= np) xsum[idx] = 0.0f;
+  for (int idx = sid; idx < Gpad * TOKP; idx += NTHR)
+    if (idx % TOKP >= np) rec[idx] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
 template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
@@ -329,9 +389,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
                     const __grid_constant__ CUtensorMap tmb0, const __grid_constant__ CUtensorMap tmc1,
                     const __grid_constant__ CUtensorMap tms1, const __grid_constant__ CUtensorMap tmb1) {
   using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE>;
-  using S = typename C::S;
+  using L = typename C::L;
   constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC, CH = C::CH;
-  constexpr float OFF = S::kOff;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const QgemvParams& q = p.q;
@@ -345,7 +404,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   const uint32_t bar_pempty = bar_pfull + 8 * kRB;
   const uint32_t part_sa = smem_u32(smem + p.off_part);
   uint8_t* xs = smem + p.off_xs;
-  float* xsum = reinterpret_cast<float*>(smem + p.off_xsum);
+  float4* xrec = reinterpret_cast<float4*>(smem + p.off_xsum);  // [Gpad][TOKP] group records
   const int E = q.num_experts;
   int* s_cnt = reinterpret_cast<int*>(smem + p.off_plan);
   int* s_start = s_cnt + E;
@@ -366,6 +425,25 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       mbar_init(bar_pempty + 8 * e, 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Dense calls know their tiles without reading memory: before waiting for
+  // the previous kernel, the producer asks L2 for the first units of its
+  // range.  A prefetch only chooses which lines sit in L2 (the point of
+  // coherence), never their contents, so it is safe even when the previous
+  // kernel writes these weights; the copies into shared memory come after the
+  // wait.
+  if (!q.ids && warp == C::PRODUCER && lane == 0) {
+    const int TTd = ((q.n_pairs + CH - 1) / CH) * p.ntiles_e;
+    const int tb0 = (int)((int64_t)TTd * blockIdx.x / gridDim.x);
+    const int te0 = (int)((int64_t)TTd * (blockIdx.x + 1) / gridDim.x);
+    const int nun = min((te0 - tb0) * p.upt, STAGES);
+    for (int i = 0; i < nun; ++i) {
+      const int t = tb0 + i / p.upt, ku = i % p.upt;
+      const int y = (t % p.ntiles_e) * 16;
+      tma_prefetch_3d(&tmc0, 0, y, ku * C::Z);
+      tma_prefetch_2d(&tms0, ku * GPU, y);
+      tma_prefetch_2d(&tmb0, ku * GPU, y);
+    }
   }
   // weights, ids and x may all come from the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -505,24 +583,23 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 
   // --------------------------------------------------------------- consumers
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t xs_sa = smem_u32(xs), xsum_sa = smem_u32(xsum);
-  // per-group sums: pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
-  const uint32_t xsum_lane = xsum_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 4);
+  const uint32_t xs_sa = smem_u32(xs), xrec_sa = smem_u32(xrec);
+  // per-group records of pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
+  const uint32_t xrec_lane = xrec_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 16);
   // shared offset (within a slot) of this lane's code words, row g, for group
   // u: coff(u).  When a warp's groups share one 128-byte slice and the group
   // step only touches chunk bits above the lane's own, coff(u) is coff(0) with
   // those chunk bits flipped (no per-group register).
   constexpr bool kXorGroups = (GPW * WPG <= 32) && (32 % (GPW * WPG) == 0) && (WPG % 4 == 0) &&
-                              (S::kRegs <= 4) && ((WPG / 4) & (4 * S::kRegs / 4 - 1)) == 0;
+                              (L::kRegs <= 4) && ((WPG / 4) & (4 * L::kRegs / 4 - 1)) == 0;
   auto coff_of = [&](int u) -> uint32_t {
-    const int w0 = (warp * GPW + u) * WPG + t * S::kRegs;  // first word in the unit row
+    const int w0 = (warp * GPW + u) * WPG + t * L::kRegs;  // first word in the unit row
     const int wb = w0 & 31;
     return (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
   };
   uint32_t coff[kXorGroups ? 1 : GPW];
 #pragma unroll
   for (int u = 0; u < (kXorGroups ? 1 : GPW); ++u) coff[u] = coff_of(u);
-  const uint32_t magic = p.magic;
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
   // groups (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
   constexpr int PITCH = GPU * 2;
@@ -546,11 +623,11 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   uint32_t xb[MT], xbu[MT];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) { xb[mt] = xs_sa; xbu[mt] = xs_sa; }
-  uint32_t su = xsum_lane;
+  uint32_t su = xrec_lane;
   // one pair: this warp's x fragments and group sums of the current k-unit,
   // in registers (reloaded only when the k-unit or the segment changes)
-  uint4 xr[C::ONE ? GPW : 1][S::kSteps / 2];
-  float xsr[C::ONE ? GPW : 1][C::NX];
+  uint4 xr[C::ONE ? GPW : 1][L::kSteps / 2];
+  float4 xsr[C::ONE ? GPW : 1];
   int xku = -1;
   Walk w;  // the work-list walk of MoE calls (a dense call is one segment)
   if constexpr (MOE) {
@@ -572,18 +649,18 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       for (int m = 0; m < np && same; ++m) same = pair_offset(q, pn[m]) == s_xoff[m];
       if (!same) {
         asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
-        stage_x<S, T, TOKP, C::NX, KC * 32>(q, pn, np, Gpad, p.tok_stride, tid, xs, xsum);
+        stage_x<L, T, TOKP, KC * 32>(q, pn, np, Gpad, p.tok_stride, tid, xs, xrec);
         if (tid < np) s_xoff[tid] = pair_offset(q, pn[tid]);
         cur_np = np;
         asm volatile("bar.sync 1, %0;" ::"n"(KC * 32) : "memory");
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
           const int tr = (mt * 8 + g) < np ? mt * 8 + g : 0;  // idle columns reread pair 0
-          xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * S::kVirt * (int)sizeof(T)) +
+          xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * L::kCodes * 2) +
                    (uint32_t)(warp * GPW * C::XG);
           xbu[mt] = xb[mt];
         }
-        su = xsum_lane;
+        su = xrec_lane;
         xku = -1;
       }
     }
@@ -599,9 +676,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
         for (int u = 0; u < GPW; ++u) {
 #pragma unroll
-          for (int q2 = 0; q2 < S::kSteps / 2; ++q2) xr[u][q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
-          xsr[u][0] = ldsf(su + (uint32_t)(u * TOKP * 4));
-          if constexpr (C::NX == 2) xsr[u][C::NX - 1] = ldsf(su + (uint32_t)((Gpad + u) * TOKP * 4));
+          for (int q2 = 0; q2 < L::kSteps / 2; ++q2) xr[u][q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
+          const uint4 r = lds128(su + (uint32_t)(u * TOKP * 16));
+          xsr[u] = make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), 0.0f);
         }
       }
     }
@@ -632,18 +709,18 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         }
 #pragma unroll
         for (int u = 0; u < GPW; ++u) {
-          uint32_t rA[S::kRegs], rB[S::kRegs];
+          uint32_t rA[L::kRegs], rB[L::kRegs];
           const uint32_t ca = kXorGroups ? csl + (coff[0] ^ (uint32_t)((u * (WPG / 4)) << 4)) : csl + coff[kXorGroups ? 0 : u];
-          if constexpr (S::kRegs >= 4) {
+          if constexpr (L::kRegs >= 4) {
             const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
 #pragma unroll
-            for (int k = 0; k < S::kRegs / 4; ++k) {
+            for (int k = 0; k < L::kRegs / 4; ++k) {
               const uint32_t ch = (uint32_t)(((c0 ^ (uint32_t)g) + k) ^ (uint32_t)g);
               const uint4 va = lds128(cbase + (ch << 4)), vb = lds128(cbase + 1024 + (ch << 4));
               rA[4 * k] = va.x; rA[4 * k + 1] = va.y; rA[4 * k + 2] = va.z; rA[4 * k + 3] = va.w;
               rB[4 * k] = vb.x; rB[4 * k + 1] = vb.y; rB[4 * k + 2] = vb.z; rB[4 * k + 3] = vb.w;
             }
-          } else if constexpr (S::kRegs == 2) {
+          } else if constexpr (L::kRegs == 2) {
             const uint2 va = lds64(ca), vb = lds64(ca + 1024);
             rA[0] = va.x; rA[1] = va.y; rB[0] = vb.x; rB[1] = vb.y;
           } else {
@@ -652,44 +729,29 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           }
           float d[MT][4];
           if constexpr (C::ONE)
-            group_dot_rx<BITS, S, T>(rA, rB, xr[u], d[0], magic);
+            group_dot_rx<L>(rA, rB, xr[u], d[0]);
           else
-            group_dot1<BITS, S, T, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d, magic);
+            group_dot1<L, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d);
           const int hw = u & 1;
           const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
           const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
+          // y += s * (2^-e * D - 1024 * 2^-e * sum x'') + b * sum x, per (row, pair)
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             float(&a_)[4] = acc[ns][mt];
             if constexpr (C::ONE) {
-              const float X0 = xsr[u][0];
-              if constexpr (C::NX == 1) {
-                a_[0] = fmaf(fmaf(-OFF, sa, ba), X0, fmaf(sa, d[0][0], a_[0]));
-                a_[2] = fmaf(fmaf(-OFF, sb_, bb), X0, fmaf(sb_, d[0][2], a_[2]));
-              } else {
-                const float O0 = xsr[u][C::NX - 1];
-                a_[0] = fmaf(ba, X0, fmaf(-OFF * sa, O0, fmaf(sa, d[0][0], a_[0])));
-                a_[2] = fmaf(bb, X0, fmaf(-OFF * sb_, O0, fmaf(sb_, d[0][2], a_[2])));
-              }
+              const float4 r = xsr[u];
+              a_[0] = fmaf(ba, r.z, fmaf(sa, fmaf(d[0][0], r.x, r.y), a_[0]));
+              a_[2] = fmaf(bb, r.z, fmaf(sb_, fmaf(d[0][2], r.x, r.y), a_[2]));
             } else {
-              const uint2 xr2 = lds64(su + (uint32_t)((u * TOKP + mt * 8) * 4));
-              const float X0 = __uint_as_float(xr2.x), X1 = __uint_as_float(xr2.y);
-              if constexpr (C::NX == 1) {
-                const float ca_ = fmaf(-OFF, sa, ba), cb_ = fmaf(-OFF, sb_, bb);
-                a_[0] = fmaf(ca_, X0, fmaf(sa, d[mt][0], a_[0]));
-                a_[1] = fmaf(ca_, X1, fmaf(sa, d[mt][1], a_[1]));
-                a_[2] = fmaf(cb_, X0, fmaf(sb_, d[mt][2], a_[2]));
-                a_[3] = fmaf(cb_, X1, fmaf(sb_, d[mt][3], a_[3]));
-              } else {
-                // bias term on sum(x), offset term on sum(x') (x' = x and 16 x)
-                const uint2 xo = lds64(su + (uint32_t)(((Gpad + u) * TOKP + mt * 8) * 4));
-                const float O0 = __uint_as_float(xo.x), O1 = __uint_as_float(xo.y);
-                const float oa = -OFF * sa, ob = -OFF * sb_;
-                a_[0] = fmaf(ba, X0, fmaf(oa, O0, fmaf(sa, d[mt][0], a_[0])));
-                a_[1] = fmaf(ba, X1, fmaf(oa, O1, fmaf(sa, d[mt][1], a_[1])));
-                a_[2] = fmaf(bb, X0, fmaf(ob, O0, fmaf(sb_, d[mt][2], a_[2])));
-                a_[3] = fmaf(bb, X1, fmaf(ob, O1, fmaf(sb_, d[mt][3], a_[3])));
-              }
+              const uint4 q0 = lds128(su + (uint32_t)((u * TOKP + mt * 8) * 16));
+              const uint4 q1 = lds128(su + (uint32_t)((u * TOKP + mt * 8) * 16 + 16));
+              const float c0 = __uint_as_float(q0.x), n0 = __uint_as_float(q0.y), X0 = __uint_as_float(q0.z);
+              const float c1 = __uint_as_float(q1.x), n1 = __uint_as_float(q1.y), X1 = __uint_as_float(q1.z);
+              a_[0] = fmaf(ba, X0, fmaf(sa, fmaf(d[mt][0], c0, n0), a_[0]));
+              a_[1] = fmaf(ba, X1, fmaf(sa, fmaf(d[mt][1], c1, n1), a_[1]));
+              a_[2] = fmaf(bb, X0, fmaf(sb_, fmaf(d[mt][2], c0, n0), a_[2]));
+              a_[3] = fmaf(bb, X1, fmaf(sb_, fmaf(d[mt][3], c1, n1), a_[3]));
             }
           }
         }
@@ -734,11 +796,11 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) xbu[mt] = xb[mt];
-      su = xsum_lane;
+      su = xrec_lane;
     } else {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) xbu[mt] += (uint32_t)(GPU * C::XG);
-      su += (uint32_t)(GPU * TOKP * 4);
+      su += (uint32_t)(GPU * TOKP * 16);
     }
     if (++slot == STAGES) {
       slot = 0;
@@ -803,14 +865,13 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   p.upt = (q.G + C::GPU - 1) / C::GPU;
   p.ntiles_e = (int)((q.n_rows + 15) / 16);
   p.CH = C::CH;
-  p.magic = C::S::kMagic;
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
   // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums | plan]
   const size_t part = C::ONE ? (size_t)kRB * C::KC * NS * 16 * 4 : (size_t)kRB * C::KC * NS * C::MT * 32 * 16;
   const size_t xs = align128((size_t)C::CH * p.tok_stride);
-  const size_t xsum = align128((size_t)Gpad * C::TOKP * 4 * C::NX);
+  const size_t xsum = align128((size_t)Gpad * C::TOKP * 16);  // float4 records
   const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
   const size_t plan = align128((size_t)(5 * q.num_experts + 1 + 2 * q.n_pairs) * sizeof(int));
   if (plan > 32 * 1024) return cudaErrorNotSupported;
@@ -874,9 +935,9 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
 // mode 0 when n_pairs <= 8, otherwise segments of up to 8 pairs (mode 1).
 template <int BITS, int GS, typename T>
 cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t st) {
-  using S = Share<BITS, GS, T>;
-  if constexpr (S::kFast) {
-    constexpr int WPG = S::kWordsPerGroup;
+  using L = Lanes<BITS, GS>;
+  if constexpr (L::kOk) {
+    constexpr int WPG = L::kWordsPerGroup;
     constexpr int UB = WPG >= 32 ? 16 : 32;  // base unit
     constexpr int UW = WPG <= 8 ? 64 : UB;   // wide unit: 4 groups per consumer
     if (dual) {
