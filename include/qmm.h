@@ -220,6 +220,67 @@ qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype
                                                 qmm_dtype out_dtype, int32_t* d_status,
                                                 void* stream);
 
+/* ------------------------------------------------------------------------
+ * MoE prefill GEMM: many tokens per expert ("ferrum-kernels 0.7.7
+ * src/stacked_expert.rs", StackedExpertGgufLinear::gemm_moe_id and
+ * gemm_moe_id_indirect, with the routing step of compute_ids_tpe_gpu).
+ *
+ *   out[p, :] = a[row(p), :] . dequant(W[ids[p]])^T,  p = token * top_k + slot
+ *   row(p) = token when ne11 == 1 (a is [batch, K]: every slot of a token reads
+ *            its row, as the gate and up projections do), p when ne11 == top_k
+ *            (a is [batch * top_k, K]: one row per pair, as the down
+ *            projection reads the per-slot activations).
+ *
+ * Two calls on one stream, no host round trip in between (the reason the
+ * page's indirect variant exists): qmm_moe_compute_ids_tpe builds, on the
+ * device, the tokens-per-expert counts, the pair indices grouped by expert
+ * and the list of work blocks (<= 256 pairs of one expert each), together
+ * with the page's 12-byte triple, in the caller's workspace; qmm_moe_gemm_id
+ * reads that schedule on the device (its grid never depends on it).
+ *
+ * Workspace: qmm_moe_gemm_workspace_bytes(n_pairs, num_experts) bytes of
+ * device memory, 4-byte aligned, owned by the caller and reused across calls;
+ * int32 fields, in order, each padded to a multiple of 4 entries where noted:
+ *   tpe[E]            pairs routed to expert e ("tokens per expert")
+ *   off[E + 1]        exclusive prefix of tpe; off[E] = pairs with a valid id
+ *   args[3]           {work blocks, largest tpe, experts with tpe > 0}
+ *   (pad), pairs[n_pairs] (pad)   pair indices grouped by expert in expert
+ *                     order (the order inside a group is unspecified);
+ *                     pairs with an id outside [0, E) come last
+ *   blk_e[nb] (pad), blk_s[nb] (pad)   expert and first entry of each block,
+ *                     nb = ceil(n_pairs / 256) + E entries reserved
+ * A pair whose id is outside [0, E) gets a zero output row and sets
+ * QMM_ERR_BAD_EXPERT_ID in *d_status (qmm_moe_compute_ids_tpe).
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes for n_pairs pairs over num_experts experts (-1 when
+ * n_pairs < 0, num_experts outside [1, 8192], or n_pairs > 2^30 - 1). */
+int64_t qmm_moe_gemm_workspace_bytes(int64_t n_pairs, int64_t num_experts);
+
+/* Routing (compute_ids_tpe): ids is device int32[n_pairs] (the [batch, top_k]
+ * routing table, row-major).  Writes the workspace fields above; one CTA.
+ * Errors: INVALID_ARG (sizes, workspace_bytes too small), ALIGNMENT (ids,
+ * workspace or d_status not 4-byte aligned), UNSUPPORTED (device), CUDA.
+ * Device-side: QMM_ERR_BAD_EXPERT_ID in *d_status (may be NULL). */
+qmm_status qmm_moe_compute_ids_tpe(const int32_t* ids, int64_t n_pairs, int64_t num_experts,
+                                   void* workspace, int64_t workspace_bytes, int32_t* d_status,
+                                   void* stream);
+
+/* The expert-grouped GEMM over the schedule in `workspace` (written by
+ * qmm_moe_compute_ids_tpe for the same n_pairs = batch * top_k and the same
+ * number of experts, earlier on this stream).  a: [batch * ne11, K] in a_dtype
+ * (bf16 or f16, equal to w->sdtype), K = w->n_cols; out: [batch * top_k,
+ * w->n_rows] in out_dtype (a_dtype or f32), row p for pair p.  tcgen05 tensor
+ * cores, fp32 accumulate, the dequantized weights rounded once to a_dtype.
+ * Errors: INVALID_ARG (shapes, ne11 not 1 or top_k, workspace too small),
+ * DTYPE, UNSUPPORTED (f32 activations, device), ALIGNMENT (a and out
+ * 16-byte aligned, workspace 4-byte aligned), CUDA.  A device-side timeout
+ * writes the affected tiles as NaN. */
+qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int64_t top_k,
+                           int64_t ne11, const void* workspace, int64_t workspace_bytes,
+                           const qmm_expert_stack* w, void* out, qmm_dtype out_dtype,
+                           void* stream);
+
 /* Diagnostic of the bounded device-side waits (not a step of the method).
  * Every TMA-fed kernel here waits on shared-memory mbarriers with a poll
  * limit and reports QMM_ERR_TIMEOUT instead of hanging when a wait gives up.

@@ -352,3 +352,32 @@ def moe_gate_up_silu_batched(a, a_dtype, ids, m, top_k, outer, inner, gate: Stac
                                               _ptr(out), lo, hi)
     rc = _run(fn, 0, m * top_k, n_threads)
     return out, rc
+
+
+def moe_batched_dense(a, a_dtype, ids, m, top_k, outer, inner, st: Stack, n_threads=None):
+    """fp64 out[p] = a[(p/top_k)*outer + (p%top_k)*inner : ... + n_cols] .
+    dequant(W[ids[p]])^T for whole-output checks of large MoE calls: each
+    expert used is dequantized by this oracle (fmaf, bit-exact), its pairs'
+    rows are gathered, and the product is one library fp64 matrix multiply
+    per expert (numpy).  Same definition as moe_gemv_id_batched (summation
+    order aside); a pair with an id outside [0, E) gets a zero row and
+    rc = ORC_ERR_ID."""
+    a = widen_f64(np.ascontiguousarray(a).reshape(-1), a_dtype)
+    ids = np.ascontiguousarray(ids, dtype=np.int32).reshape(-1)
+    P = m * top_k
+    out = np.zeros((P, st.n_rows), dtype=np.float64)
+    rc = ORC_OK
+    K = st.n_cols
+    n_experts = st.c.num_experts
+    for e in np.unique(ids[:P]):
+        sel = np.nonzero(ids[:P] == e)[0]
+        if e < 0 or e >= n_experts:
+            rc = ORC_ERR_ID
+            continue
+        r0, r1 = int(e) * st.n_rows, (int(e) + 1) * st.n_rows
+        w = dequantize(st.packed[r0:r1], st.scales[r0:r1], st.biases[r0:r1], st.c.s_dtype, K,
+                       st.c.gs, st.c.bits, F32, n_threads).astype(np.float64)
+        offs = (sel // top_k) * outer + (sel % top_k) * inner
+        rows = a[offs[:, None] + np.arange(K)[None, :]]
+        out[sel] = rows @ w.T
+    return out, rc

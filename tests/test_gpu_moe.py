@@ -181,3 +181,30 @@ def test_moe_config_full_size(case):
     ref_d, rc = oracle.moe_gemv_id(h16_np, oracle.BF16, ids.numpy().reshape(-1), T * k, dff, od)
     assert rc == oracle.ORC_OK
     gate(out.cpu().numpy(), ref_d, f"{case.name} down")
+
+
+@pytest.mark.parametrize("gs,n_cols", [(64, 768), (32, 768), (128, 768), (64, 1280), (32, 256)])
+@pytest.mark.parametrize("n_sel", [5, 24])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_moe_short_rows_one_copy_scales(gs, n_cols, n_sel, dtype):
+    """Rows whose scale/bias rows are not 16-byte strided (K / gs = 12, 24, 6,
+    20, 8 groups): the streaming kernel takes a whole row tile per unit and
+    its 16 scale (bias) rows as one contiguous copy, skipping groups past the
+    row; one pair per segment (5 pairs) and segments of 8 (24 pairs)."""
+    E, n_rows, bits = 10, 96, 4
+    st, ost = make_stack(E, n_rows, n_cols, bits, gs, 60 + gs + n_cols, dtype)
+    stride = n_cols + 8
+    dts = {torch.bfloat16: "bf16", torch.float16: "f16"}[dtype]
+    a = wl.gen_x(1, stride * n_sel, 61, dts).reshape(-1)
+    ids = torch.randint(0, E, (n_sel,), generator=torch.Generator().manual_seed(62), dtype=torch.int32)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    g32, g16 = Guarded((n_sel, n_rows), torch.float32), Guarded((n_sel, n_rows), dtype)
+    api.qmm_moe_gemv_id(a.to(DEV), ids.to(DEV), n_sel, stride, st, out=g32.out, d_status=status)
+    api.qmm_moe_gemv_id(a.to(DEV), ids.to(DEV), n_sel, stride, st, out=g16.out, d_status=status)
+    torch.cuda.synchronize()
+    out32, out16 = g32.check("short rows"), g16.check("short rows 16-bit")
+    assert int(status.item()) == 0
+    ref, rc = oracle.moe_gemv_id(np_storage(a), ORC[dtype], ids.numpy(), n_sel, stride, ost)
+    assert rc == oracle.ORC_OK
+    gate(out32.cpu().numpy(), ref, f"short rows g{gs} K{n_cols} n{n_sel}")
+    rne_equal(out16, out32)

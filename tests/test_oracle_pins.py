@@ -506,3 +506,26 @@ def test_matmul_dense_agrees_with_matmul(bits):
     p2[:, 0] = 0
     y3 = oracle.matmul_dense(x, oracle.BF16, p2, s, b, oracle.BF16, N, gs, bits)
     assert np.any(np.abs(y3 - y1) > bound)
+
+
+@pytest.mark.parametrize("outer_inner", [(64, 0), (4 * 64, 64)])
+def test_moe_batched_dense_agrees_with_the_loops(outer_inner):
+    """the per-expert library-GEMM form of the MoE oracle equals the plain
+    per-pair loops within fp64 summation-order error; bad ids zero-filled"""
+    E, n_rows, n_cols, bits, gs, m, top_k = 6, 24, 64, 4, 32, 5, 4
+    outer, inner = outer_inner
+    w = wl.gen_weight(E * n_rows, n_cols, 41).numpy()
+    p, s, b = oracle.quantize(w, oracle.F32, gs, bits, oracle.BF16)
+    st = oracle.Stack(p, s, b, oracle.BF16, E, n_rows, n_cols, gs, bits)
+    a = wl.storage_numpy(wl.gen_x(1, m * outer + top_k * inner + n_cols, 42)).reshape(-1)
+    ids = wl.gen_moe_ids(m, E, top_k, 43).numpy()
+    ids[2, 1] = E + 3  # an out-of-range id
+    ref, rc = oracle.moe_gemv_id_batched(a, oracle.BF16, ids, m, top_k, outer, inner, st)
+    got, rc2 = oracle.moe_batched_dense(a, oracle.BF16, ids, m, top_k, outer, inner, st)
+    assert rc == rc2 == oracle.ORC_ERR_ID
+    assert np.all(got[2 * top_k + 1] == 0)
+    assert np.allclose(got, ref, rtol=0, atol=1e-12)
+    # a swapped offset (inner and outer exchanged) is caught
+    if inner:
+        bad, _ = oracle.moe_batched_dense(a, oracle.BF16, ids, m, top_k, inner, outer, st)
+        assert not np.allclose(bad, ref, rtol=0, atol=1e-6)

@@ -331,3 +331,52 @@ def qmm_moe_gemv_id_gate_up_silu_batched(a: torch.Tensor, ids: torch.Tensor, m: 
         _stream(stream))
     check("qmm_moe_gemv_id_gate_up_silu_batched", rc)
     return out
+
+
+# ------------------------------------------------------------------ MoE prefill GEMM
+def qmm_moe_gemm_workspace_bytes(n_pairs: int, num_experts: int) -> int:
+    return int(_lib.load().qmm_moe_gemm_workspace_bytes(n_pairs, num_experts))
+
+
+def moe_workspace(n_pairs: int, num_experts: int, device=None) -> torch.Tensor:
+    """A device workspace of the size qmm_moe_compute_ids_tpe needs (int32)."""
+    nb = qmm_moe_gemm_workspace_bytes(n_pairs, num_experts)
+    if nb < 0:
+        check("qmm_moe_gemm_workspace_bytes", _lib.QMM_ERR_INVALID_ARG)
+    return torch.empty((nb + 3) // 4, dtype=torch.int32, device=device or "cuda")
+
+
+def qmm_moe_compute_ids_tpe(ids: torch.Tensor, num_experts: int, workspace: torch.Tensor,
+                            d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Route the [batch, top_k] ids on the device into `workspace`."""
+    n = ids.numel()
+    _need(ids, "ids", n, (torch.int32,))
+    _need(workspace, "workspace", 0, (torch.int32,))
+    if d_status is not None:
+        _need(d_status, "d_status", 1, (torch.int32,))
+    _on_device(ids=ids, workspace=workspace, d_status=d_status)
+    rc = _lib.load().qmm_moe_compute_ids_tpe(_ptr(ids), n, num_experts, _ptr(workspace),
+                                             workspace.numel() * 4, _ptr(d_status), _stream(stream))
+    check("qmm_moe_compute_ids_tpe", rc)
+    return workspace
+
+
+def qmm_moe_gemm_id(a: torch.Tensor, batch: int, top_k: int, ne11: int, workspace: torch.Tensor,
+                    w: ExpertStack, out_dtype: torch.dtype | None = None, out=None,
+                    stream=None) -> torch.Tensor:
+    """out[p] = a[row(p)] . dequant(W[ids[p]])^T over the routed workspace;
+    a is [batch * ne11, K] (ne11 = 1 or top_k); out is [batch * top_k, n_rows]."""
+    n_pairs = batch * top_k
+    if out is None:
+        out = torch.empty(n_pairs, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    _need(a, "a", batch * ne11 * w.n_cols, _FLOAT)
+    named = w.validate()
+    _need(workspace, "workspace", 0, (torch.int32,))
+    _need(out, "out", n_pairs * w.n_rows, _FLOAT)
+    _on_device(a=a, workspace=workspace, out=out, **named)
+    c = w.c()
+    rc = _lib.load().qmm_moe_gemm_id(_ptr(a), dtype_code(a.dtype), batch, top_k, ne11,
+                                     _ptr(workspace), workspace.numel() * 4, ctypes.byref(c),
+                                     _ptr(out), dtype_code(out.dtype), _stream(stream))
+    check("qmm_moe_gemm_id", rc)
+    return out

@@ -131,6 +131,15 @@ struct GemmParams {
   void* y;
   int y_dtype;
   int M, N, K, G, wpr;
+  // MoE prefill form (MOE instantiation): the schedule that the routing
+  // kernel wrote (see moe_gemm.cu); N is the rows of one expert and y is
+  // [n_pairs, N]
+  const int32_t* ws_off;    // [E + 1] exclusive prefix of pairs per expert; off[E] = valid pairs
+  const int32_t* ws_args;   // [3] blocks of <= 256 pairs, largest expert count, experts used
+  const int32_t* ws_pairs;  // [n_pairs] pair indices grouped by expert, bad ids last
+  const int32_t* ws_blk_e;  // expert of block b
+  const int32_t* ws_blk_s;  // first entry (into ws_pairs) of block b
+  int E, top_k, ne11, n_pairs;
 };
 
 // ------------------------------------------------------------------ dequant helpers
@@ -178,15 +187,41 @@ __device__ __forceinline__ void codes_to_pairs(const uint32_t (&w)[2 * B], uint3
   }
 }
 
-// The CTA's tiles, in order: tile = blockIdx.x + lt * gridDim.x.  Weight-row
-// tiles vary slowest, so the CTAs running at the same time share their x
-// tiles and weight rows through L2.
+// The CTA's tiles, in order: tile = blockIdx.x + lt * gridDim.x.
+//   dense: weight-row tiles vary slowest, so the CTAs running at the same time
+//          share their x tiles and weight rows through L2;
+//   MoE:   blocks of <= 256 pairs of one expert vary slowest, so the CTAs
+//          running at the same time share the gathered activation rows.
+// m0 is the first token (dense) or the first entry of the pair list (MoE);
+// cnt the tokens (pairs) of the tile; e the expert.
 struct TileOf {
-  int n0, m0;
+  int n0, m0, cnt, e;
 };
-__device__ __forceinline__ TileOf tile_of(int lt, int m_tiles) {
+template <bool MOE>
+__device__ __forceinline__ TileOf tile_of(const GemmParams& p, int lt, int m_tiles, int n_tiles) {
   const int t = blockIdx.x + lt * gridDim.x;
-  return TileOf{(t / m_tiles) * gemm::kBM, (t % m_tiles) * gemm::kBN};
+  if constexpr (MOE) {
+    const int b = t / n_tiles, nt = t - b * n_tiles;
+    const int e = __ldg(p.ws_blk_e + b), m0 = __ldg(p.ws_blk_s + b);
+    return TileOf{nt * gemm::kBM, m0, min(gemm::kBN, __ldg(p.ws_off + e + 1) - m0), e};
+  } else {
+    const int nt = t / m_tiles, mt = t - nt * m_tiles;
+    return TileOf{nt * gemm::kBM, mt * gemm::kBN, min(gemm::kBN, p.M - mt * gemm::kBN), 0};
+  }
+}
+// row of the activation matrix that token slot j of a MoE tile reads
+// (slots past the tile's pairs read the first pair's row; they are never stored)
+__device__ __forceinline__ int moe_a_row(const GemmParams& p, const TileOf& tl, int j) {
+  const int pr = __ldg(p.ws_pairs + tl.m0 + (j < tl.cnt ? j : 0));
+  return p.ne11 == 1 ? pr / p.top_k : pr;
+}
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, int c0, int r0, int r1, int r2,
+                                            int r3, uint32_t b) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(m), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(b)
+      : "memory");
 }
 
 // Persistent: every CTA walks its tiles (static round robin over the grid).
@@ -199,7 +234,7 @@ __device__ __forceinline__ TileOf tile_of(int lt, int m_tiles) {
 //   warps 6..9  epilogue: tcgen05.ld of the finished accumulator, release it,
 //               store y directly from registers (per instruction, a warp
 //               writes 32 consecutive weight rows of one token)
-template <int B, int GS, typename T>
+template <int B, int GS, typename T, bool MOE>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
 qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   using namespace gemm;
@@ -219,8 +254,6 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   const int nk = (p.K + kBK - 1) / kBK;
   const int m_tiles = (p.M + kBN - 1) / kBN;
   const int n_tiles = (p.N + kBM - 1) / kBM;
-  const int T_all = m_tiles * n_tiles;
-  const int my_tiles = blockIdx.x < T_all ? (T_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -244,33 +277,52 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // x and the weights may come from the previous kernel in the stream
+  // x, the weights and the MoE schedule may come from the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int T_all = (MOE ? __ldg(p.ws_args) : m_tiles) * n_tiles;
+  const int my_tiles = (int)blockIdx.x < T_all ? (T_all - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      int j = 0, issued = 0;
-      bool stop = false;
-      for (int lt = 0; lt < my_tiles && !stop; ++lt) {
-        const TileOf tl = tile_of(lt, m_tiles);
-        for (int i = 0; i < nk; ++i, ++j) {
-          const int s = j % kStages, u = j / kStages;
-          if (j >= kStages && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) {
-            *abort_flag = 1;
-            stop = true;
-            break;
-          }
+    // dense: lane 0 loads each stage's [256 x 64] x tile; MoE: lane 0 posts
+    // the stage's bytes and every lane gathers the activation rows of 8 token
+    // slots (two 4-row gathers, one row per slot)
+    int j = 0, issued = 0;
+    bool stop = false;
+    for (int lt = 0; lt < my_tiles && !stop; ++lt) {
+      const TileOf tl = tile_of<MOE>(p, lt, m_tiles, n_tiles);
+      int rw[8];
+      if constexpr (MOE) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rw[q] = moe_a_row(p, tl, 8 * lane + q);
+      }
+      for (int i = 0; i < nk; ++i, ++j) {
+        const int s = j % kStages, u = j / kStages;
+        bool ok = true;
+        if (lane == 0 && j >= kStages) ok = bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag);
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+          if (lane == 0) *abort_flag = 1;
+          stop = true;
+          break;
+        }
+        if constexpr (MOE) {
+          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
+          __syncwarp();
+          const uint32_t d = su32(xs + s * kXStage) + (uint32_t)(lane * 8 * 128);
+          tma_gather4(d, &tmx, i * kBK, rw[0], rw[1], rw[2], rw[3], full0 + 8 * s);
+          tma_gather4(d + 512, &tmx, i * kBK, rw[4], rw[5], rw[6], rw[7], full0 + 8 * s);
+        } else if (lane == 0) {
           mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
           tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, tl.m0, full0 + 8 * s);
-          issued = j + 1;
         }
+        issued = j + 1;
       }
-      // no copy may still be landing when the CTA exits: the last copy of every
-      // slot is waited for with the full bound, also after an abort
+    }
+    // no copy may still be landing when the CTA exits: the last copy of every
+    // slot is waited for with the full bound, also after an abort
+    if (lane == 0)
       for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
         mbar_wait_n(full0 + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u, gemm::kSpins);
-    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -323,11 +375,14 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     auto load = [&](int j, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
       const bool in = j < total;
       const int lt = in ? j / nk : 0, i = in ? j - lt * nk : 0;
-      const int n = tile_of(lt, m_tiles).n0 + r;
+      const TileOf tl = tile_of<MOE>(p, in ? lt : 0, m_tiles, n_tiles);
+      const int n = tl.n0 + r;
       const bool nval = in && n < p.N;
-      const uint32_t* row = p.packed + (int64_t)(nval ? n : 0) * p.wpr;
-      const T* srow = reinterpret_cast<const T*>(p.scales) + (int64_t)(nval ? n : 0) * p.G;
-      const T* brow = reinterpret_cast<const T*>(p.biases) + (int64_t)(nval ? n : 0) * p.G;
+      // row of the (stacked) weight matrix: expert e's rows start at e * N
+      const int64_t wr = nval ? (int64_t)tl.e * p.N + n : 0;
+      const uint32_t* row = p.packed + wr * p.wpr;
+      const T* srow = reinterpret_cast<const T*>(p.scales) + wr * p.G;
+      const T* brow = reinterpret_cast<const T*>(p.biases) + wr * p.G;
       const int k0 = i * kBK;
       load_codes<B>(row, k0 * B / 32, p.wpr, nval, w);
 #pragma unroll
@@ -400,9 +455,25 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     const int qq = warp & 3;          // TMEM lane quarter this warp may access
     const int r = qq * 32 + lane;     // weight row of the tile
     const bool f32out = p.y_dtype == QMM_F32;
+    auto put = [&](int64_t idx, float f) {
+      if (f32out)
+        reinterpret_cast<float*>(p.y)[idx] = f;
+      else
+        reinterpret_cast<T*>(p.y)[idx] = from_f32<T>(f);
+    };
+    if constexpr (MOE) {
+      // pairs whose id was out of range (listed last) get zero rows
+      const int bad0 = __ldg(p.ws_off + p.E);
+      const int64_t nz = (int64_t)(p.n_pairs - bad0) * p.N;
+      const int et = (warp - 6) * 32 + lane;
+      for (int64_t z = (int64_t)blockIdx.x * 128 + et; z < nz; z += (int64_t)gridDim.x * 128) {
+        const int pr = __ldg(p.ws_pairs + bad0 + (int)(z / p.N));
+        put((int64_t)pr * p.N + z % p.N, 0.0f);
+      }
+    }
     bool failed = false;
     for (int lt = 0; lt < my_tiles; ++lt) {
-      const TileOf tl = tile_of(lt, m_tiles);
+      const TileOf tl = tile_of<MOE>(p, lt, m_tiles, n_tiles);
       const int b = lt & 1;
       const int n = tl.n0 + r;
       if (!failed) {
@@ -419,13 +490,12 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
         if (n < p.N) {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
-            const int m = tl.m0 + c * 32 + jj;
-            if (m < p.M) {
+            const int slot = c * 32 + jj;
+            if (slot < tl.cnt) {
               const float f = failed ? __int_as_float(0x7fc00000) : __uint_as_float(v[jj]);
-              if (f32out)
-                reinterpret_cast<float*>(p.y)[(int64_t)m * p.N + n] = f;
-              else
-                reinterpret_cast<T*>(p.y)[(int64_t)m * p.N + n] = from_f32<T>(f);
+              // dense: token m0 + slot; MoE: the pair listed at m0 + slot
+              const int64_t orow = MOE ? (int64_t)__ldg(p.ws_pairs + tl.m0 + slot) : (int64_t)(tl.m0 + slot);
+              put(orow * p.N + n, f);
             }
           }
         }
@@ -451,9 +521,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
 
-template <int B, int GS, typename T>
-static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, cudaStream_t st) {
-  auto k = qgemm_tc_kernel<B, GS, T>;
+template <int B, int GS, typename T, bool MOE>
+static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, int grid, cudaStream_t st) {
+  auto k = qgemm_tc_kernel<B, GS, T, MOE>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -463,10 +533,8 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, 
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
-  // persistent: one CTA per SM (or per tile when there are fewer tiles)
-  const int tiles = ((prm.N + gemm::kBM - 1) / gemm::kBM) * ((prm.M + gemm::kBN - 1) / gemm::kBN);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(tiles, qmm_host::num_sms()));
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(gemm::kThreads);
   cfg.dynamicSmemBytes = gemm::kSmem;
   cfg.stream = st;
@@ -478,13 +546,13 @@ static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, 
   return cudaLaunchKernelEx(&cfg, k, prm, tmx);
 }
 
-template <typename T>
-static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const CUtensorMap& tmx,
+template <typename T, bool MOE>
+static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const CUtensorMap& tmx, int grid,
                                  cudaStream_t st) {
 #define QMM_G(BB)                                                             \
-  if (gs == 32) return launch_gemm_t<BB, 32, T>(prm, tmx, st);                \
-  if (gs == 64) return launch_gemm_t<BB, 64, T>(prm, tmx, st);                \
-  return launch_gemm_t<BB, 128, T>(prm, tmx, st);
+  if (gs == 32) return launch_gemm_t<BB, 32, T, MOE>(prm, tmx, grid, st);     \
+  if (gs == 64) return launch_gemm_t<BB, 64, T, MOE>(prm, tmx, grid, st);     \
+  return launch_gemm_t<BB, 128, T, MOE>(prm, tmx, grid, st);
   switch (bits) {
     case 2: { QMM_G(2) }
     case 3: { QMM_G(3) }
@@ -495,26 +563,30 @@ static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const 
 #undef QMM_G
 }
 
+// 2-D map over x [rows, K] (16-bit): boxes of 64 k x box_rows rows, 128-byte swizzle
+static bool make_x_map(CUtensorMap* m, const void* x, int x_dtype, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
+  const cuuint32_t box[2] = {gemm::kBK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      x_dtype == QMM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(m, dt, 2, const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // cudaErrorNotSupported: the call does not fit this kernel (the caller falls back)
 cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
                             void* y, int y_dtype, cudaStream_t st) {
   if (M > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->rows > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
-  EncodeTiledFn enc = tensor_map_encoder();
-  if (!enc) return cudaErrorNotSupported;
   CUtensorMap tmx;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)(K * 2)};
-  const cuuint32_t box[2] = {gemm::kBK, gemm::kBN};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapDataType dt =
-      x_dtype == QMM_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (enc(&tmx, dt, 2, const_cast<void*>(x), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorNotSupported;
-  GemmParams prm;
+  if (!make_x_map(&tmx, x, x_dtype, M, K, gemm::kBN)) return cudaErrorNotSupported;
+  GemmParams prm{};
   prm.packed = w->packed;
   prm.scales = w->scales;
   prm.biases = w->biases;
@@ -525,8 +597,49 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   prm.K = (int)K;
   prm.G = (int)(K / w->group_size);
   prm.wpr = (int)(K * w->bits / 32);
-  if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16>(w->bits, w->group_size, prm, tmx, st);
-  return launch_gemm_b<__half>(w->bits, w->group_size, prm, tmx, st);
+  // persistent: one CTA per SM (or per tile when there are fewer tiles)
+  const int64_t tiles = ((prm.N + gemm::kBM - 1) / gemm::kBM) * (int64_t)((prm.M + gemm::kBN - 1) / gemm::kBN);
+  const int grid = (int)std::min<int64_t>(tiles, qmm_host::num_sms());
+  if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, false>(w->bits, w->group_size, prm, tmx, grid, st);
+  return launch_gemm_b<__half, false>(w->bits, w->group_size, prm, tmx, grid, st);
+}
+
+// MoE prefill GEMM over the schedule that moe_route_kernel wrote into `ws`
+// (see moe_gemm.cu for the layout): a is [a_rows, K], out is [n_pairs, n_rows].
+cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const qmm_expert_stack* w,
+                             const int32_t* ws_off, const int32_t* ws_args, const int32_t* ws_pairs,
+                             const int32_t* ws_blk_e, const int32_t* ws_blk_s, int top_k, int ne11,
+                             int n_pairs, void* out, int out_dtype, cudaStream_t st) {
+  const int64_t K = w->n_cols;
+  if (a_rows > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->n_rows * w->num_experts > (int64_t)INT32_MAX)
+    return cudaErrorNotSupported;
+  if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
+  CUtensorMap tma;  // one-row boxes: the producer gathers 4 rows per copy
+  if (!make_x_map(&tma, a, a_dtype, a_rows, K, 1)) return cudaErrorNotSupported;
+  GemmParams prm{};
+  prm.packed = w->packed;
+  prm.scales = w->scales;
+  prm.biases = w->biases;
+  prm.y = out;
+  prm.y_dtype = out_dtype;
+  prm.M = 0;
+  prm.N = (int)w->n_rows;
+  prm.K = (int)K;
+  prm.G = (int)(K / w->group_size);
+  prm.wpr = (int)(K * w->bits / 32);
+  prm.ws_off = ws_off;
+  prm.ws_args = ws_args;
+  prm.ws_pairs = ws_pairs;
+  prm.ws_blk_e = ws_blk_e;
+  prm.ws_blk_s = ws_blk_s;
+  prm.E = (int)w->num_experts;
+  prm.top_k = top_k;
+  prm.ne11 = ne11;
+  prm.n_pairs = n_pairs;
+  // the work list is known only on the device: one CTA per SM
+  const int grid = qmm_host::num_sms();
+  if (a_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, true>(w->bits, w->group_size, prm, tma, grid, st);
+  return launch_gemm_b<__half, true>(w->bits, w->group_size, prm, tma, grid, st);
 }
 
 }  // namespace qmm

@@ -66,6 +66,7 @@ struct Params {
   int CH;               // pairs per segment
   int tok_stride;       // bytes between staged rows of x
   int stages;           // ring depth
+  uint32_t tx;          // bytes that land per unit (all matrices)
   int off_code, off_sb, off_bar, off_part, off_xs, off_xsum, off_plan;
 };
 
@@ -102,8 +103,12 @@ struct Lanes {
 
 // MODE 0: one pair per segment; 1: up to 8; 2: up to 16.  UG: groups per unit
 // (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
-// matrices per pair (2: gate and up).
-template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
+// matrices per pair (2: gate and up).  SB1: rows of G <= UG groups whose
+// scale/bias rows are not 16-byte strided (G % 8 != 0, e.g. K = 768 at group
+// 64): a unit is a whole row tile, its 16 scale (bias) rows arrive as one
+// contiguous 1-D bulk copy of 32 G bytes, unswizzled, and groups >= G are
+// skipped.
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false>
 struct Cfg {
   using L = Lanes<BITS, GS>;
   static constexpr int MT = MODE == 2 ? 2 : 1;
@@ -117,7 +122,6 @@ struct Cfg {
   static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
   static constexpr int CODE_BYTES = Z * 16 * 128;                 // one matrix
   static constexpr int SB_BYTES = 16 * GPU * 2;                   // scales (or biases) of one matrix
-  static constexpr uint32_t TX = NS * (CODE_BYTES + 2 * SB_BYTES);
   static constexpr int TOKP = 8 * MT;
   static constexpr int CH = ONE ? 1 : TOKP;                       // pairs per segment
   static constexpr int XG = 4 * L::kCodes * 2;                    // staged f16 x bytes per group
@@ -142,6 +146,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(map), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
+}
+
+// Contiguous global -> shared copy of `bytes` (a multiple of 16, both
+// addresses 16-byte aligned), counted on the mbarrier's transaction bytes.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // L2 prefetches of one box of a tensor map (no shared memory, no barrier)
@@ -383,12 +395,12 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     if (idx % TOKP >= np) rec[idx] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
-__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS, MOE>::THREADS, 1)
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1>
+__global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS, MOE, SB1>::THREADS, 1)
 qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, const __grid_constant__ CUtensorMap tms0,
                     const __grid_constant__ CUtensorMap tmb0, const __grid_constant__ CUtensorMap tmc1,
                     const __grid_constant__ CUtensorMap tms1, const __grid_constant__ CUtensorMap tmb1) {
-  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE>;
+  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE, SB1>;
   using L = typename C::L;
   constexpr int GPU = C::GPU, GPW = C::GPW, TOKP = C::TOKP, WPG = C::WPG, MT = C::MT, KC = C::KC, CH = C::CH;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -497,12 +509,18 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         }
         const int y = s_dist[w.j] * (int)q.n_rows + w.rt * 16;  // first row in the expert stack
         const uint32_t fb = bar_full + 8 * slot;
-        mbar_arrive_expect_tx(fb, C::TX);
+        mbar_arrive_expect_tx(fb, p.tx);
         const uint32_t cd = code_ring + (uint32_t)(slot * NS * C::CODE_BYTES);
         const uint32_t sd = sb_ring + (uint32_t)(slot * NS * 2 * C::SB_BYTES);
         tma_load_3d(cd, &tmc0, 0, y, ku * C::Z, fb);
-        tma_load_2d(sd, &tms0, ku * GPU, y, fb);
-        tma_load_2d(sd + C::SB_BYTES, &tmb0, ku * GPU, y, fb);
+        if constexpr (SB1) {  // rows y .. y + 15 of the [rows, G] arrays, contiguous
+          const uint32_t nb = (uint32_t)(32 * q.G);
+          bulk_load_1d(sd, reinterpret_cast<const uint8_t*>(q.scales[0]) + (int64_t)y * q.G * 2, nb, fb);
+          bulk_load_1d(sd + C::SB_BYTES, reinterpret_cast<const uint8_t*>(q.biases[0]) + (int64_t)y * q.G * 2, nb, fb);
+        } else {
+          tma_load_2d(sd, &tms0, ku * GPU, y, fb);
+          tma_load_2d(sd + C::SB_BYTES, &tmb0, ku * GPU, y, fb);
+        }
         if constexpr (NS == 2) {
           tma_load_3d(cd + C::CODE_BYTES, &tmc1, 0, y, ku * C::Z, fb);
           tma_load_2d(sd + 2 * C::SB_BYTES, &tms1, ku * GPU, y, fb);
@@ -602,10 +620,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   for (int u = 0; u < (kXorGroups ? 1 : GPW); ++u) coff[u] = coff_of(u);
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
   // groups (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
-  constexpr int PITCH = GPU * 2;
+  // (SB1: plain [16][G] rows, pitch 2 G bytes)
+  const int PITCH = SB1 ? 2 * q.G : GPU * 2;
   const int sfx = PITCH == 128 ? (g & 7) : PITCH == 64 ? ((g >> 1) & 3) : ((g >> 2) & 1);
   const int sbyte = warp * GPW * 2;
-  const uint32_t soff = (uint32_t)(g * PITCH + ((((sbyte >> 4) ^ sfx)) << 4) + (sbyte & 15));
+  const uint32_t soff = SB1 ? (uint32_t)(g * PITCH + sbyte)
+                            : (uint32_t)(g * PITCH + ((((sbyte >> 4) ^ sfx)) << 4) + (sbyte & 15));
+  // SB1: this warp's groups past the row (>= G) take no part in the sums
+  const int live = SB1 ? min(GPW, max(0, q.G - warp * GPW)) : GPW;
 
   float acc[NS][MT][4];
 #pragma unroll
@@ -692,7 +714,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint32_t ra = ssl + (uint32_t)(h * 8 * PITCH);
-          if constexpr (GPW == 1) {
+          if constexpr (SB1) {  // 2-byte aligned only: one value at a time
+#pragma unroll
+            for (int c = 0; c < (GPW + 1) / 2; ++c) {
+              sv[h][c] = lds16(ra + 4 * c) | (2 * c + 1 < GPW ? lds16(ra + 4 * c + 2) << 16 : 0u);
+              bv[h][c] = lds16(ra + C::SB_BYTES + 4 * c) |
+                         (2 * c + 1 < GPW ? lds16(ra + C::SB_BYTES + 4 * c + 2) << 16 : 0u);
+            }
+          } else if constexpr (GPW == 1) {
             sv[h][0] = lds16(ra);
             bv[h][0] = lds16(ra + C::SB_BYTES);
           } else if constexpr (GPW == 2) {
@@ -709,6 +738,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         }
 #pragma unroll
         for (int u = 0; u < GPW; ++u) {
+          if (SB1 && u >= live) break;  // warp-uniform
           uint32_t rA[L::kRegs], rB[L::kRegs];
           const uint32_t ca = kXorGroups ? csl + (coff[0] ^ (uint32_t)((u * (WPG / 4)) << 4)) : csl + coff[kXorGroups ? 0 : u];
           if constexpr (L::kRegs >= 4) {
@@ -850,12 +880,19 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
 }
 
 // cudaErrorNotSupported sends the caller to the general kernels.
-template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE>
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false>
 cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
-  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE>;
+  using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE, SB1>;
   if (MOE != (q.ids != nullptr)) return cudaErrorNotSupported;
   const int64_t rows_total = q.n_rows * q.num_experts;
-  if (q.n_pairs < 1 || q.G % 8 != 0 || q.wpr % 32 != 0 || rows_total < 16 || q.G < C::GPU) return cudaErrorNotSupported;
+  if (q.n_pairs < 1 || q.wpr % 32 != 0 || rows_total < 16) return cudaErrorNotSupported;
+  if (SB1) {
+    // one unit per row tile; 16-row tiles of every expert start on 16-byte
+    // aligned scale/bias rows and never run past the arrays
+    if (q.G > C::GPU || q.n_rows % 16 != 0 || NS != 1) return cudaErrorNotSupported;
+  } else if (q.G % 8 != 0 || q.G < C::GPU) {
+    return cudaErrorNotSupported;
+  }
   if (rows_total + 16 >= ((int64_t)1 << 31) || (int64_t)q.n_pairs * q.K >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
   for (int ns = 0; ns < NS; ++ns)
     if (((uintptr_t)q.packed[ns] | (uintptr_t)q.scales[ns] | (uintptr_t)q.biases[ns]) & 15) return cudaErrorNotSupported;
@@ -865,6 +902,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   p.upt = (q.G + C::GPU - 1) / C::GPU;
   p.ntiles_e = (int)((q.n_rows + 15) / 16);
   p.CH = C::CH;
+  p.tx = (uint32_t)(NS * C::CODE_BYTES + NS * (SB1 ? 2 * 32 * q.G : 2 * C::SB_BYTES));
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
@@ -881,7 +919,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   };
   // about 144 KB of the weight stream in flight per SM (measured: deeper rings
   // and an L2 prefetch window ahead of the ring were not faster)
-  int stages = (int)((144 * 1024) / C::TX);
+  int stages = (int)((144 * 1024) / p.tx);
   stages = stages < 2 ? 2 : (stages > kMaxStages ? kMaxStages : stages);
   while (stages > 2 && total(stages) > (size_t)kSmemMax) --stages;
   if (total(stages) > (size_t)kSmemMax) return cudaErrorNotSupported;
@@ -896,14 +934,19 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   const size_t smem = total(stages);
 
   CUtensorMap tm[6];
-  for (int ns = 0; ns < NS; ++ns)
-    if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z) ||
-        !make_sb_map(&tm[3 * ns + 1], q.scales[ns], rows_total, q.G, C::GPU) ||
-        !make_sb_map(&tm[3 * ns + 2], q.biases[ns], rows_total, q.G, C::GPU))
+  for (int ns = 0; ns < NS; ++ns) {
+    if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z)) return cudaErrorNotSupported;
+    if (SB1) {  // no scale/bias maps: 1-D bulk copies
+      tm[3 * ns + 1] = tm[3 * ns];
+      tm[3 * ns + 2] = tm[3 * ns];
+    } else if (!make_sb_map(&tm[3 * ns + 1], q.scales[ns], rows_total, q.G, C::GPU) ||
+               !make_sb_map(&tm[3 * ns + 2], q.biases[ns], rows_total, q.G, C::GPU)) {
       return cudaErrorNotSupported;
+    }
+  }
   if (NS == 1) { tm[3] = tm[0]; tm[4] = tm[1]; tm[5] = tm[2]; }
 
-  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS, MOE>;
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS, MOE, SB1>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -945,6 +988,17 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
       return launch_stream<BITS, GS, T, 1, UB, 2, true>(q, st);
     }
     if (q.ids) {
+      if (q.G % 8 != 0 || q.G < UB) {  // short or odd rows (e.g. the MoE down projection)
+        if (q.G <= 16) {
+          if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, 16, 1, true, true>(q, st);
+          return launch_stream<BITS, GS, T, 1, 16, 1, true, true>(q, st);
+        }
+        if constexpr (WPG <= 16) {  // a 32-group unit of at most 16 slices
+          if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, 32, 1, true, true>(q, st);
+          return launch_stream<BITS, GS, T, 1, 32, 1, true, true>(q, st);
+        }
+        return cudaErrorNotSupported;
+      }
       if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 1, true>(q, st);
       return launch_stream<BITS, GS, T, 1, UB, 1, true>(q, st);
     }
