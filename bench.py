@@ -485,7 +485,7 @@ def _gbs(nbytes, ms, hbm_peak):
 def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
     out = {}
     for name, fn in (("moe", secondary_moe), ("sweep", secondary_sweep),
-                     ("prefill", secondary_prefill)):
+                     ("prefill", secondary_prefill), ("moe_prefill", secondary_moe_prefill)):
         try:
             out[name] = fn(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust)
         except Exception as e:  # pragma: no cover
@@ -568,6 +568,40 @@ def secondary_sweep(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust)
             out[c.name] = _gbs(decode_bytes(c.M, c.N, c.K, c.bits, c.group_size), t, hbm_peak)
         del qws, qw
         torch.cuda.empty_cache()
+    return out
+
+
+def secondary_moe_prefill(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    """MoE prefill (128 experts, top-8): device routing, then the expert-grouped
+    GEMMs gate [768 x 2048] (token rows) and down [2048 x 768] (pair rows)"""
+    out = {}
+    E, dff, dm, k = 128, 768, 2048, 8
+    g = api.ExpertStack.from_qweight(
+        api.qmm_quantize(wl.gen_weight(E * dff, dm, 4600).to(dev), 64, 4, torch.bfloat16), E)
+    d = api.ExpertStack.from_qweight(
+        api.qmm_quantize(wl.gen_weight(E * dm, dff, 4601).to(dev), 64, 4, torch.bfloat16), E)
+    for T in (256, 2048):
+        P = T * k
+        ids = wl.gen_moe_ids(T, E, k, 4602 + T).to(dev)
+        a = wl.gen_x(T, dm, 4603 + T).to(dev)
+        h = wl.gen_x(P, dff, 4604 + T).to(dev)
+        ws = api.moe_workspace(P, E, dev)
+        og = torch.empty(P, dff, dtype=torch.bfloat16, device=dev)
+        od = torch.empty(P, dm, dtype=torch.bfloat16, device=dev)
+        t_r = time_graph(torch, lambda: api.qmm_moe_compute_ids_tpe(ids, E, ws, stream=stream), stream,
+                         reps=10, inner=5)
+        t_g = time_graph(torch, lambda: api.qmm_moe_gemm_id(a, T, k, 1, ws, g, out=og, stream=stream),
+                         stream, reps=10, inner=3)
+        t_d = time_graph(torch, lambda: api.qmm_moe_gemm_id(h, T, k, k, ws, d, out=od, stream=stream),
+                         stream, reps=10, inner=3)
+        for name, t, n in (("gate", t_g, dff), ("down", t_d, dm)):
+            kk = dm if name == "gate" else dff
+            tf = 2 * P * n * kk / (t * 1e-3) / 1e12
+            out[f"moe_prefill_t{T}_{name}"] = {"TFLOP/s": round(tf, 1),
+                                               "frac_of_measured_burst": round(tf / bf16_peak, 3),
+                                               "frac_of_datasheet_2250": round(tf / BF16_DATASHEET_TFLOPS, 3),
+                                               "us": round(t * 1e3, 2)}
+        out[f"moe_prefill_t{T}_routing"] = {"us": round(t_r * 1e3, 2), "pairs": P}
     return out
 
 
