@@ -76,6 +76,16 @@ def bind(path: str) -> ctypes.CDLL:
     L.orc_words_per_row.restype = i64
     L.orc_pack_row.argtypes = [vp, i64, c_int, vp]
     L.orc_pack_row.restype = None
+    L.orc_fp4_e2m1.argtypes = [ctypes.c_uint32]
+    L.orc_fp4_e2m1.restype = ctypes.c_float
+    L.orc_e8m0.argtypes = [ctypes.c_uint32]
+    L.orc_e8m0.restype = ctypes.c_float
+    L.orc_fp8_e4m3.argtypes = [ctypes.c_uint32]
+    L.orc_fp8_e4m3.restype = ctypes.c_float
+    L.orc_dequantize_mx.argtypes = [vp, vp, c_int, i64, i64, vp, c_int, i64, i64]
+    L.orc_dequantize_mx.restype = c_int
+    L.orc_matmul_mx.argtypes = [vp, c_int, i64, i64, vp, vp, c_int, i64, vp, i64, i64]
+    L.orc_matmul_mx.restype = c_int
     L.orc_code_integral.argtypes = [vp, c_int, i64]
     L.orc_code_integral.restype = ctypes.c_uint32
     L.orc_code_u64.argtypes = [vp, i64, c_int, i64]
@@ -381,3 +391,55 @@ def moe_batched_dense(a, a_dtype, ids, m, top_k, outer, inner, st: Stack, n_thre
         rows = a[offs[:, None] + np.arange(K)[None, :]]
         out[sel] = rows @ w.T
     return out, rc
+
+
+# ---------------------------------------------------------------- microscaled modes
+MODE_AFFINE, MODE_MXFP4, MODE_MXFP8, MODE_NVFP4 = 0, 1, 2, 3
+MX_PARAMS = {MODE_MXFP4: (4, 32), MODE_MXFP8: (8, 32), MODE_NVFP4: (4, 16)}  # (bits, group size)
+
+
+def fp4_e2m1(code: int) -> float:
+    return float(lib().orc_fp4_e2m1(int(code)))
+
+
+def e8m0(s: int) -> float:
+    return float(lib().orc_e8m0(int(s)))
+
+
+def fp8_e4m3(b: int) -> float:
+    return float(lib().orc_fp8_e4m3(int(b)))
+
+
+def dequantize_mx(packed, scales, mode: int, cols: int, out_dtype: int, n_threads=None) -> np.ndarray:
+    """w_hat = lane(q) * scale(s) of a microscaled matrix: packed [rows,
+    cols*bits/32] u32, scales [rows, cols/gs] u8 (no biases)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows = packed.shape[0]
+    out = np.zeros((rows, cols), dtype=_NP_STORAGE[out_dtype])
+    L = lib()
+
+    def fn(a, b):
+        return L.orc_dequantize_mx(_ptr(packed), _ptr(scales), mode, rows, cols, _ptr(out), out_dtype,
+                                   a, b)
+    rc = _run(fn, 0, rows, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle dequantize_mx rejected the arguments (rc={rc})")
+    return out
+
+
+def matmul_mx(x, x_dtype: int, packed, scales, mode: int, N: int, n_threads=None) -> np.ndarray:
+    """fp64 y[M, N] = x . dequant_mx(W)^T (W is [N, K] quantized along K)."""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    packed = np.ascontiguousarray(packed, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    y = np.zeros((M, N), dtype=np.float64)
+    L = lib()
+
+    def fn(a, b):
+        return L.orc_matmul_mx(_ptr(x), x_dtype, M, K, _ptr(packed), _ptr(scales), mode, N, _ptr(y), a, b)
+    rc = _run(fn, 0, N, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle matmul_mx rejected the arguments (rc={rc})")
+    return y

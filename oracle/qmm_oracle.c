@@ -470,3 +470,94 @@ int orc_moe_gate_up_silu_batched(const void* a, int a_dtype, const int32_t* ids,
   }
   return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* microscaled modes ([emily] dequantize_mxfp4_impl, dequantize_mxfp8_impl, */
+/* dequantize_nvfp4_impl, fp4_lut, e8m0_lut, fp8_e4m3_lut; group sizes:      */
+/* [emily] "one per group of 32 lanes" for mxfp4/mxfp8, [ollama]             */
+/* quantizeParams {16, 4, "nvfp4"}, {32, 8, "mxfp8"})                        */
+/* ------------------------------------------------------------------------ */
+
+enum { ORC_MODE_AFFINE = 0, ORC_MODE_MXFP4 = 1, ORC_MODE_MXFP8 = 2, ORC_MODE_NVFP4 = 3 };
+
+/* FP4-E2M1 lane: bit 3 sign, bits 2..1 exponent (bias 1), bit 0 mantissa;
+ * exponent 0 is the subnormal 0.5 * m, otherwise 2^(e-1) * (1 + m/2). */
+float orc_fp4_e2m1(uint32_t c) {
+  int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  float mag = e == 0 ? 0.5f * (float)m : ldexpf(1.0f + 0.5f * (float)m, e - 1);
+  return s ? -mag : mag;
+}
+
+/* FP8-E8M0 scale byte: 2^(s - 127) (s = 255 overflows fp32 to +inf) */
+float orc_e8m0(uint32_t s) { return ldexpf(1.0f, (int)(s & 0xff) - 127); }
+
+/* FP8-E4M3 byte as the page decodes it: the low 7 bits shifted left by 7
+ * read as a binary16, times 256, then the sign of bit 7 (so 0x7F and 0xFF
+ * are +-480 rather than NaN). */
+float orc_fp8_e4m3(uint32_t b) {
+  float mag = orc_f16_to_f32((uint16_t)((b & 0x7f) << 7)) * 256.0f;
+  return (b & 0x80) ? -mag : mag;
+}
+
+/* bits and group size of a microscaled mode (0 for any other mode) */
+int orc_mx_params(int mode, int* bits, int* gs) {
+  switch (mode) {
+    case ORC_MODE_MXFP4: *bits = 4; *gs = 32; return 1;
+    case ORC_MODE_MXFP8: *bits = 8; *gs = 32; return 1;
+    case ORC_MODE_NVFP4: *bits = 4; *gs = 16; return 1;
+    default: return 0;
+  }
+}
+
+static float mx_lane(int mode, uint32_t code) {
+  return mode == ORC_MODE_MXFP8 ? orc_fp8_e4m3(code) : orc_fp4_e2m1(code);
+}
+
+static float mx_scale(int mode, uint8_t sbyte) {
+  return mode == ORC_MODE_NVFP4 ? orc_fp8_e4m3(sbyte) : orc_e8m0(sbyte);
+}
+
+/* w_hat[r][i] = lane(q) * scale(s[r][i / gs]): one fp32 product (the page
+ * multiplies the two table values in bf16; both tables' values and their
+ * products are exact in bf16 for the scales the quantizers emit, so the fp32
+ * product is the same number).  No bias. */
+static float dequant_mx_one(const uint32_t* row, const uint8_t* scales, int mode, int bits, int gs,
+                            int64_t r, int64_t G, int64_t i) {
+  uint32_t q = orc_code_integral(row, bits, i);
+  return mx_lane(mode, q) * mx_scale(mode, scales[r * G + i / gs]);
+}
+
+int orc_dequantize_mx(const uint32_t* packed, const uint8_t* scales, int mode, int64_t rows,
+                      int64_t cols, void* out, int out_dtype, int64_t r0, int64_t r1) {
+  int bits, gs;
+  if (!orc_mx_params(mode, &bits, &gs) || rows < 0 || cols <= 0 || cols % gs) return ORC_ERR_ARG;
+  int64_t wpr = orc_words_per_row(cols, bits);
+  int64_t G = cols / gs;
+  for (int64_t r = r0; r < r1; ++r)
+    for (int64_t i = 0; i < cols; ++i)
+      store_f(out, out_dtype, r * cols + i,
+              dequant_mx_one(packed + r * wpr, scales, mode, bits, gs, r, G, i));
+  return ORC_OK;
+}
+
+/* y[m][n] = sum_k x[m][k] * w_hat[n][k] (W is [N, K] quantized along K), in
+ * fp64 with k increasing.  Output columns [n0, n1) only. */
+int orc_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const uint32_t* packed,
+                  const uint8_t* scales, int mode, int64_t N, double* y, int64_t n0, int64_t n1) {
+  int bits, gs;
+  if (!orc_mx_params(mode, &bits, &gs) || M < 0 || K <= 0 || N <= 0 || K % gs) return ORC_ERR_ARG;
+  int64_t wpr = orc_words_per_row(K, bits);
+  int64_t G = K / gs;
+  float* wcol = (float*)malloc(sizeof(float) * (size_t)K);
+  if (!wcol) return ORC_ERR_ARG;
+  for (int64_t n = n0; n < n1; ++n) {
+    for (int64_t k = 0; k < K; ++k) wcol[k] = dequant_mx_one(packed + n * wpr, scales, mode, bits, gs, n, G, k);
+    for (int64_t m = 0; m < M; ++m) {
+      double sum = 0.0;
+      for (int64_t kk = 0; kk < K; ++kk) sum += (double)load_f(x, x_dtype, m * K + kk) * (double)wcol[kk];
+      y[m * N + n] = sum;
+    }
+  }
+  free(wcol);
+  return ORC_OK;
+}

@@ -141,6 +141,33 @@ MUTANTS = [
      "  for (int64_t k = 0; k < K; ++k) {\n    float wv = transpose",
      "  for (int64_t k = 1; k < K; ++k) {\n    float wv = transpose",
      [P(pins.test_matmul_brute_force_exact, bits=4, transpose=True)]),
+    # microscaled modes
+    ("E2M1 sign bit ignored",
+     "  return s ? -mag : mag;\n}\n\n/* FP8-E8M0", "  return mag;\n}\n\n/* FP8-E8M0",
+     [P(pins.test_fp4_e2m1_matches_the_printed_table)]),
+    ("E2M1 exponent bias 0",
+     "ldexpf(1.0f + 0.5f * (float)m, e - 1)", "ldexpf(1.0f + 0.5f * (float)m, e)",
+     [P(pins.test_fp4_e2m1_matches_the_printed_table)]),
+    ("E8M0 bias 128",
+     "ldexpf(1.0f, (int)(s & 0xff) - 127)", "ldexpf(1.0f, (int)(s & 0xff) - 128)",
+     [P(pins.test_e8m0_is_two_to_the_byte_minus_127)]),
+    ("E4M3 exponent shifted by 8",
+     "(uint16_t)((b & 0x7f) << 7)", "(uint16_t)((b & 0x7f) << 8)",
+     [P(pins.test_fp8_e4m3_matches_the_format_and_the_page)]),
+    ("nvfp4 scales read as E8M0",
+     "return mode == ORC_MODE_NVFP4 ? orc_fp8_e4m3(sbyte) : orc_e8m0(sbyte);",
+     "return orc_e8m0(sbyte);",
+     [P(pins.test_dequant_mx_exact_rational, mode=oracle.MODE_NVFP4)]),
+    ("mxfp8 lanes decoded as E2M1",
+     "return mode == ORC_MODE_MXFP8 ? orc_fp8_e4m3(code) : orc_fp4_e2m1(code);",
+     "return orc_fp4_e2m1(code & 15);",
+     [P(pins.test_dequant_mx_exact_rational, mode=oracle.MODE_MXFP8)]),
+    ("nvfp4 group of 32",
+     "case ORC_MODE_NVFP4: *bits = 4; *gs = 16; return 1;", "case ORC_MODE_NVFP4: *bits = 4; *gs = 32; return 1;",
+     [P(pins.test_dequant_mx_exact_rational, mode=oracle.MODE_NVFP4)]),
+    ("microscaled matmul drops the last term",
+     "for (int64_t kk = 0; kk < K; ++kk) sum +=", "for (int64_t kk = 0; kk + 1 < K; ++kk) sum +=",
+     [P(pins.test_matmul_mx_brute_force, mode=oracle.MODE_MXFP4)]),
 ]
 
 

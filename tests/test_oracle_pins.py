@@ -529,3 +529,79 @@ def test_moe_batched_dense_agrees_with_the_loops(outer_inner):
     if inner:
         bad, _ = oracle.moe_batched_dense(a, oracle.BF16, ids, m, top_k, inner, outer, st)
         assert not np.allclose(bad, ref, rtol=0, atol=1e-6)
+
+
+# ------------------------------------------------------------------ microscaled modes
+def test_fp4_e2m1_matches_the_printed_table():
+    tab = GOLDEN["fp4_e2m1_table"]["value"]
+    got = [oracle.fp4_e2m1(c) for c in range(16)]
+    assert got == tab
+    assert [math.copysign(1.0, v) for v in got] == [math.copysign(1.0, v) for v in tab]  # -0.0 kept
+
+
+def test_e8m0_is_two_to_the_byte_minus_127():
+    bias = GOLDEN["e8m0_rule"]["bias"]
+    for s in range(256):
+        exp = math.ldexp(1.0, s - bias)
+        got = oracle.e8m0(s)
+        assert (got == exp) if exp < 3.4e38 else math.isinf(got)
+
+
+def test_fp8_e4m3_matches_the_format_and_the_page():
+    """every finite OCP E4M3 byte decodes as torch's float8_e4m3fn does; the
+    two bytes that format calls NaN decode to +-480 as the page states"""
+    b = torch.arange(256, dtype=torch.uint8)
+    ref = b.view(torch.float8_e4m3fn).to(torch.float32).tolist()
+    sat = GOLDEN["fp8_e4m3_saturation"]
+    for i in range(256):
+        got = oracle.fp8_e4m3(i)
+        if i in (0x7F, 0xFF):
+            assert got == sat[f"0x{i:02x}"]
+        else:
+            assert got == ref[i] and math.copysign(1.0, got) == math.copysign(1.0, ref[i])
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_MXFP4, oracle.MODE_MXFP8, oracle.MODE_NVFP4])
+def test_dequant_mx_exact_rational(mode):
+    """w_hat = lane(q) * scale(s) exactly (the products are exact in fp32),
+    lanes read LSB-first, one scale per group of the mode's group size"""
+    preset = GOLDEN["microscaled_presets"][{1: "mxfp4", 2: "mxfp8", 3: "nvfp4"}[mode]]
+    bits, gs = oracle.MX_PARAMS[mode]
+    assert (bits, gs) == (preset["bits"], preset["group_size"])
+    rows, cols = 5, 4 * gs
+    rng = np.random.default_rng(11 + mode)
+    codes = rng.integers(0, 1 << bits, (rows, cols), dtype=np.uint8)
+    if mode == oracle.MODE_MXFP8:
+        codes[codes == 0x7F] = 0x7E  # keep the saturation bytes out of the exactness check
+    if mode == oracle.MODE_NVFP4:
+        sc = rng.integers(0, 0x7E, (rows, cols // gs), dtype=np.uint8)  # positive E4M3 scales
+    else:
+        sc = rng.integers(100, 150, (rows, cols // gs), dtype=np.uint8)
+    packed = np.stack([oracle.pack_row(r, bits) for r in codes])
+    out = oracle.dequantize_mx(packed, sc, mode, cols, oracle.F32)
+    lane = (lambda c: oracle.fp8_e4m3(c)) if mode == oracle.MODE_MXFP8 else (lambda c: oracle.fp4_e2m1(c))
+    scl = (lambda s: oracle.fp8_e4m3(s)) if mode == oracle.MODE_NVFP4 else (lambda s: oracle.e8m0(s))
+    for r in range(rows):
+        for i in range(cols):
+            exp = Fraction(lane(int(codes[r, i]))) * Fraction(scl(int(sc[r, i // gs])))
+            assert Fraction(float(out[r, i])) == exp
+
+
+@pytest.mark.parametrize("mode", [oracle.MODE_MXFP4, oracle.MODE_MXFP8, oracle.MODE_NVFP4])
+def test_matmul_mx_brute_force(mode):
+    bits, gs = oracle.MX_PARAMS[mode]
+    N, K, M = 6, 2 * gs, 3
+    rng = np.random.default_rng(21 + mode)
+    codes = rng.integers(0, 1 << bits, (N, K), dtype=np.uint8)
+    sc = rng.integers(110, 130, (N, K // gs), dtype=np.uint8) if mode != oracle.MODE_NVFP4 else \
+        rng.integers(0x20, 0x50, (N, K // gs), dtype=np.uint8)
+    packed = np.stack([oracle.pack_row(r, bits) for r in codes])
+    x = wl.storage_numpy(wl.gen_x(M, K, 22))
+    y = oracle.matmul_mx(x, oracle.BF16, packed, sc, mode, N)
+    wd = oracle.dequantize_mx(packed, sc, mode, K, oracle.F32).astype(np.float64)
+    xs = oracle.widen_f64(x, oracle.BF16)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xs[m, k])) * Fraction(float(wd[n, k])) for k in range(K))
+            bound = K * 2.0 ** -52 * float(np.abs(xs[m]) @ np.abs(wd[n]))
+            assert abs(float(exact) - y[m, n]) <= bound
