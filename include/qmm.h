@@ -82,10 +82,26 @@ typedef enum {
   QMM_ERR_BAD_EXPERT_ID = 7  /* (device) an id outside [0, num_experts) */
 } qmm_status;
 
-typedef enum { QMM_F32 = 0, QMM_F16 = 1, QMM_BF16 = 2 } qmm_dtype;
+/* QMM_U8 is only the storage of the microscaled modes' scale bytes. */
+typedef enum { QMM_F32 = 0, QMM_F16 = 1, QMM_BF16 = 2, QMM_U8 = 3 } qmm_dtype;
 
-/* Only affine is implemented; the microscaled modes named on the emily page
- * (mxfp4, mxfp8, nvfp4) are rejected with QMM_ERR_UNSUPPORTED. */
+/* Quantization modes ("emily 0.5.1 lib/emily/quantization.ex", the modes of
+ * dequantize_defn/1, with the group sizes of "ollama
+ * x/create/client/quantize.go" quantizeParams):
+ *   AFFINE: b-bit codes, w = q * scale + bias per group (scales/biases in the
+ *           activation dtype);
+ *   MXFP4:  bits 4, group 32: FP4-E2M1 lanes times an FP8-E8M0 scale byte
+ *           (2^(s - 127));
+ *   MXFP8:  bits 8, group 32: FP8-E4M3 lanes times an E8M0 scale byte;
+ *   NVFP4:  bits 4, group 16: FP4-E2M1 lanes times an FP8-E4M3 scale byte.
+ * The E4M3 decode is the page's: the low 7 bits shifted left by 7 read as a
+ * binary16, times 256, sign from bit 7 (0x7F and 0xFF read as +-480, not
+ * NaN).  A microscaled qmm_qweight has sdtype QMM_U8, scales [rows,
+ * cols/group_size] uint8, biases unused (may be NULL), and bits/group_size
+ * equal to the mode's (QMM_ERR_INVALID_ARG otherwise); w_hat = lane * scale
+ * in fp32.  The microscaled modes are served by qmm_dequantize and
+ * qmm_matmul (transpose = 1, any float x); qmm_quantize and the MoE calls
+ * are affine only (the pages print no quantizer for these modes). */
 typedef enum {
   QMM_MODE_AFFINE = 0,
   QMM_MODE_MXFP4 = 1,

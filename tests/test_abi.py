@@ -37,7 +37,7 @@ def test_enum_values_match_header():
     for name, val in [("QMM_OK", 0), ("QMM_ERR_INVALID_ARG", 1), ("QMM_ERR_UNSUPPORTED", 2),
                       ("QMM_ERR_DTYPE", 3), ("QMM_ERR_ALIGNMENT", 4), ("QMM_ERR_CUDA", 5),
                       ("QMM_ERR_TIMEOUT", 6), ("QMM_ERR_BAD_EXPERT_ID", 7), ("QMM_F32", 0),
-                      ("QMM_F16", 1), ("QMM_BF16", 2)]:
+                      ("QMM_F16", 1), ("QMM_BF16", 2), ("QMM_U8", 3)]:
         assert re.search(rf"\b{name}\s*=\s*{val}\b", HEADER), name
         assert getattr(_lib, name) == val
 
@@ -70,7 +70,13 @@ def test_matmul_validation(L):
     assert matmul(L, qw(bits=5)) == _lib.QMM_ERR_INVALID_ARG
     assert matmul(L, qw(gs=48)) == _lib.QMM_ERR_INVALID_ARG
     assert matmul(L, qw(cols=96, gs=64)) == _lib.QMM_ERR_INVALID_ARG
-    assert matmul(L, qw(mode=_lib.QMM_MODE_NVFP4)) == _lib.QMM_ERR_UNSUPPORTED
+    assert matmul(L, qw(mode=7)) == _lib.QMM_ERR_UNSUPPORTED
+    # microscaled: scale bytes (QMM_U8), the mode's own bits and group size
+    assert matmul(L, qw(mode=_lib.QMM_MODE_NVFP4)) == _lib.QMM_ERR_DTYPE
+    assert matmul(L, qw(mode=_lib.QMM_MODE_NVFP4, sdtype=_lib.QMM_U8, bits=4, gs=32)) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(mode=_lib.QMM_MODE_MXFP8, sdtype=_lib.QMM_U8, bits=4, gs=32)) == _lib.QMM_ERR_INVALID_ARG
+    assert matmul(L, qw(mode=_lib.QMM_MODE_MXFP4, sdtype=_lib.QMM_U8, bits=4, gs=32),
+                  transpose=0) == _lib.QMM_ERR_UNSUPPORTED
     assert matmul(L, qw(), x_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
     assert matmul(L, qw(), y_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
     assert matmul(L, qw(), K=256) == _lib.QMM_ERR_INVALID_ARG

@@ -21,7 +21,7 @@ QMM_ERR_CUDA = 5
 QMM_ERR_TIMEOUT = 6
 QMM_ERR_BAD_EXPERT_ID = 7
 
-QMM_F32, QMM_F16, QMM_BF16 = 0, 1, 2
+QMM_F32, QMM_F16, QMM_BF16, QMM_U8 = 0, 1, 2, 3
 QMM_MODE_AFFINE, QMM_MODE_MXFP4, QMM_MODE_MXFP8, QMM_MODE_NVFP4 = 0, 1, 2, 3
 
 # every symbol include/qmm.h declares

@@ -13,9 +13,13 @@ from dataclasses import dataclass
 import torch
 
 from . import _lib
-from ._lib import QMM_BF16, QMM_F16, QMM_F32, QMM_MODE_AFFINE, ExpertStackC, QWeightC, check
+from ._lib import (QMM_BF16, QMM_F16, QMM_F32, QMM_MODE_AFFINE, QMM_MODE_MXFP4, QMM_MODE_MXFP8,
+                   QMM_MODE_NVFP4, QMM_U8, ExpertStackC, QWeightC, check)
 
-_TO_CODE = {torch.float32: QMM_F32, torch.float16: QMM_F16, torch.bfloat16: QMM_BF16}
+_TO_CODE = {torch.float32: QMM_F32, torch.float16: QMM_F16, torch.bfloat16: QMM_BF16,
+            torch.uint8: QMM_U8}
+# bits and group size of the microscaled modes
+MX_PARAMS = {QMM_MODE_MXFP4: (4, 32), QMM_MODE_MXFP8: (8, 32), QMM_MODE_NVFP4: (4, 16)}
 _FROM_CODE = {v: k for k, v in _TO_CODE.items()}
 
 
@@ -104,8 +108,17 @@ class QWeight:
 
     def validate(self) -> dict:
         """packed, scales and biases hold rows x (words | groups) elements;
-        returns them by name for the device check."""
+        returns them by name for the device check.  Microscaled modes: uint8
+        scales, no biases."""
         n = self.rows
+        if self.mode != QMM_MODE_AFFINE:
+            if self.mode not in MX_PARAMS or MX_PARAMS[self.mode] != (self.bits, self.group_size):
+                check("qmm", _lib.QMM_ERR_INVALID_ARG)
+            if self.cols % self.group_size or self.cols % 32:
+                check("qmm", _lib.QMM_ERR_INVALID_ARG)
+            _need(self.packed, "packed", n * self.cols * self.bits // 32, _PACKED)
+            _need(self.scales, "scales", n * (self.cols // self.group_size), (torch.uint8,))
+            return {"packed": self.packed, "scales": self.scales}
         _need(self.packed, "packed", n * _words(self.cols, self.bits), _PACKED)
         G = _groups(self.cols, self.group_size)
         _need(self.scales, "scales", n * G, _FLOAT)
@@ -116,6 +129,13 @@ class QWeight:
         return QWeightC(_ptr(self.packed), _ptr(self.scales), _ptr(self.biases),
                         dtype_code(self.scales.dtype), self.rows, self.cols, self.group_size,
                         self.bits, self.mode)
+
+
+def mx_qweight(packed: torch.Tensor, scales: torch.Tensor, mode: int, rows: int, cols: int) -> QWeight:
+    """A microscaled matrix (mxfp4 / mxfp8 / nvfp4): packed [rows,
+    cols*bits/32] int32 lanes, scales [rows, cols/group_size] uint8 bytes."""
+    bits, gs = MX_PARAMS[mode]
+    return QWeight(packed, scales, None, rows, cols, gs, bits, mode)
 
 
 @dataclass
@@ -147,7 +167,7 @@ class ExpertStack:
                             self.n_cols, self.group_size, self.bits)
 
     @staticmethod
-    def from_qweight(q: QWeight, num_experts: int) -> "ExpertStack":
+    def from_qweight(q: "QWeight", num_experts: int) -> "ExpertStack":
         assert q.rows % num_experts == 0
         return ExpertStack(q.packed, q.scales, q.biases, num_experts, q.rows // num_experts,
                            q.cols, q.group_size, q.bits)

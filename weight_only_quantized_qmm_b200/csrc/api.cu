@@ -16,6 +16,9 @@ cudaError_t launch_generic(const void* x, int x_dtype, int64_t M, int64_t K, con
                            int transpose, void* y, int y_dtype, cudaStream_t st);
 cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
                             void* y, int y_dtype, cudaStream_t st);
+cudaError_t launch_dequantize_mx(const qmm_qweight* w, void* out, int out_dtype, cudaStream_t st);
+cudaError_t launch_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
+                             int y_dtype, cudaStream_t st);
 }  // namespace qmm
 
 #include "qgemv.cuh"
@@ -51,9 +54,27 @@ static int64_t batched_pairs(int64_t m, int64_t top_k) {
   return (m > 0 && top_k > kMaxMoePairs / m) ? kMaxMoePairs + 1 : m * top_k;
 }
 
+// bits and group size of a microscaled mode (false for any other mode)
+static bool mx_params(int mode, int* bits, int* gs) {
+  switch (mode) {
+    case QMM_MODE_MXFP4: *bits = 4; *gs = 32; return true;
+    case QMM_MODE_MXFP8: *bits = 8; *gs = 32; return true;
+    case QMM_MODE_NVFP4: *bits = 4; *gs = 16; return true;
+    default: return false;
+  }
+}
+
 static qmm_status check_qweight(const qmm_qweight* w) {
   if (!w) return QMM_ERR_INVALID_ARG;
-  if (w->mode != QMM_MODE_AFFINE) return QMM_ERR_UNSUPPORTED;
+  if (w->mode != QMM_MODE_AFFINE) {
+    int bits = 0, gs = 0;
+    if (!mx_params(w->mode, &bits, &gs)) return QMM_ERR_UNSUPPORTED;
+    if (w->sdtype != QMM_U8) return QMM_ERR_DTYPE;
+    if (w->bits != bits || w->group_size != gs || w->rows < 0 || w->cols <= 0 || w->cols % 32 != 0)
+      return QMM_ERR_INVALID_ARG;
+    if (!aligned16(w->packed) || !aligned16(w->scales)) return QMM_ERR_ALIGNMENT;
+    return QMM_OK;
+  }
   if (!dtype_ok(w->sdtype)) return QMM_ERR_DTYPE;
   if (w->rows < 0 || !packable(w->cols, w->group_size, w->bits)) return QMM_ERR_INVALID_ARG;
   if (!aligned16(w->packed) || !aligned16(w->scales) || !aligned16(w->biases)) return QMM_ERR_ALIGNMENT;
@@ -137,6 +158,8 @@ qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, 
   if (!aligned16(out)) return QMM_ERR_ALIGNMENT;
   s = device_check();
   if (s != QMM_OK) return s;
+  if (w->mode != QMM_MODE_AFFINE)
+    return launch_status(qmm::launch_dequantize_mx(w, out, out_dtype, (cudaStream_t)stream));
   return launch_status(qmm::launch_dequantize(w, out, out_dtype, (cudaStream_t)stream));
 }
 
@@ -147,8 +170,10 @@ qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
   if (s != QMM_OK) return s;
   if (transpose != 0 && transpose != 1) return QMM_ERR_INVALID_ARG;
   if (!dtype_ok(x_dtype) || !dtype_ok(y_dtype)) return QMM_ERR_DTYPE;
-  if (x_dtype != w->sdtype) return QMM_ERR_DTYPE;
+  // affine: x and the scales share a dtype; microscaled: any float x
+  if (w->mode == QMM_MODE_AFFINE && x_dtype != w->sdtype) return QMM_ERR_DTYPE;
   if (y_dtype != x_dtype && y_dtype != QMM_F32) return QMM_ERR_DTYPE;
+  if (w->mode != QMM_MODE_AFFINE && !transpose) return QMM_ERR_UNSUPPORTED;
   if (M < 0 || K <= 0) return QMM_ERR_INVALID_ARG;
   const int64_t N = transpose ? w->rows : w->cols;
   if ((transpose ? w->cols : w->rows) != K) return QMM_ERR_INVALID_ARG;
@@ -157,6 +182,7 @@ qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
   s = device_check();
   if (s != QMM_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
+  if (w->mode != QMM_MODE_AFFINE) return launch_status(qmm::launch_matmul_mx(x, x_dtype, M, K, w, y, y_dtype, st));
   const bool half_types = (x_dtype == QMM_BF16 || x_dtype == QMM_F16);
   if (transpose && half_types && M <= 16) {
     qmm::QgemvParams p = qmm::make_dense_params(x, M, K, w, y, y_dtype);
