@@ -31,16 +31,40 @@ namespace gemm {
 constexpr int kBM = 128;                 // weight rows per CTA (UMMA M)
 constexpr int kBN = 256;                 // tokens per CTA (UMMA N)
 constexpr int kBK = 64;                  // k per stage: one 128-byte swizzle row of 16-bit values
-constexpr int kStages = 4;
 constexpr int kThreads = 320;            // 10 warps
 constexpr int kXStage = kBN * kBK * 2;   // 32 KB
 constexpr int kAStage = kBM * kBK * 2;   // 16 KB
-constexpr int kTileBytes = kStages * (kXStage + kAStage);
-constexpr int kSmem = 1024 + kTileBytes + 256;  // + alignment slack + barriers (17 used)
+constexpr int kSBChunk = kBM * 8 * 2;    // 8 groups of scales (or biases) of 128 rows: 2 KB
 constexpr uint32_t kSpins = 1u << 22;
+
+// Shared-memory plan of one instantiation.  TW: the packed codes (per stage,
+// [128 rows x 64 codes]) and the scales/biases (per chunk of 8 groups) arrive
+// by TMA; otherwise the dequant warps read them from global memory.
+template <int B, bool TW>
+struct Plan {
+  static constexpr int STAGES = TW ? 3 : 4;
+  static constexpr int CODE_STAGE = TW ? kBM * 2 * B * 4 : 0;  // 64 codes = 2B words per row
+  static constexpr int X0 = 0;
+  static constexpr int A0 = STAGES * kXStage;
+  static constexpr int C0 = A0 + STAGES * kAStage;
+  static constexpr int SB0 = C0 + STAGES * CODE_STAGE;          // [2 chunks][scales | biases]
+  static constexpr int BAR0 = SB0 + (TW ? 2 * 2 * kSBChunk : 0);
+  static constexpr int SMEM = 1024 + BAR0 + 256;                // + alignment slack, barriers
+  static_assert(SMEM <= 227 * 1024, "shared memory plan");
+};
 }  // namespace gemm
 
 // ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -234,21 +258,31 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, 
 //   warps 6..9  epilogue: tcgen05.ld of the finished accumulator, release it,
 //               store y directly from registers (per instruction, a warp
 //               writes 32 consecutive weight rows of one token)
-template <int B, int GS, typename T, bool MOE>
+template <int B, int GS, typename T, bool MOE, bool TW>
 __global__ void __launch_bounds__(gemm::kThreads, 1)
-qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
+qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmc,
+                const __grid_constant__ CUtensorMap tms, const __grid_constant__ CUtensorMap tmb) {
   using namespace gemm;
+  using PL = Plan<B, TW>;
+  constexpr int kStages = PL::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (su32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* xs = smem;                                 // [kStages][256 x 128 B]
-  uint8_t* as = smem + kStages * kXStage;             // [kStages][128 x 128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTileBytes);
+  uint8_t* xs = smem + PL::X0;                        // [kStages][256 x 128 B]
+  uint8_t* as = smem + PL::A0;                        // [kStages][128 x 128 B]
+  uint8_t* cs = smem + PL::C0;                        // [kStages][128 rows x 2B words] (TW)
+  uint8_t* sbs = smem + PL::SB0;                      // [2][scales 2 KB | biases 2 KB] (TW)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::BAR0);
   const uint32_t full0 = su32(bars), afull0 = full0 + 8 * kStages, empty0 = afull0 + 8 * kStages;
   const uint32_t accf0 = empty0 + 8 * kStages;      // [2] accumulator complete
   const uint32_t tfree0 = accf0 + 16;               // [2] accumulator read out by the epilogue
   const uint32_t drain = tfree0 + 16;               // every issued MMA complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 5);
+  const uint32_t sbfull0 = drain + 8;               // [2] scale/bias chunk landed (TW)
+  const uint32_t sbempty0 = sbfull0 + 16;           // [2] scale/bias chunk consumed (TW)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * kStages + 9);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  // stages per scale/bias chunk (8 groups): a chunk starts at k-stage i when
+  // i % SPC == 0 and ends at the chunk's last stage or the row's last stage
+  constexpr int SPC = (8 * GS) / kBK;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (p.K + kBK - 1) / kBK;
@@ -266,6 +300,10 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     mbar_init(tfree0, 4);
     mbar_init(tfree0 + 8, 4);
     mbar_init(drain, 1);
+    mbar_init(sbfull0, 1);
+    mbar_init(sbfull0 + 8, 1);
+    mbar_init(sbempty0, 4);
+    mbar_init(sbempty0 + 8, 4);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -287,10 +325,11 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     // dense: lane 0 loads each stage's [256 x 64] x tile; MoE: lane 0 posts
     // the stage's bytes and every lane gathers the activation rows of 8 token
     // slots (two 4-row gathers, one row per slot)
-    int j = 0, issued = 0;
+    int j = 0, issued = 0, cc = 0, cissued = 0;
     bool stop = false;
     for (int lt = 0; lt < my_tiles && !stop; ++lt) {
       const TileOf tl = tile_of<MOE>(p, lt, m_tiles, n_tiles);
+      const int wrow0 = tl.e * p.N + tl.n0;  // first row of the (stacked) weight matrix
       int rw[8];
       if constexpr (MOE) {
 #pragma unroll
@@ -299,30 +338,57 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
       for (int i = 0; i < nk; ++i, ++j) {
         const int s = j % kStages, u = j / kStages;
         bool ok = true;
+        if constexpr (TW) {
+          // a new chunk of 8 groups of scales/biases: its ring slot is free once
+          // the dequant warps released the chunk two before it
+          if (i % SPC == 0) {
+            const int cs_ = cc & 1;
+            if (lane == 0 && cc >= 2) ok = bar_wait(sbempty0 + 8 * cs_, ((cc >> 1) - 1) & 1, abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
+              if (lane == 0) *abort_flag = 1;
+              stop = true;
+              break;
+            }
+            if (lane == 0) {
+              const uint32_t sb = su32(sbs + cs_ * 2 * kSBChunk), bar = sbfull0 + 8 * cs_;
+              mbar_arrive_expect_tx(bar, 2 * kSBChunk);
+              tma_2d(sb, &tms, (i * kBK / GS) & ~7, wrow0, bar);
+              tma_2d(sb + kSBChunk, &tmb, (i * kBK / GS) & ~7, wrow0, bar);
+            }
+            cissued = ++cc;
+          }
+        }
         if (lane == 0 && j >= kStages) ok = bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag);
         if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) {
           if (lane == 0) *abort_flag = 1;
           stop = true;
           break;
         }
+        constexpr uint32_t kTx = kXStage + PL::CODE_STAGE;
         if constexpr (MOE) {
-          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
+          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, kTx);
           __syncwarp();
           const uint32_t d = su32(xs + s * kXStage) + (uint32_t)(lane * 8 * 128);
           tma_gather4(d, &tmx, i * kBK, rw[0], rw[1], rw[2], rw[3], full0 + 8 * s);
           tma_gather4(d + 512, &tmx, i * kBK, rw[4], rw[5], rw[6], rw[7], full0 + 8 * s);
         } else if (lane == 0) {
-          mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
+          mbar_arrive_expect_tx(full0 + 8 * s, kTx);
           tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, tl.m0, full0 + 8 * s);
+        }
+        if constexpr (TW) {
+          if (lane == 0) tma_2d(su32(cs + s * PL::CODE_STAGE), &tmc, i * 2 * B, wrow0, full0 + 8 * s);
         }
         issued = j + 1;
       }
     }
     // no copy may still be landing when the CTA exits: the last copy of every
     // slot is waited for with the full bound, also after an abort
-    if (lane == 0)
+    if (lane == 0) {
       for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
         mbar_wait_n(full0 + 8 * (i % kStages), (uint32_t)(i / kStages) & 1u, gemm::kSpins);
+      for (int c = cissued > 2 ? cissued - 2 : 0; c < cissued; ++c)
+        mbar_wait_n(sbfull0 + 8 * (c & 1), (uint32_t)(c >> 1) & 1u, gemm::kSpins);
+    }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
@@ -366,88 +432,133 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx) {
     constexpr bool kF32Path = (B == 8) && !std::is_same<T, __half>::value;
     const int total = my_tiles * nk;
 
-    // codes and scales/biases are prefetched kAhead stages ahead into a register
-    // ring (compile-time indices: the stage loop is unrolled by kAhead); stage j
-    // is k-stage j % nk of the CTA's tile j / nk
-    constexpr int kAhead = 3;
-    uint32_t rw[kAhead][2 * B];
-    T rs[kAhead][NGS], rb[kAhead][NGS];
-    auto load = [&](int j, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
-      const bool in = j < total;
-      const int lt = in ? j / nk : 0, i = in ? j - lt * nk : 0;
-      const TileOf tl = tile_of<MOE>(p, in ? lt : 0, m_tiles, n_tiles);
-      const int n = tl.n0 + r;
-      const bool nval = in && n < p.N;
-      // row of the (stacked) weight matrix: expert e's rows start at e * N
-      const int64_t wr = nval ? (int64_t)tl.e * p.N + n : 0;
-      const uint32_t* row = p.packed + wr * p.wpr;
-      const T* srow = reinterpret_cast<const T*>(p.scales) + wr * p.G;
-      const T* brow = reinterpret_cast<const T*>(p.biases) + wr * p.G;
-      const int k0 = i * kBK;
-      load_codes<B>(row, k0 * B / 32, p.wpr, nval, w);
-#pragma unroll
-      for (int jj = 0; jj < NGS; ++jj) {
-        const int gidx = (k0 + jj * GS) / GS;
-        const bool ok = nval && gidx < p.G;
-        sv[jj] = ok ? srow[gidx] : from_f32<T>(0.0f);
-        bv[jj] = ok ? brow[gidx] : from_f32<T>(0.0f);
+    // w_hat of this thread's row for stage s (64 codes cw, the stage's NGS
+    // scales/biases) written into the stage's A tile, then handed to the MMA
+    auto emit = [&](int s, const uint32_t (&cw)[2 * B], const T (&cs_)[NGS], const T (&cb_)[NGS]) {
+      uint32_t pr[32];
+      float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
+      if constexpr (kF32Path) {
+        sf0 = to_f32(cs_[0]); bf0 = to_f32(cb_[0]);
+        sf1 = to_f32(cs_[NGS - 1]); bf1 = to_f32(cb_[NGS - 1]);
+      } else {
+        codes_to_pairs<B, T>(cw, pr);
       }
-    };
+      const uint32_t s2a = (uint32_t)bits16(cs_[0]) * 0x00010001u;
+      const uint32_t b2a = (uint32_t)bits16(cb_[0]) * 0x00010001u;
+      const uint32_t s2b = (uint32_t)bits16(cs_[NGS - 1]) * 0x00010001u;
+      const uint32_t b2b = (uint32_t)bits16(cb_[NGS - 1]) * 0x00010001u;
+      uint8_t* arow = as + s * kAStage + r * 128;
 #pragma unroll
-    for (int a = 0; a < kAhead; ++a) load(a, rw[a], rs[a], rb[a]);
-    for (int j0 = 0; j0 < total; j0 += kAhead) {
+      for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = pairs 4c..4c+3 = codes 8c..8c+7
+        uint4 v;
+        uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-      for (int a = 0; a < kAhead; ++a) {
-        const int j = j0 + a;
-        if (j >= total) break;
-        const int s = j % kStages, u = j / kStages;
-        uint32_t cw[2 * B];
-        T cs[NGS], cb[NGS];
-#pragma unroll
-        for (int q = 0; q < 2 * B; ++q) cw[q] = rw[a][q];
-#pragma unroll
-        for (int q = 0; q < NGS; ++q) { cs[q] = rs[a][q]; cb[q] = rb[a][q]; }
-        load(j + kAhead, rw[a], rs[a], rb[a]);  // refill this ring slot kAhead stages ahead
-        // the A buffer of this stage is free once the MMAs of stage j - kStages are done
-        if (u > 0 && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) *abort_flag = 1;
-        uint32_t pr[32];
-        float sf0 = 0.f, bf0 = 0.f, sf1 = 0.f, bf1 = 0.f;
-        if constexpr (kF32Path) {
-          sf0 = to_f32(cs[0]); bf0 = to_f32(cb[0]);
-          sf1 = to_f32(cs[NGS - 1]); bf1 = to_f32(cb[NGS - 1]);
-        } else {
-          codes_to_pairs<B, T>(cw, pr);
-        }
-        const uint32_t s2a = (uint32_t)bits16(cs[0]) * 0x00010001u;
-        const uint32_t b2a = (uint32_t)bits16(cb[0]) * 0x00010001u;
-        const uint32_t s2b = (uint32_t)bits16(cs[NGS - 1]) * 0x00010001u;
-        const uint32_t b2b = (uint32_t)bits16(cb[NGS - 1]) * 0x00010001u;
-        uint8_t* arow = as + s * kAStage + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {  // 16-byte chunk c = pairs 4c..4c+3 = codes 8c..8c+7
-          uint4 v;
-          uint32_t* vv = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int pi = 4 * c + e;
-            const bool second = NGS > 1 && (2 * pi) >= GS;
-            if constexpr (kF32Path) {
-              // 8-bit codes do not fit the bf16 magic: q exact in fp32, fmaf, one bf16 rounding
-              const float q0 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi)) - 8388608.0f;
-              const float q1 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi + 1)) - 8388608.0f;
-              const float sv = second ? sf1 : sf0, bv = second ? bf1 : bf0;
-              const __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(q0, sv, bv), fmaf(q1, sv, bv));
-              vv[e] = *reinterpret_cast<const uint32_t*>(&h);
-            } else {
-              const uint32_t qv = h2_sub<T>(pr[pi], OFF2);  // exact q
-              vv[e] = h2_fma<T>(qv, second ? s2b : s2a, second ? b2b : b2a);
-            }
+        for (int e = 0; e < 4; ++e) {
+          const int pi = 4 * c + e;
+          const bool second = NGS > 1 && (2 * pi) >= GS;
+          if constexpr (kF32Path) {
+            // 8-bit codes do not fit the bf16 magic: q exact in fp32, fmaf, one bf16 rounding
+            const float q0 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi)) - 8388608.0f;
+            const float q1 = __uint_as_float(0x4B000000u | stream_code<B>(cw, 2 * pi + 1)) - 8388608.0f;
+            const float sv = second ? sf1 : sf0, bv = second ? bf1 : bf0;
+            const __nv_bfloat162 h = __floats2bfloat162_rn(fmaf(q0, sv, bv), fmaf(q1, sv, bv));
+            vv[e] = *reinterpret_cast<const uint32_t*>(&h);
+          } else {
+            const uint32_t qv = h2_sub<T>(pr[pi], OFF2);  // exact q
+            vv[e] = h2_fma<T>(qv, second ? s2b : s2a, second ? b2b : b2a);
           }
-          *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = v;
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
-        __syncwarp();
-        if (lane == 0) mbar_arrive(afull0 + 8 * s);
+        *reinterpret_cast<uint4*>(arow + ((c ^ (r & 7)) << 4)) = v;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(afull0 + 8 * s);
+    };
+
+    if constexpr (TW) {
+      // codes and scales/biases were staged by TMA: stage j is k-stage j % nk
+      // of the CTA's tile j / nk; its codes landed with the stage's x tile
+      int cc = 0;  // scale/bias chunks entered
+      for (int j = 0; j < total; ++j) {
+        const int lt = j / nk, i = j - lt * nk;
+        const int s = j % kStages, u = j / kStages;
+        if (i % SPC == 0) {
+          if (!bar_wait(sbfull0 + 8 * (cc & 1), (uint32_t)(cc >> 1) & 1u, abort_flag)) *abort_flag = 1;
+          ++cc;
+        }
+        const int slot = (cc - 1) & 1;
+        if (!bar_wait(full0 + 8 * s, u & 1, abort_flag)) *abort_flag = 1;
+        // (the A buffer of stage s is free: the producer waited for its MMAs
+        // before this stage's copies, whose landing the wait above saw)
+        uint32_t cw[2 * B];
+        const uint32_t crow = su32(cs + s * PL::CODE_STAGE) + (uint32_t)(r * 8 * B);
+#pragma unroll
+        for (int q = 0; q < B / 2; ++q) {
+          const uint4 v = lds128(crow + 16 * q);
+          cw[4 * q] = v.x; cw[4 * q + 1] = v.y; cw[4 * q + 2] = v.z; cw[4 * q + 3] = v.w;
+        }
+        T cs_[NGS], cb_[NGS];
+        const uint32_t srow = su32(sbs + slot * 2 * kSBChunk) + (uint32_t)(r * 16);
+#pragma unroll
+        for (int q = 0; q < NGS; ++q) {
+          const int gi = ((i * kBK) / GS + q) & 7;
+          const unsigned short sv = (unsigned short)lds16(srow + 2 * gi);
+          const unsigned short bv = (unsigned short)lds16(srow + kSBChunk + 2 * gi);
+          memcpy(&cs_[q], &sv, 2);
+          memcpy(&cb_[q], &bv, 2);
+        }
+        emit(s, cw, cs_, cb_);
+        if (i % SPC == SPC - 1 || i == nk - 1) {  // last stage of the chunk: release it
+          if (lane == 0) mbar_arrive(sbempty0 + 8 * slot);
+        }
+      }
+    } else {
+      // codes and scales/biases are prefetched kAhead stages ahead into a
+      // register ring (compile-time indices: the stage loop is unrolled by
+      // kAhead); stage j is k-stage j % nk of the CTA's tile j / nk
+      constexpr int kAhead = 3;
+      uint32_t rw[kAhead][2 * B];
+      T rs[kAhead][NGS], rb[kAhead][NGS];
+      auto load = [&](int j, uint32_t (&w)[2 * B], T (&sv)[NGS], T (&bv)[NGS]) {
+        const bool in = j < total;
+        const int lt = in ? j / nk : 0, i = in ? j - lt * nk : 0;
+        const TileOf tl = tile_of<MOE>(p, in ? lt : 0, m_tiles, n_tiles);
+        const int n = tl.n0 + r;
+        const bool nval = in && n < p.N;
+        // row of the (stacked) weight matrix: expert e's rows start at e * N
+        const int64_t wr = nval ? (int64_t)tl.e * p.N + n : 0;
+        const uint32_t* row = p.packed + wr * p.wpr;
+        const T* srow = reinterpret_cast<const T*>(p.scales) + wr * p.G;
+        const T* brow = reinterpret_cast<const T*>(p.biases) + wr * p.G;
+        const int k0 = i * kBK;
+        load_codes<B>(row, k0 * B / 32, p.wpr, nval, w);
+#pragma unroll
+        for (int jj = 0; jj < NGS; ++jj) {
+          const int gidx = (k0 + jj * GS) / GS;
+          const bool ok = nval && gidx < p.G;
+          sv[jj] = ok ? srow[gidx] : from_f32<T>(0.0f);
+          bv[jj] = ok ? brow[gidx] : from_f32<T>(0.0f);
+        }
+      };
+#pragma unroll
+      for (int a = 0; a < kAhead; ++a) load(a, rw[a], rs[a], rb[a]);
+      for (int j0 = 0; j0 < total; j0 += kAhead) {
+#pragma unroll
+        for (int a = 0; a < kAhead; ++a) {
+          const int j = j0 + a;
+          if (j >= total) break;
+          const int s = j % kStages, u = j / kStages;
+          uint32_t cw[2 * B];
+          T cs_[NGS], cb_[NGS];
+#pragma unroll
+          for (int q = 0; q < 2 * B; ++q) cw[q] = rw[a][q];
+#pragma unroll
+          for (int q = 0; q < NGS; ++q) { cs_[q] = rs[a][q]; cb_[q] = rb[a][q]; }
+          load(j + kAhead, rw[a], rs[a], rb[a]);  // refill this ring slot kAhead stages ahead
+          // the A buffer of this stage is free once the MMAs of stage j - kStages are done
+          if (u > 0 && !bar_wait(empty0 + 8 * s, (u - 1) & 1, abort_flag)) *abort_flag = 1;
+          emit(s, cw, cs_, cb_);
+        }
       }
     }
   } else {
@@ -521,38 +632,48 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn tensor_map_encoder();
 
-template <int B, int GS, typename T, bool MOE>
-static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap& tmx, int grid, cudaStream_t st) {
-  auto k = qgemm_tc_kernel<B, GS, T, MOE>;
+template <int B, int GS, typename T, bool MOE, bool TW>
+static cudaError_t launch_gemm_t(const GemmParams& prm, const CUtensorMap (&tm)[4], int grid, cudaStream_t st) {
+  auto k = qgemm_tc_kernel<B, GS, T, MOE, TW>;
+  constexpr int SMEM = gemm::Plan<B, TW>::SMEM;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gemm::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     configured[dev] = 1;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(gemm::kThreads);
-  cfg.dynamicSmemBytes = gemm::kSmem;
+  cfg.dynamicSmemBytes = SMEM;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, prm, tmx);
+  return cudaLaunchKernelEx(&cfg, k, prm, tm[0], tm[1], tm[2], tm[3]);
+}
+
+template <int B, int GS, typename T, bool MOE>
+static cudaError_t launch_gemm_w(bool tw, const GemmParams& prm, const CUtensorMap (&tm)[4], int grid,
+                                 cudaStream_t st) {
+  if constexpr (B != 3) {  // 64 3-bit codes are 24 bytes: not a TMA box width
+    if (tw) return launch_gemm_t<B, GS, T, MOE, true>(prm, tm, grid, st);
+  }
+  return launch_gemm_t<B, GS, T, MOE, false>(prm, tm, grid, st);
 }
 
 template <typename T, bool MOE>
-static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const CUtensorMap& tmx, int grid,
-                                 cudaStream_t st) {
-#define QMM_G(BB)                                                             \
-  if (gs == 32) return launch_gemm_t<BB, 32, T, MOE>(prm, tmx, grid, st);     \
-  if (gs == 64) return launch_gemm_t<BB, 64, T, MOE>(prm, tmx, grid, st);     \
-  return launch_gemm_t<BB, 128, T, MOE>(prm, tmx, grid, st);
+static cudaError_t launch_gemm_b(int bits, int gs, bool tw, const GemmParams& prm, const CUtensorMap (&tm)[4],
+                                 int grid, cudaStream_t st) {
+#define QMM_G(BB)                                                                  \
+  if (gs == 32) return launch_gemm_w<BB, 32, T, MOE>(tw, prm, tm, grid, st);       \
+  if (gs == 64) return launch_gemm_w<BB, 64, T, MOE>(tw, prm, tm, grid, st);       \
+  return launch_gemm_w<BB, 128, T, MOE>(tw, prm, tm, grid, st);
   switch (bits) {
     case 2: { QMM_G(2) }
     case 3: { QMM_G(3) }
@@ -561,6 +682,37 @@ static cudaError_t launch_gemm_b(int bits, int gs, const GemmParams& prm, const 
     default: { QMM_G(8) }
   }
 #undef QMM_G
+}
+
+// Maps of the weight side for the TMA-staged dequant: packed codes [rows, wpr]
+// u32 in [2 * bits words x 128 rows] boxes (one stage), scales and biases
+// [rows, G] 16-bit in [8 groups x 128 rows] boxes (one chunk).  False (the
+// caller reads the weights from global memory instead) when the rows are not
+// 16-byte strided or a stage's codes are not a whole number of 16 bytes.
+static bool make_w_maps(CUtensorMap* tc, CUtensorMap* ts, CUtensorMap* tb, const uint32_t* packed,
+                        const void* scales, const void* biases, int64_t rows, int64_t wpr, int64_t G, int bits) {
+  if (bits == 3 || wpr % 4 != 0 || G % 8 != 0) return false;
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t estr[2] = {1, 1};
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)wpr, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(wpr * 4)};
+    const cuuint32_t box[2] = {(cuuint32_t)(2 * bits), (cuuint32_t)gemm::kBM};
+    if (enc(tc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
+  const cuuint32_t box[2] = {8, (cuuint32_t)gemm::kBM};
+  for (int a = 0; a < 2; ++a)
+    if (enc(a ? tb : ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(a ? biases : scales), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  return true;
 }
 
 // 2-D map over x [rows, K] (16-bit): boxes of 64 k x box_rows rows, 128-byte swizzle
@@ -584,8 +736,11 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   if (M > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->rows > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
-  CUtensorMap tmx;
-  if (!make_x_map(&tmx, x, x_dtype, M, K, gemm::kBN)) return cudaErrorNotSupported;
+  CUtensorMap tm[4];
+  if (!make_x_map(&tm[0], x, x_dtype, M, K, gemm::kBN)) return cudaErrorNotSupported;
+  const bool tw = make_w_maps(&tm[1], &tm[2], &tm[3], w->packed, w->scales, w->biases, w->rows,
+                              K * w->bits / 32, K / w->group_size, w->bits);
+  if (!tw) tm[1] = tm[2] = tm[3] = tm[0];
   GemmParams prm{};
   prm.packed = w->packed;
   prm.scales = w->scales;
@@ -600,8 +755,8 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   // persistent: one CTA per SM (or per tile when there are fewer tiles)
   const int64_t tiles = ((prm.N + gemm::kBM - 1) / gemm::kBM) * (int64_t)((prm.M + gemm::kBN - 1) / gemm::kBN);
   const int grid = (int)std::min<int64_t>(tiles, qmm_host::num_sms());
-  if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, false>(w->bits, w->group_size, prm, tmx, grid, st);
-  return launch_gemm_b<__half, false>(w->bits, w->group_size, prm, tmx, grid, st);
+  if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, false>(w->bits, w->group_size, tw, prm, tm, grid, st);
+  return launch_gemm_b<__half, false>(w->bits, w->group_size, tw, prm, tm, grid, st);
 }
 
 // MoE prefill GEMM over the schedule that moe_route_kernel wrote into `ws`
@@ -614,8 +769,11 @@ cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const q
   if (a_rows > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->n_rows * w->num_experts > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
-  CUtensorMap tma;  // one-row boxes: the producer gathers 4 rows per copy
-  if (!make_x_map(&tma, a, a_dtype, a_rows, K, 1)) return cudaErrorNotSupported;
+  CUtensorMap tm[4];  // x: one-row boxes (the producer gathers 4 rows per copy)
+  if (!make_x_map(&tm[0], a, a_dtype, a_rows, K, 1)) return cudaErrorNotSupported;
+  const bool tw = make_w_maps(&tm[1], &tm[2], &tm[3], w->packed, w->scales, w->biases,
+                              w->n_rows * w->num_experts, K * w->bits / 32, K / w->group_size, w->bits);
+  if (!tw) tm[1] = tm[2] = tm[3] = tm[0];
   GemmParams prm{};
   prm.packed = w->packed;
   prm.scales = w->scales;
@@ -638,8 +796,8 @@ cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const q
   prm.n_pairs = n_pairs;
   // the work list is known only on the device: one CTA per SM
   const int grid = qmm_host::num_sms();
-  if (a_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, true>(w->bits, w->group_size, prm, tma, grid, st);
-  return launch_gemm_b<__half, true>(w->bits, w->group_size, prm, tma, grid, st);
+  if (a_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, true>(w->bits, w->group_size, tw, prm, tm, grid, st);
+  return launch_gemm_b<__half, true>(w->bits, w->group_size, tw, prm, tm, grid, st);
 }
 
 }  // namespace qmm
