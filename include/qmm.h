@@ -297,6 +297,29 @@ qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int6
                            const qmm_expert_stack* w, void* out, qmm_dtype out_dtype,
                            void* stream);
 
+/* Allocation-free MoE prefill GEMM: routing and GEMM of qmm_moe_compute_ids_tpe
+ * + qmm_moe_gemm_id in one call, with the routing schedule kept in a fixed
+ * scratch array inside this library instead of a caller workspace.  The pages
+ * have no counterpart; it serves callers that cannot provide device memory:
+ * an operator or plugin interface that hands the op only its inputs and
+ * outputs, or a latency-critical path where cudaMalloc (which may
+ * synchronize the device) is not allowed.
+ * Same arguments and results as the two calls (ids: device int32[batch *
+ * top_k]; out: [batch * top_k, w->n_rows]), the same errors, plus
+ * QMM_ERR_UNSUPPORTED when batch * top_k > 16384 or w->num_experts > 256 (the
+ * scratch's capacity).  The scratch (about 70 KB) is held by every GPU that
+ * loads the library until the process exits.  The first call on a device
+ * looks up the scratch's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  Every
+ * call shares the one scratch array of its device: calls that overlap on the
+ * GPU (on different streams, or in different threads) race and must be
+ * serialized by the caller.  Each call rewrites all of the scratch it reads.
+ * Allocates nothing. */
+qmm_status qmm_moe_gemm_id_noalloc(const void* a, qmm_dtype a_dtype, const int32_t* ids,
+                                   int64_t batch, int64_t top_k, int64_t ne11,
+                                   const qmm_expert_stack* w, void* out, qmm_dtype out_dtype,
+                                   int32_t* d_status, void* stream);
+
 /* Diagnostic of the bounded device-side waits (not a step of the method).
  * Every TMA-fed kernel here waits on shared-memory mbarriers with a poll
  * limit and reports QMM_ERR_TIMEOUT instead of hanging when a wait gives up.

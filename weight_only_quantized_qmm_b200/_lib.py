@@ -30,7 +30,8 @@ EXPORTS = (
     "qmm_quantize", "qmm_dequantize", "qmm_matmul", "qmm_moe_gemv_id",
     "qmm_moe_gemv_id_batched", "qmm_moe_gemv_id_gate_up_silu",
     "qmm_moe_gemv_id_gate_up_silu_batched", "qmm_moe_gemm_workspace_bytes",
-    "qmm_moe_compute_ids_tpe", "qmm_moe_gemm_id", "qmm_selftest_bounded_wait",
+    "qmm_moe_compute_ids_tpe", "qmm_moe_gemm_id", "qmm_moe_gemm_id_noalloc",
+    "qmm_selftest_bounded_wait",
 )
 
 
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
     L.qmm_moe_compute_ids_tpe.restype = c_int
     L.qmm_moe_gemm_id.argtypes = [vp, c_int, i64, i64, i64, vp, i64, stp, vp, c_int, vp]
     L.qmm_moe_gemm_id.restype = c_int
+    L.qmm_moe_gemm_id_noalloc.argtypes = [vp, c_int, vp, i64, i64, i64, stp, vp, c_int, vp, vp]
+    L.qmm_moe_gemm_id_noalloc.restype = c_int
     L.qmm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp, vp, vp]
     L.qmm_selftest_bounded_wait.restype = c_int
     _lib = L

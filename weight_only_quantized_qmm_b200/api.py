@@ -400,3 +400,27 @@ def qmm_moe_gemm_id(a: torch.Tensor, batch: int, top_k: int, ne11: int, workspac
                                      _ptr(out), dtype_code(out.dtype), _stream(stream))
     check("qmm_moe_gemm_id", rc)
     return out
+
+
+def qmm_moe_gemm_id_noalloc(a: torch.Tensor, ids: torch.Tensor, batch: int, top_k: int, ne11: int,
+                            w: ExpertStack, out_dtype: torch.dtype | None = None, out=None,
+                            d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Routing and MoE prefill GEMM in one call, without a workspace: the
+    schedule lives in the library's own fixed device scratch (at most 16384
+    pairs and 256 experts; calls that overlap on the GPU race)."""
+    n_pairs = batch * top_k
+    if out is None:
+        out = torch.empty(n_pairs, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
+    _need(a, "a", batch * ne11 * w.n_cols, _FLOAT)
+    named = w.validate()
+    _need(ids, "ids", n_pairs, (torch.int32,))
+    _need(out, "out", n_pairs * w.n_rows, _FLOAT)
+    if d_status is not None:
+        _need(d_status, "d_status", 1, (torch.int32,))
+    _on_device(a=a, ids=ids, out=out, d_status=d_status, **named)
+    c = w.c()
+    rc = _lib.load().qmm_moe_gemm_id_noalloc(_ptr(a), dtype_code(a.dtype), _ptr(ids), batch, top_k, ne11,
+                                             ctypes.byref(c), _ptr(out), dtype_code(out.dtype),
+                                             _ptr(d_status), _stream(stream))
+    check("qmm_moe_gemm_id_noalloc", rc)
+    return out

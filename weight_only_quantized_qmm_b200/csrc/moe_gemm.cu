@@ -41,17 +41,12 @@ constexpr int64_t kMaxRouteExperts = 8192;
 struct MoeWs {
   int64_t tpe, off, args, pairs, blk_e, blk_s, total;
 };
-inline MoeWs moe_ws_layout(int64_t n_pairs, int64_t E) {
-  MoeWs L;
+constexpr MoeWs moe_ws_layout(int64_t n_pairs, int64_t E) {
   const int64_t nb = (n_pairs + kMoeBlock - 1) / kMoeBlock + E;  // blocks, at most
-  L.tpe = 0;
-  L.off = E;
-  L.args = 2 * E + 1;
-  L.pairs = (2 * E + 4 + 3) / 4 * 4;
-  L.blk_e = L.pairs + (n_pairs + 3) / 4 * 4;
-  L.blk_s = L.blk_e + (nb + 3) / 4 * 4;
-  L.total = L.blk_s + (nb + 3) / 4 * 4;
-  return L;
+  const int64_t pairs = (2 * E + 4 + 3) / 4 * 4;
+  const int64_t blk_e = pairs + (n_pairs + 3) / 4 * 4;
+  const int64_t blk_s = blk_e + (nb + 3) / 4 * 4;
+  return MoeWs{0, E, 2 * E + 1, pairs, blk_e, blk_s, blk_s + (nb + 3) / 4 * 4};
 }
 
 // One CTA.  Shared memory: per-expert counts, running fill positions and
@@ -241,3 +236,75 @@ qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int6
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free form of the MoE prefill GEMM.  Some callers cannot hand
+// this library a workspace: an operator or plugin interface that gives the op
+// only its input and output tensors, or a latency-critical path on which
+// cudaMalloc (which may synchronize the device) is not allowed.  For them the
+// routing schedule lives in a fixed array in this library's own device
+// memory, sized for the largest call below; every GPU that loads the library
+// holds it (70 KB) until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNoAllocMaxPairs = 16384;   // batch * top_k
+constexpr int64_t kNoAllocMaxExperts = 256;
+constexpr int64_t kNoAllocWords = qmm::moe_ws_layout(kNoAllocMaxPairs, kNoAllocMaxExperts).total;
+
+// The scratch.  Host code must not pass this name to a kernel (on the host it
+// is only a stand-in for the device symbol): the device address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) int32_t g_moe_scratch[kNoAllocWords];
+
+// Device address of the scratch on the current device (looked up on the first
+// call per device, with that device current).
+qmm_status scratch_address(int32_t** out) {
+  static int32_t* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QMM_ERR_CUDA;
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_scratch) != cudaSuccess || p == nullptr) return QMM_ERR_CUDA;
+    cache[dev] = static_cast<int32_t*>(p);
+  }
+  *out = cache[dev];
+  return QMM_OK;
+}
+
+}  // namespace
+
+extern "C" qmm_status qmm_moe_gemm_id_noalloc(const void* a, qmm_dtype a_dtype, const int32_t* ids, int64_t batch,
+                                              int64_t top_k, int64_t ne11, const qmm_expert_stack* w, void* out,
+                                              qmm_dtype out_dtype, int32_t* d_status, void* stream) {
+  qmm_status s = check_moe_gemm_stack(w);
+  if (s != QMM_OK) return s;
+  if (!qmm_host::dtype_ok(a_dtype) || !qmm_host::dtype_ok(out_dtype)) return QMM_ERR_DTYPE;
+  if (a_dtype != w->sdtype) return QMM_ERR_DTYPE;
+  if (out_dtype != a_dtype && out_dtype != QMM_F32) return QMM_ERR_DTYPE;
+  if (!dtype_ok16(a_dtype)) return QMM_ERR_UNSUPPORTED;
+  if (batch < 0 || top_k < 1 || (ne11 != 1 && ne11 != top_k)) return QMM_ERR_INVALID_ARG;
+  // the built-in scratch serves at most kNoAllocMaxPairs pairs and
+  // kNoAllocMaxExperts experts
+  if (batch > kNoAllocMaxPairs / top_k || w->num_experts > kNoAllocMaxExperts) return QMM_ERR_UNSUPPORTED;
+  const int64_t n_pairs = batch * top_k;
+  if (n_pairs == 0) return QMM_OK;
+  if (!qmm_host::aligned16(a) || !qmm_host::aligned16(out) || !aligned4(ids)) return QMM_ERR_ALIGNMENT;
+  if (d_status && !aligned4(d_status)) return QMM_ERR_ALIGNMENT;
+  if ((w->n_cols * 2) % 16 != 0) return QMM_ERR_UNSUPPORTED;
+  s = qmm_device_check();
+  if (s != QMM_OK) return s;
+  int32_t* ws = nullptr;
+  s = scratch_address(&ws);
+  if (s != QMM_OK) return s;
+  // the routing step rewrites every field of the scratch that the GEMM reads
+  cudaStream_t st = (cudaStream_t)stream;
+  s = route(ids, n_pairs, w->num_experts, ws, kNoAllocWords * 4, d_status, st);
+  if (s != QMM_OK) return s;
+  const MoeWs L = qmm::moe_ws_layout(n_pairs, w->num_experts);
+  const cudaError_t e =
+      qmm::launch_qgemm_moe(a, a_dtype, batch * ne11, w, ws + L.off, ws + L.args, ws + L.pairs, ws + L.blk_e,
+                            ws + L.blk_s, (int)top_k, (int)ne11, (int)n_pairs, out, out_dtype, st);
+  if (e == cudaErrorNotSupported) return QMM_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
+}
