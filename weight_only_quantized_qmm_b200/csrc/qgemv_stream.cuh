@@ -646,11 +646,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) { xb[mt] = xs_sa; xbu[mt] = xs_sa; }
   uint32_t su = xrec_lane;
-  // one pair: this warp's x fragments and group sums of the current k-unit,
-  // in registers (reloaded only when the k-unit or the segment changes)
-  uint4 xr[C::ONE ? GPW : 1][L::kSteps / 2];
-  float4 xsr[C::ONE ? GPW : 1];
-  int xku = -1;
   Walk w;  // the work-list walk of MoE calls (a dense call is one segment)
   if constexpr (MOE) {
     if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
@@ -683,7 +678,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           xbu[mt] = xb[mt];
         }
         su = xrec_lane;
-        xku = -1;
       }
     }
     bool ok = mbar_try_wait(bfull, phase);
@@ -691,18 +685,6 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     if (__any_sync(0xffffffffu, !ok)) {
       if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
       failed = true;
-    }
-    if constexpr (C::ONE) {
-      if (ku != xku) {
-        xku = ku;
-#pragma unroll
-        for (int u = 0; u < GPW; ++u) {
-#pragma unroll
-          for (int q2 = 0; q2 < L::kSteps / 2; ++q2) xr[u][q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
-          const uint4 r = lds128(su + (uint32_t)(u * TOKP * 16));
-          xsr[u] = make_float4(__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z), 0.0f);
-        }
-      }
     }
     if (!failed) {
 #pragma unroll
@@ -758,9 +740,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
             rB[0] = lds32(ca + 1024);
           }
           float d[MT][4];
-          if constexpr (C::ONE)
-            group_dot_rx<L>(rA, rB, xr[u], d[0]);
-          else
+          if constexpr (C::ONE) {
+            // this group's x fragments (staged in the mma's k order); measured:
+            // reading them per group beats holding every group's in registers
+            uint4 bf[L::kSteps / 2];
+#pragma unroll
+            for (int q2 = 0; q2 < L::kSteps / 2; ++q2) bf[q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
+            group_dot_rx<L>(rA, rB, bf, d[0]);
+          } else
             group_dot1<L, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d);
           const int hw = u & 1;
           const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
@@ -770,7 +757,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           for (int mt = 0; mt < MT; ++mt) {
             float(&a_)[4] = acc[ns][mt];
             if constexpr (C::ONE) {
-              const float4 r = xsr[u];
+              const uint4 rq = lds128(su + (uint32_t)(u * TOKP * 16));
+              const float4 r = make_float4(__uint_as_float(rq.x), __uint_as_float(rq.y), __uint_as_float(rq.z), 0.0f);
               a_[0] = fmaf(ba, r.z, fmaf(sa, fmaf(d[0][0], r.x, r.y), a_[0]));
               a_[2] = fmaf(bb, r.z, fmaf(sb_, fmaf(d[0][2], r.x, r.y), a_[2]));
             } else {
