@@ -86,6 +86,12 @@ def bind(path: str) -> ctypes.CDLL:
     L.orc_dequantize_mx.restype = c_int
     L.orc_matmul_mx.argtypes = [vp, c_int, i64, i64, vp, vp, c_int, i64, vp, i64, i64]
     L.orc_matmul_mx.restype = c_int
+    L.orc_quantize_dynamic_int8.argtypes = [vp, c_int, i64, vp, vp]
+    L.orc_quantize_dynamic_int8.restype = c_int
+    L.orc_dequantize_dynamic_int8.argtypes = [vp, i64, vp, vp, c_int]
+    L.orc_dequantize_dynamic_int8.restype = c_int
+    L.orc_matmul_dynamic_int8.argtypes = [vp, c_int, i64, i64, vp, vp, i64, vp, i64, i64]
+    L.orc_matmul_dynamic_int8.restype = c_int
     L.orc_code_integral.argtypes = [vp, c_int, i64]
     L.orc_code_integral.restype = ctypes.c_uint32
     L.orc_code_u64.argtypes = [vp, i64, c_int, i64]
@@ -442,4 +448,45 @@ def matmul_mx(x, x_dtype: int, packed, scales, mode: int, N: int, n_threads=None
     rc = _run(fn, 0, N, n_threads)
     if rc != ORC_OK:
         raise ValueError(f"oracle matmul_mx rejected the arguments (rc={rc})")
+    return y
+
+
+# ---------------------------------------------------------------- per-tensor dynamic int8
+def quantize_dynamic_int8(w, w_dtype: int):
+    """whole-tensor min/max int8: (q int8 same shape, params float32[4] =
+    {input_min, input_max, output_min, output_max})"""
+    w = np.ascontiguousarray(w)
+    q = np.zeros(w.shape, dtype=np.int8)
+    params = np.zeros(4, dtype=np.float32)
+    rc = lib().orc_quantize_dynamic_int8(_ptr(w), w_dtype, w.size, _ptr(q), _ptr(params))
+    if rc != ORC_OK:
+        raise ValueError(f"oracle quantize_dynamic_int8 rejected the arguments (rc={rc})")
+    return q, params
+
+
+def dequantize_dynamic_int8(q, params, out_dtype: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    params = np.ascontiguousarray(params, dtype=np.float32)
+    out = np.zeros(q.shape, dtype=_NP_STORAGE[out_dtype])
+    rc = lib().orc_dequantize_dynamic_int8(_ptr(q), q.size, _ptr(params), _ptr(out), out_dtype)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle dequantize_dynamic_int8 rejected the arguments (rc={rc})")
+    return out
+
+
+def matmul_dynamic_int8(x, x_dtype: int, q, params, n_threads=None) -> np.ndarray:
+    """fp64 y[M, N] = x . w_hat^T for an int8 [N, K] weight"""
+    x = np.ascontiguousarray(x)
+    M, K = x.shape
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N = q.shape[0]
+    params = np.ascontiguousarray(params, dtype=np.float32)
+    y = np.zeros((M, N), dtype=np.float64)
+    L = lib()
+
+    def fn(a, b):
+        return L.orc_matmul_dynamic_int8(_ptr(x), x_dtype, M, K, _ptr(q), _ptr(params), N, _ptr(y), a, b)
+    rc = _run(fn, 0, N, n_threads)
+    if rc != ORC_OK:
+        raise ValueError(f"oracle matmul_dynamic_int8 rejected the arguments (rc={rc})")
     return y

@@ -16,7 +16,10 @@
  *   [mlex]   "mlex 0.1.3 src/quant.rs" -- quantize_dynamic_int8: min/max
  *            quantizer, scale floored at f32::EPSILON, round() = half away
  *            from zero.  Used here as the model for the per-group affine
- *            quantizer (whose own body is not printed on any page).
+ *            quantizer (whose own body is not printed on any page), and
+ *            written out itself (quantize_dynamic_int8,
+ *            dequantize_dynamic_int8 with DynamicRangeParams) for the
+ *            per-tensor int8 scheme.
  *   [ferrum] "ferrum-kernels 0.7.7 src/stacked_expert.rs" -- gemv_moe_id,
  *            gemv_moe_id_batched, gemv_moe_id_gate_up_silu(_batched).
  *
@@ -559,5 +562,69 @@ int orc_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const uint32
     }
   }
   free(wcol);
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* per-tensor dynamic-range int8 ([mlex] quantize_dynamic_int8,             */
+/* dequantize_dynamic_int8, DynamicRangeParams)                             */
+/* ------------------------------------------------------------------------ */
+
+/* params = {input_min, input_max, output_min, output_max} = {mn, mx, mn, mx}
+ * with mn, mx the whole tensor's min and max (fp32 compares);
+ * scale = max((mx - mn) / 255, FLT_EPSILON);
+ * q = clamp(round((w - mn) / scale) - 128, -128, 127), each of -, /, round
+ * (half away from zero), -128 in fp32. */
+int orc_quantize_dynamic_int8(const void* w, int w_dtype, int64_t n, int8_t* q, float* params) {
+  if (n <= 0) return ORC_ERR_ARG;
+  float mn = load_f(w, w_dtype, 0), mx = mn;
+  for (int64_t i = 1; i < n; ++i) {
+    float v = load_f(w, w_dtype, i);
+    if (v < mn) mn = v;
+    if (v > mx) mx = v;
+  }
+  float scale = (mx - mn) / 255.0f;
+  if (scale < FLT_EPSILON) scale = FLT_EPSILON;
+  for (int64_t i = 0; i < n; ++i) {
+    float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;
+    if (t < -128.0f) t = -128.0f;
+    if (t > 127.0f) t = 127.0f;
+    q[i] = (int8_t)t;
+  }
+  params[0] = mn;
+  params[1] = mx;
+  params[2] = mn;
+  params[3] = mx;
+  return ORC_OK;
+}
+
+/* w_hat = ((float)q + 128) * scale + output_min, scale = (output_max -
+ * output_min) / 255: the page's three fp32 operations in its order (the sum
+ * with 128 is exact; the product and the final sum round once each). */
+static float dyn8_one(int8_t q, const float* params) {
+  float scale = (params[3] - params[2]) / 255.0f;
+  float shifted = (float)q + 128.0f;
+  float scaled = shifted * scale;
+  return scaled + params[2];
+}
+
+int orc_dequantize_dynamic_int8(const int8_t* q, int64_t n, const float* params, void* out, int out_dtype) {
+  if (n < 0) return ORC_ERR_ARG;
+  for (int64_t i = 0; i < n; ++i) store_f(out, out_dtype, i, dyn8_one(q[i], params));
+  return ORC_OK;
+}
+
+/* y[m][n] = sum_k x[m][k] * w_hat[n][k] (W is [N, K] int8), fp64 sums with k
+ * increasing.  Output columns [n0, n1) only. */
+int orc_matmul_dynamic_int8(const void* x, int x_dtype, int64_t M, int64_t K, const int8_t* q,
+                            const float* params, int64_t N, double* y, int64_t n0, int64_t n1) {
+  if (M < 0 || K <= 0 || N <= 0) return ORC_ERR_ARG;
+  for (int64_t nn = n0; nn < n1; ++nn)
+    for (int64_t m = 0; m < M; ++m) {
+      double dot = 0.0;
+      for (int64_t k = 0; k < K; ++k)
+        dot += (double)load_f(x, x_dtype, m * K + k) * (double)dyn8_one(q[nn * K + k], params);
+      y[m * N + nn] = dot;
+    }
   return ORC_OK;
 }

@@ -168,6 +168,27 @@ MUTANTS = [
     ("microscaled matmul drops the last term",
      "for (int64_t kk = 0; kk < K; ++kk) sum +=", "for (int64_t kk = 0; kk + 1 < K; ++kk) sum +=",
      [P(pins.test_matmul_mx_brute_force, mode=oracle.MODE_MXFP4)]),
+    # per-tensor dynamic int8
+    ("dynamic int8 offset 127",
+     "float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;",
+     "float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 127.0f;",
+     [P(pins.test_dynamic_int8_page_round_trip)]),
+    ("dynamic int8 dequant adds the input minimum twice",
+     "return scaled + params[2];", "return scaled + 2.0f * params[2];",
+     [P(pins.test_dynamic_int8_dequant_exact_rational)]),
+    ("dynamic int8 divides by 256",
+     "float scale = (params[3] - params[2]) / 255.0f;", "float scale = (params[3] - params[2]) / 256.0f;",
+     [P(pins.test_dynamic_int8_dequant_exact_rational), P(pins.test_dynamic_int8_page_round_trip)]),
+    ("dynamic int8 without the epsilon floor",
+     "if (scale < FLT_EPSILON) scale = FLT_EPSILON;", "",
+     [P(pins.test_dynamic_int8_constant_tensor)]),
+    ("dynamic int8 codes truncated",
+     "float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;",
+     "float t = floorf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;",
+     [P(pins.test_dynamic_int8_codes_are_nearest)]),
+    ("dynamic int8 matmul reads the weight transposed",
+     "(double)dyn8_one(q[nn * K + k], params);", "(double)dyn8_one(q[k * N + nn], params);",
+     [P(pins.test_dynamic_int8_matmul_brute_force)]),
 ]
 
 

@@ -605,3 +605,75 @@ def test_matmul_mx_brute_force(mode):
             exact = sum(Fraction(float(xs[m, k])) * Fraction(float(wd[n, k])) for k in range(K))
             bound = K * 2.0 ** -52 * float(np.abs(xs[m]) @ np.abs(wd[n]))
             assert abs(float(exact) - y[m, n]) <= bound
+
+
+# ------------------------------------------------------------------ per-tensor dynamic int8
+def test_dynamic_int8_page_round_trip():
+    """the page's own fixture: every element comes back within one step + 1e-4"""
+    g = GOLDEN["dynamic_int8_round_trip"]
+    w = np.array(g["weights"], dtype=np.float32)
+    q, params = oracle.quantize_dynamic_int8(w, oracle.F32)
+    assert params.tolist() == [w.min(), w.max(), w.min(), w.max()]
+    back = oracle.dequantize_dynamic_int8(q, params, oracle.F32)
+    tol = (params[3] - params[2]) / g["divisor"] + g["extra_tol"]
+    assert np.all(np.abs(back.astype(np.float64) - w) <= tol)
+    lo, hi = g["code_range"]
+    assert q.min() == lo and q.max() == hi  # the extremes land on the end codes
+
+
+def test_dynamic_int8_dequant_exact_rational():
+    """w_hat = fl(fl(fl(q + 128) * scale) + min), scale = fl((max - min) / 255):
+    each fp32 operation rounded once, checked with exact rationals"""
+    rng = np.random.default_rng(5)
+    q = rng.integers(-128, 128, 300, dtype=np.int8)
+    for mn, mx in [(-0.37, 0.81), (-3.0, -1.0), (1e-3, 2e-3), (-1e4, 3e4)]:
+        params = np.array([mn, mx, mn, mx], dtype=np.float32)
+        out = oracle.dequantize_dynamic_int8(q, params, oracle.F32)
+        f32 = lambda fr: Fraction(float(np.float32(float(fr))))  # noqa: E731  round to nearest fp32
+        scale = f32(Fraction(float(params[3])) - Fraction(float(params[2])))
+        scale = f32(scale / 255)
+        for i in range(q.size):
+            sh = Fraction(int(q[i]) + 128)
+            exp = f32(f32(sh * scale) + Fraction(float(params[2])))
+            assert Fraction(float(out[i])) == exp
+
+
+def test_dynamic_int8_codes_are_nearest():
+    """each code is the nearest point of the affine 256-point grid (brute force
+    over all 256 codes, ties allowed either way within the fp32 rounding)"""
+    rng = np.random.default_rng(6)
+    w = (rng.standard_normal(513) * 0.7).astype(np.float32)
+    q, params = oracle.quantize_dynamic_int8(w, oracle.F32)
+    mn = float(params[0])
+    scale = float(np.float32((np.float32(params[1]) - np.float32(params[0])) / np.float32(255)))
+    grid = np.arange(256, dtype=np.float64) * scale + mn
+    for i in range(w.size):
+        d = np.abs(grid - float(w[i]))
+        best = d.min()
+        assert d[int(q[i]) + 128] <= best + 1e-6 * scale
+
+
+def test_dynamic_int8_constant_tensor():
+    """max == min: the scale floor FLT_EPSILON keeps it finite; all codes -128
+    and the dequantized tensor is the constant exactly"""
+    w = np.full(40, 0.625, dtype=np.float32)
+    q, params = oracle.quantize_dynamic_int8(w, oracle.F32)
+    assert np.all(q == -128)
+    back = oracle.dequantize_dynamic_int8(q, params, oracle.F32)
+    assert np.all(back == np.float32(0.625))
+
+
+def test_dynamic_int8_matmul_brute_force():
+    rng = np.random.default_rng(7)
+    N, K, M = 5, 96, 3
+    w = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)
+    q, params = oracle.quantize_dynamic_int8(w, oracle.F32)
+    x = wl.storage_numpy(wl.gen_x(M, K, 8))
+    y = oracle.matmul_dynamic_int8(x, oracle.BF16, q, params)
+    wd = oracle.dequantize_dynamic_int8(q, params, oracle.F32).astype(np.float64)
+    xs = oracle.widen_f64(x, oracle.BF16)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xs[m, k])) * Fraction(float(wd[n, k])) for k in range(K))
+            bound = K * 2.0 ** -52 * float(np.abs(xs[m]) @ np.abs(wd[n]))
+            assert abs(float(exact) - y[m, n]) <= bound
