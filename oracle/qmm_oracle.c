@@ -571,25 +571,28 @@ int orc_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const uint32
 /* ------------------------------------------------------------------------ */
 
 /* params = {input_min, input_max, output_min, output_max} = {mn, mx, mn, mx}
- * with mn, mx the whole tensor's min and max (fp32 compares);
+ * with mn, mx the whole tensor's min and max: a fold that starts at +inf
+ * (-inf) and takes fminf (fmaxf), which passes over NaN elements as the
+ * page's f32::min / f32::max do;
  * scale = max((mx - mn) / 255, FLT_EPSILON);
  * q = clamp(round((w - mn) / scale) - 128, -128, 127), each of -, /, round
- * (half away from zero), -128 in fp32. */
+ * (half away from zero), -128 in fp32; a NaN t becomes code 0 (the page's
+ * float-to-i8 cast). */
 int orc_quantize_dynamic_int8(const void* w, int w_dtype, int64_t n, int8_t* q, float* params) {
   if (n <= 0) return ORC_ERR_ARG;
-  float mn = load_f(w, w_dtype, 0), mx = mn;
-  for (int64_t i = 1; i < n; ++i) {
+  float mn = INFINITY, mx = -INFINITY;
+  for (int64_t i = 0; i < n; ++i) {
     float v = load_f(w, w_dtype, i);
-    if (v < mn) mn = v;
-    if (v > mx) mx = v;
+    mn = fminf(mn, v);
+    mx = fmaxf(mx, v);
   }
   float scale = (mx - mn) / 255.0f;
-  if (scale < FLT_EPSILON) scale = FLT_EPSILON;
+  if (!(scale >= FLT_EPSILON)) scale = FLT_EPSILON; /* f32::max: a NaN side loses */
   for (int64_t i = 0; i < n; ++i) {
     float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;
     if (t < -128.0f) t = -128.0f;
     if (t > 127.0f) t = 127.0f;
-    q[i] = (int8_t)t;
+    q[i] = isnan(t) ? (int8_t)0 : (int8_t)t;
   }
   params[0] = mn;
   params[1] = mx;

@@ -180,7 +180,7 @@ MUTANTS = [
      "float scale = (params[3] - params[2]) / 255.0f;", "float scale = (params[3] - params[2]) / 256.0f;",
      [P(pins.test_dynamic_int8_dequant_exact_rational), P(pins.test_dynamic_int8_page_round_trip)]),
     ("dynamic int8 without the epsilon floor",
-     "if (scale < FLT_EPSILON) scale = FLT_EPSILON;", "",
+     "if (!(scale >= FLT_EPSILON)) scale = FLT_EPSILON;", "",
      [P(pins.test_dynamic_int8_constant_tensor)]),
     ("dynamic int8 codes truncated",
      "float t = roundf((load_f(w, w_dtype, i) - mn) / scale) - 128.0f;",

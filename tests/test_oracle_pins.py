@@ -677,3 +677,15 @@ def test_dynamic_int8_matmul_brute_force():
             exact = sum(Fraction(float(xs[m, k])) * Fraction(float(wd[n, k])) for k in range(K))
             bound = K * 2.0 ** -52 * float(np.abs(xs[m]) @ np.abs(wd[n]))
             assert abs(float(exact) - y[m, n]) <= bound
+
+
+def test_dynamic_int8_nan_elements_follow_the_page_fold():
+    """NaN elements take no part in min/max (f32::min / f32::max skip NaN) and
+    quantize to code 0 (a NaN float cast to i8 is 0); the other codes are the
+    ones the tensor without them gets"""
+    w = np.array([0.5, np.nan, -1.0, 2.0, np.nan, 0.0], dtype=np.float32)
+    q, params = oracle.quantize_dynamic_int8(w, oracle.F32)
+    assert params.tolist() == [-1.0, 2.0, -1.0, 2.0]
+    assert q[1] == 0 and q[4] == 0
+    q2, _ = oracle.quantize_dynamic_int8(w[~np.isnan(w)], oracle.F32)
+    assert q[~np.isnan(w)].tolist() == q2.tolist()
