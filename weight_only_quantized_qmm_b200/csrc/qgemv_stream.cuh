@@ -71,9 +71,11 @@ struct Params {
 };
 
 // Layout of one thread's quarter of a group for the f16 lane arithmetic:
-// kCodes consecutive codes in kRegs packed words; each word yields kOPW f16
-// pairs, pair j holding codes j and j + kOPW of the word, both at bit offset
-// pos(j) inside their 16-bit half (a code at bit p reads as 1024 + q * 2^p).
+// kCodes codes in kRegs packed words, word k of quarter t being word
+// t + 4k of the group's row (so that one ldmatrix.x4 hands each thread its
+// words of rows g and g + 8); each word yields kOPW f16 pairs, pair j
+// holding codes j and j + kOPW of the word, both at bit offset pos(j) inside
+// their 16-bit half (a code at bit p reads as 1024 + q * 2^p).
 //   8-bit: pairs (0,2) (1,3), offset 0 (byte permutes, no mask);
 //   4-bit: pairs (0,4) (1,5) (2,6) (3,7), offsets 0, 4, 0, 4 (the last two
 //          from the word shifted right by 8);
@@ -99,7 +101,17 @@ struct Lanes {
   __host__ __device__ static constexpr int lo_code(int o) { return (o / kOPW) * kLPW + o % kOPW; }
   __host__ __device__ static constexpr int hi_code(int o) { return lo_code(o) + kOPW; }
   __host__ __device__ static constexpr int lo_pos(int o) { return pos(o % kOPW); }
+  // first code (within the group) of word k of quarter t
+  __host__ __device__ static constexpr int word_code(int t, int k) { return (t + 4 * k) * kLPW; }
 };
+
+// Four 8x8 16-bit matrices from shared memory in the mma fragment layout
+// (lanes 8m .. 8m + 7 give the row addresses of matrix m).
+__device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(a));
+}
 
 // MODE 0: one pair per segment; 1: up to 8; 2: up to 16.  UG: groups per unit
 // (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
@@ -340,14 +352,22 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     const int m = act ? gq / Gpad : 0, gl = act ? gq - m * Gpad : 0;
     __align__(16) T xv[L::kCodes];
     if (act && gl < q.G) {
-      const T* xa = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS + tt * L::kCodes;
-      if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
+      const T* xg = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS;
+      constexpr int WB = L::kLPW * (int)sizeof(T);  // bytes of x under one packed word
 #pragma unroll
-        for (int c = 0; c < L::kCodes * (int)sizeof(T) / 16; ++c)
-          reinterpret_cast<uint4*>(xv)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
-      } else {
+      for (int k = 0; k < L::kRegs; ++k) {
+        const T* xa = xg + L::word_code(tt, k);
+        T* dst = xv + k * L::kLPW;
+        if (WB % 16 == 0 && (reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
 #pragma unroll
-        for (int c = 0; c < L::kCodes; ++c) xv[c] = xa[c];
+          for (int c = 0; c < WB / 16; ++c)
+            reinterpret_cast<uint4*>(dst)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
+        } else if (WB == 8 && (reinterpret_cast<uintptr_t>(xa) & 7) == 0) {
+          *reinterpret_cast<uint2*>(dst) = __ldg(reinterpret_cast<const uint2*>(xa));
+        } else {
+#pragma unroll
+          for (int c = 0; c < L::kLPW; ++c) dst[c] = xa[c];
+        }
       }
     } else {
 #pragma unroll
@@ -604,20 +624,22 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   const uint32_t xs_sa = smem_u32(xs), xrec_sa = smem_u32(xrec);
   // per-group records of pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
   const uint32_t xrec_lane = xrec_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 16);
-  // shared offset (within a slot) of this lane's code words, row g, for group
-  // u: coff(u).  When a warp's groups share one 128-byte slice and the group
-  // step only touches chunk bits above the lane's own, coff(u) is coff(0) with
-  // those chunk bits flipped (no per-group register).
-  constexpr bool kXorGroups = (GPW * WPG <= 32) && (32 % (GPW * WPG) == 0) && (WPG % 4 == 0) &&
-                              (L::kRegs <= 4) && ((WPG / 4) & (4 * L::kRegs / 4 - 1)) == 0;
-  auto coff_of = [&](int u) -> uint32_t {
-    const int w0 = (warp * GPW + u) * WPG + t * L::kRegs;  // first word in the unit row
-    const int wb = w0 & 31;
-    return (uint32_t)((w0 >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
+  // Code words of group u.  kRegs == 1: the lane's word t of rows g and
+  // g + 8 (two 32-bit loads).  kRegs >= 2: ldmatrix.x4 per pair of words
+  // (t + 4k, t + 4k + 4): lane l gives the row address of matrix l / 8 =
+  // {row l%8, row l%8 + 8} x {chunk c, chunk c + 1}; the 128-byte swizzle puts
+  // chunk c of row r at c ^ (r & 7).
+  const int lr = lane & 7, lm = lane >> 3;
+  auto code_addr = [&](int u, int k2) -> uint32_t {
+    const int w0 = (warp * GPW + u) * WPG;  // first word of the group in the unit row
+    if constexpr (L::kRegs == 1) {
+      const int wb = (w0 + t) & 31;
+      return (uint32_t)(((w0 + t) >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
+    } else {
+      const int ch = ((w0 & 31) >> 2) + 2 * k2 + (lm >> 1);  // 16-byte chunk within the 128-byte row
+      return (uint32_t)((w0 >> 5) * 2048 + (lr + 8 * (lm & 1)) * 128 + ((ch ^ lr) << 4));
+    }
   };
-  uint32_t coff[kXorGroups ? 1 : GPW];
-#pragma unroll
-  for (int u = 0; u < (kXorGroups ? 1 : GPW); ++u) coff[u] = coff_of(u);
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
   // groups (row g's chunk c sits at chunk c ^ f(g); f is the same for row g + 8)
   // (SB1: plain [16][G] rows, pitch 2 G bytes)
@@ -722,22 +744,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         for (int u = 0; u < GPW; ++u) {
           if (SB1 && u >= live) break;  // warp-uniform
           uint32_t rA[L::kRegs], rB[L::kRegs];
-          const uint32_t ca = kXorGroups ? csl + (coff[0] ^ (uint32_t)((u * (WPG / 4)) << 4)) : csl + coff[kXorGroups ? 0 : u];
-          if constexpr (L::kRegs >= 4) {
-            const uint32_t cbase = ca & ~(uint32_t)127, c0 = (ca >> 4) & 7;  // row base, first chunk
-#pragma unroll
-            for (int k = 0; k < L::kRegs / 4; ++k) {
-              const uint32_t ch = (uint32_t)(((c0 ^ (uint32_t)g) + k) ^ (uint32_t)g);
-              const uint4 va = lds128(cbase + (ch << 4)), vb = lds128(cbase + 1024 + (ch << 4));
-              rA[4 * k] = va.x; rA[4 * k + 1] = va.y; rA[4 * k + 2] = va.z; rA[4 * k + 3] = va.w;
-              rB[4 * k] = vb.x; rB[4 * k + 1] = vb.y; rB[4 * k + 2] = vb.z; rB[4 * k + 3] = vb.w;
-            }
-          } else if constexpr (L::kRegs == 2) {
-            const uint2 va = lds64(ca), vb = lds64(ca + 1024);
-            rA[0] = va.x; rA[1] = va.y; rB[0] = vb.x; rB[1] = vb.y;
-          } else {
+          if constexpr (L::kRegs == 1) {
+            const uint32_t ca = csl + code_addr(u, 0);
             rA[0] = lds32(ca);
             rB[0] = lds32(ca + 1024);
+          } else {
+#pragma unroll
+            for (int k2 = 0; k2 < L::kRegs / 2; ++k2)
+              ldsm_x4(csl + code_addr(u, k2), rA[2 * k2], rB[2 * k2], rA[2 * k2 + 1], rB[2 * k2 + 1]);
           }
           float d[MT][4];
           if constexpr (C::ONE) {
