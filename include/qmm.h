@@ -1,6 +1,6 @@
 /*
  * qmm.h -- C ABI of libqmm.so: weight-only quantized matmul on NVIDIA B200
- * (sm_100a), affine mode.
+ * (sm_100a): affine, microscaled and per-tensor int8 weights.
  *
  * What is computed (sources cited by page title and section):
  *   - Packed weights: b-bit codes (b in {2,3,4,6,8}) stored LSB-first along
@@ -169,11 +169,12 @@ qmm_status qmm_quantize(const void* w, qmm_dtype w_dtype, int64_t rows, int64_t 
                         void* scales, void* biases, void* stream);
 
 /* Standalone dequantization ("emily 0.5.1 lib/emily/quantization.ex",
- * dequantize_defn/1): out[r][i] = fmaf(q, scale, bias), stored in out_dtype
- * with one RNE rounding for f16/bf16 and none for f32.  out: [w->rows,
- * w->cols] row-major.  Bit-exact.  w->rows == 0 is a no-op.
- * Errors: INVALID_ARG (shape rules, null w), UNSUPPORTED (mode other than
- * affine, or the device), DTYPE, ALIGNMENT, CUDA. */
+ * dequantize_defn/1): out[r][i] = fmaf(q, scale, bias) (affine) or
+ * lane(q) * scale (microscaled), stored in out_dtype with one RNE rounding
+ * for f16/bf16 and none for f32.  out: [w->rows, w->cols] row-major.
+ * Bit-exact.  w->rows == 0 is a no-op.
+ * Errors: INVALID_ARG (shape rules, null w), UNSUPPORTED (an unknown mode,
+ * or the device), DTYPE, ALIGNMENT, CUDA. */
 qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, void* stream);
 
 /* Quantized matmul ("emily 0.5.1 lib/emily/quantization.ex",
@@ -187,13 +188,70 @@ qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, 
  * row-major.  Accumulation is fp32.  M == 0 is a no-op.  bf16/f16 with
  * transpose = 1 use the tensor-core kernels (M <= 16: the streaming GEMV;
  * M > 16: the tcgen05 GEMM).
+ * Microscaled modes take any float x, transpose = 1 only.
  * Errors: INVALID_ARG (shape rules, K != the weight's input dimension,
- * transpose not 0/1, M < 0), UNSUPPORTED (mode other than affine, or a
- * device that is not compute capability 10.0), DTYPE (x_dtype !=
- * w->sdtype, or y_dtype neither x_dtype nor f32), ALIGNMENT, CUDA. */
+ * transpose not 0/1, M < 0), UNSUPPORTED (an unknown mode, a microscaled
+ * mode with transpose = 0, or a device that is not compute capability
+ * 10.0), DTYPE (affine x_dtype != w->sdtype, or y_dtype neither x_dtype nor
+ * f32), ALIGNMENT, CUDA. */
 qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
                       const qmm_qweight* w, int transpose, void* y, qmm_dtype y_dtype,
                       void* stream);
+
+/* Fused projection over parts that share the input dimension
+ * ("ferrum-quantization 0.7.2 src/quant_linear.rs", QuantLinear::
+ * from_gguf_fused: each part keeps its own storage and quantization
+ * parameters, and the forward pass is one matvec per part):
+ * y[:, off_p : off_p + N_p] = x . dequant(W_p)^T for p in [0, n_parts),
+ * N_p = parts[p].rows, off_p = N_0 + ... + N_{p-1}; y is [M, sum N_p]
+ * row-major.  Parts may differ in bits, group size and mode; each one
+ * follows qmm_matmul's rules with transpose = 1 and runs the kernel
+ * qmm_matmul picks for it, writing its columns of y in place (no
+ * concatenated copy of the weights or of the outputs).
+ * Errors: INVALID_ARG (parts NULL, n_parts outside [1, 64], or any part
+ * breaking qmm_matmul's rules), the other qmm_matmul errors per part.  All
+ * parts are checked before the first launch; a launch failure returns at
+ * once with the earlier parts already queued on the stream. */
+qmm_status qmm_matmul_parts(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
+                            const qmm_qweight* parts, int n_parts, void* y, qmm_dtype y_dtype,
+                            void* stream);
+
+/* Per-tensor dynamic-range int8 ("mlex 0.1.3 src/quant.rs",
+ * DynamicRangeParams, quantize_dynamic_int8, dequantize_dynamic_int8): one
+ * scale and zero point for a whole tensor.  params is a DEVICE float[4]
+ * {input_min, input_max, output_min, output_max} (4-byte aligned); the
+ * codes q are int8 in the tensor's own layout (a [N, K] weight is N*K codes,
+ * row-major).
+ *   w_hat = fl(fl(fl(q + 128) * scale) + output_min),
+ *   scale = fl((output_max - output_min) / 255)     (fp32, three roundings)
+ *
+ * qmm_quantize_dynamic_int8: params = {min, max, min, max} of the n elements
+ * of w (a fold from +-infinity that passes over NaN), then
+ * q = clamp(round_half_away((w - min) / s) - 128, -128, 127) with
+ * s = max((max - min) / 255, FLT_EPSILON), every step in fp32; a NaN
+ * element gets code 0.  Bit-exact.  Four kernels on `stream` (min/max
+ * reduction through params, codes, params).
+ * Errors: DTYPE (w_dtype), INVALID_ARG (n <= 0), ALIGNMENT (w, q 16-byte;
+ * params 4-byte), UNSUPPORTED (device), CUDA. */
+qmm_status qmm_quantize_dynamic_int8(const void* w, qmm_dtype w_dtype, int64_t n, int8_t* q,
+                                     float* params, void* stream);
+
+/* out[i] = w_hat(q[i]) stored in out_dtype (one RNE rounding for f16/bf16).
+ * Bit-exact.  n == 0 is a no-op.
+ * Errors: DTYPE, INVALID_ARG (n < 0), ALIGNMENT (q, out 16-byte; params
+ * 4-byte), UNSUPPORTED, CUDA. */
+qmm_status qmm_dequantize_dynamic_int8(const int8_t* q, int64_t n, const float* params, void* out,
+                                       qmm_dtype out_dtype, void* stream);
+
+/* y[M, N] = x[M, K] . w_hat^T for an int8 weight q [N, K] (row-major), any
+ * float x; y_dtype is x_dtype or QMM_F32.  fp32 accumulation, the row dot
+ * regrouped as scale * sum x (q + 128) + output_min * sum x.  M == 0 or
+ * N == 0 is a no-op.
+ * Errors: DTYPE, INVALID_ARG (M < 0, K <= 0, N < 0), ALIGNMENT (x, q, y
+ * 16-byte; params 4-byte), UNSUPPORTED, CUDA. */
+qmm_status qmm_matmul_dynamic_int8(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
+                                   const int8_t* q, int64_t N, const float* params, void* y,
+                                   qmm_dtype y_dtype, void* stream);
 
 /* MoE indirect GEMV ("ferrum-kernels 0.7.7 src/stacked_expert.rs",
  * gemv_moe_id):

@@ -219,3 +219,37 @@ def test_binding_refuses_host_tensors():
         api.qmm_matmul(torch.zeros(1, 64), qw)
     with pytest.raises(ValueError, match="CUDA"):
         api.qmm_dequantize(qw)
+
+
+def test_parts_validation(L):
+    arr = (_lib.QWeightC * 2)(qw(), qw(rows=16))
+    call = lambda parts, n, K=128, x_dtype=_lib.QMM_BF16, M=1, y=A: L.qmm_matmul_parts(  # noqa: E731
+        A, x_dtype, M, K, parts, n, y, _lib.QMM_BF16, None)
+    assert call(None, 2) == _lib.QMM_ERR_INVALID_ARG
+    assert call(arr, 0) == _lib.QMM_ERR_INVALID_ARG
+    assert call(arr, 65) == _lib.QMM_ERR_INVALID_ARG
+    assert call(arr, 2, K=256) == _lib.QMM_ERR_INVALID_ARG      # a part's input dimension differs
+    assert call(arr, 2, x_dtype=_lib.QMM_F16) == _lib.QMM_ERR_DTYPE
+    bad = (_lib.QWeightC * 2)(qw(), qw(bits=5))
+    assert call(bad, 2) == _lib.QMM_ERR_INVALID_ARG             # every part is checked first
+    assert call(arr, 2, M=0) == _lib.QMM_OK                     # nothing to do
+    assert call(arr, 2, y=A + 8) == _lib.QMM_ERR_ALIGNMENT
+
+
+def test_dynamic_int8_validation(L):
+    q = L.qmm_quantize_dynamic_int8
+    assert q(A, 9, 16, A, A, None) == _lib.QMM_ERR_DTYPE
+    assert q(A, _lib.QMM_F32, 0, A, A, None) == _lib.QMM_ERR_INVALID_ARG
+    assert q(A, _lib.QMM_F32, 16, A + 4, A, None) == _lib.QMM_ERR_ALIGNMENT
+    assert q(A, _lib.QMM_F32, 16, A, A + 2, None) == _lib.QMM_ERR_ALIGNMENT
+    d = L.qmm_dequantize_dynamic_int8
+    assert d(A, -1, A, A, _lib.QMM_F32, None) == _lib.QMM_ERR_INVALID_ARG
+    assert d(A, 0, A, A, _lib.QMM_F32, None) == _lib.QMM_OK
+    assert d(A, 16, A, A, 9, None) == _lib.QMM_ERR_DTYPE
+    assert d(A, 16, None, A, _lib.QMM_F32, None) == _lib.QMM_ERR_ALIGNMENT
+    m = L.qmm_matmul_dynamic_int8
+    assert m(A, _lib.QMM_BF16, 1, 64, A, 8, A, A, _lib.QMM_F16, None) == _lib.QMM_ERR_DTYPE
+    assert m(A, _lib.QMM_BF16, -1, 64, A, 8, A, A, _lib.QMM_BF16, None) == _lib.QMM_ERR_INVALID_ARG
+    assert m(A, _lib.QMM_BF16, 1, 0, A, 8, A, A, _lib.QMM_BF16, None) == _lib.QMM_ERR_INVALID_ARG
+    assert m(A, _lib.QMM_BF16, 0, 64, A, 8, A, A, _lib.QMM_BF16, None) == _lib.QMM_OK
+    assert m(A, _lib.QMM_BF16, 1, 64, A + 1, 8, A, A, _lib.QMM_BF16, None) == _lib.QMM_ERR_ALIGNMENT

@@ -31,7 +31,8 @@ EXPORTS = (
     "qmm_moe_gemv_id_batched", "qmm_moe_gemv_id_gate_up_silu",
     "qmm_moe_gemv_id_gate_up_silu_batched", "qmm_moe_gemm_workspace_bytes",
     "qmm_moe_compute_ids_tpe", "qmm_moe_gemm_id", "qmm_moe_gemm_id_noalloc",
-    "qmm_selftest_bounded_wait",
+    "qmm_selftest_bounded_wait", "qmm_matmul_parts", "qmm_quantize_dynamic_int8",
+    "qmm_dequantize_dynamic_int8", "qmm_matmul_dynamic_int8",
 )
 
 
@@ -101,6 +102,14 @@ def load() -> ctypes.CDLL:
     L.qmm_moe_gemm_id_noalloc.restype = c_int
     L.qmm_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp, vp, vp]
     L.qmm_selftest_bounded_wait.restype = c_int
+    L.qmm_matmul_parts.argtypes = [vp, c_int, i64, i64, qwp, c_int, vp, c_int, vp]
+    L.qmm_matmul_parts.restype = c_int
+    L.qmm_quantize_dynamic_int8.argtypes = [vp, c_int, i64, vp, vp, vp]
+    L.qmm_quantize_dynamic_int8.restype = c_int
+    L.qmm_dequantize_dynamic_int8.argtypes = [vp, i64, vp, vp, c_int, vp]
+    L.qmm_dequantize_dynamic_int8.restype = c_int
+    L.qmm_matmul_dynamic_int8.argtypes = [vp, c_int, i64, i64, vp, i64, vp, vp, c_int, vp]
+    L.qmm_matmul_dynamic_int8.restype = c_int
     _lib = L
     return L
 

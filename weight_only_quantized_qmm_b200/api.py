@@ -272,6 +272,88 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
     return out.reshape(*lead, N)
 
 
+def qmm_matmul_parts(x: torch.Tensor, parts, y_dtype: torch.dtype | None = None, out=None,
+                     stream=None) -> torch.Tensor:
+    """Fused projection: y[..., off_p : off_p + N_p] = x . dequant(W_p)^T for
+    the QWeights in `parts` (same input dimension, any bits / group size /
+    mode each); y is [..., sum N_p]."""
+    parts = list(parts)
+    if not parts:
+        check("qmm_matmul_parts", _lib.QMM_ERR_INVALID_ARG)
+    lead = x.shape[:-1]
+    K = x.shape[-1]
+    x2 = x.reshape(-1, K).contiguous()
+    M = x2.shape[0]
+    Ntot = sum(p.rows for p in parts)
+    _need(x2, "x", M * K, _FLOAT)
+    named = {}
+    for i, p in enumerate(parts):
+        named.update({f"part{i}.{k}": v for k, v in p.validate().items()})
+    if out is None:
+        out = torch.empty(M, Ntot, dtype=y_dtype or x.dtype, device=x2.device)
+    _need(out, "out", M * Ntot, _FLOAT)
+    if out.numel() != M * Ntot:
+        raise ValueError(f"qmm_matmul_parts: out holds {out.numel()} elements, expected {M}x{Ntot}")
+    _on_device(x=x2, out=out, **named)
+    arr = (QWeightC * len(parts))(*[p.c() for p in parts])
+    rc = _lib.load().qmm_matmul_parts(_ptr(x2), dtype_code(x2.dtype), M, K, arr, len(parts), _ptr(out),
+                                      dtype_code(out.dtype), _stream(stream))
+    check("qmm_matmul_parts", rc)
+    return out.reshape(*lead, Ntot)
+
+
+def qmm_quantize_dynamic_int8(w: torch.Tensor, stream=None):
+    """Whole-tensor min/max int8: (q int8 with w's shape, params float32[4] on
+    the device = {input_min, input_max, output_min, output_max})."""
+    w = w.contiguous()
+    _need(w, "w", w.numel(), _FLOAT)
+    _on_device(w=w)
+    q = torch.empty(w.shape, dtype=torch.int8, device=w.device)
+    params = torch.empty(4, dtype=torch.float32, device=w.device)
+    rc = _lib.load().qmm_quantize_dynamic_int8(_ptr(w), dtype_code(w.dtype), w.numel(), _ptr(q), _ptr(params),
+                                               _stream(stream))
+    check("qmm_quantize_dynamic_int8", rc)
+    return q, params
+
+
+def qmm_dequantize_dynamic_int8(q: torch.Tensor, params: torch.Tensor, out_dtype: torch.dtype = torch.float32,
+                                out=None, stream=None) -> torch.Tensor:
+    _need(q, "q", q.numel(), (torch.int8,))
+    _need(params, "params", 4, (torch.float32,))
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    _need(out, "out", q.numel(), _FLOAT)
+    _on_device(q=q, params=params, out=out)
+    rc = _lib.load().qmm_dequantize_dynamic_int8(_ptr(q), q.numel(), _ptr(params), _ptr(out),
+                                                 dtype_code(out.dtype), _stream(stream))
+    check("qmm_dequantize_dynamic_int8", rc)
+    return out
+
+
+def qmm_matmul_dynamic_int8(x: torch.Tensor, q: torch.Tensor, params: torch.Tensor,
+                            y_dtype: torch.dtype | None = None, out=None, stream=None) -> torch.Tensor:
+    """y = x . w_hat^T for an int8 [N, K] weight with per-tensor params; x [..., K]."""
+    if q.dim() != 2:
+        raise ValueError(f"qmm_matmul_dynamic_int8: q must be 2-D [N, K], got {tuple(q.shape)}")
+    N, K = q.shape
+    lead = x.shape[:-1]
+    if x.shape[-1] != K:
+        check("qmm_matmul_dynamic_int8", _lib.QMM_ERR_INVALID_ARG)
+    x2 = x.reshape(-1, K).contiguous()
+    M = x2.shape[0]
+    _need(x2, "x", M * K, _FLOAT)
+    _need(q, "q", N * K, (torch.int8,))
+    _need(params, "params", 4, (torch.float32,))
+    if out is None:
+        out = torch.empty(M, N, dtype=y_dtype or x.dtype, device=x2.device)
+    _need(out, "out", M * N, _FLOAT)
+    _on_device(x=x2, q=q, params=params, out=out)
+    rc = _lib.load().qmm_matmul_dynamic_int8(_ptr(x2), dtype_code(x2.dtype), M, K, _ptr(q), N, _ptr(params),
+                                             _ptr(out), dtype_code(out.dtype), _stream(stream))
+    check("qmm_matmul_dynamic_int8", rc)
+    return out.reshape(*lead, N)
+
+
 def _moe_checks(a, ids, n_pairs, top_k, outer, inner, stacks, out, n_out_rows, d_status):
     _need(a, "a", _last_pair_end(n_pairs, top_k, outer, inner, stacks[0].n_cols), _FLOAT)
     named = {}

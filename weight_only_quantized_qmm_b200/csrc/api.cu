@@ -13,12 +13,17 @@ cudaError_t launch_quantize(int w_dtype, int s_dtype, int bits, const void* w, i
                             cudaStream_t st);
 cudaError_t launch_dequantize(const qmm_qweight* w, void* out, int out_dtype, cudaStream_t st);
 cudaError_t launch_generic(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
-                           int transpose, void* y, int y_dtype, cudaStream_t st);
+                           int transpose, void* y, int64_t ldy, int y_dtype, cudaStream_t st);
 cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
-                            void* y, int y_dtype, cudaStream_t st);
+                            void* y, int64_t ldy, int y_dtype, cudaStream_t st);
 cudaError_t launch_dequantize_mx(const qmm_qweight* w, void* out, int out_dtype, cudaStream_t st);
 cudaError_t launch_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
-                             int y_dtype, cudaStream_t st);
+                             int64_t ldy, int y_dtype, cudaStream_t st);
+cudaError_t launch_quantize_dyn8(const void* w, int w_dtype, int64_t n, int8_t* q, float* params, cudaStream_t st);
+cudaError_t launch_dequantize_dyn8(const int8_t* q, int64_t n, const float* params, void* out, int out_dtype,
+                                   cudaStream_t st);
+cudaError_t launch_matmul_dyn8(const void* x, int x_dtype, int64_t M, int64_t K, const int8_t* q, int64_t N,
+                               const float* params, void* y, int y_dtype, cudaStream_t st);
 }  // namespace qmm
 
 #include "qgemv.cuh"
@@ -47,6 +52,8 @@ static bool aligned4(const void* p) { return p && ((reinterpret_cast<uintptr_t>(
 
 // Largest MoE call the kernels' per-CTA plans are sized for (pairs, experts).
 constexpr int64_t kMaxMoePairs = 65536;
+// Most parts of one fused projection.
+constexpr int kMaxParts = 64;
 
 // m * top_k pairs of a batched MoE call; a product above kMaxMoePairs is
 // reported as kMaxMoePairs + 1 (rejected as unsupported) without overflowing.
@@ -163,9 +170,9 @@ qmm_status qmm_dequantize(const qmm_qweight* w, void* out, qmm_dtype out_dtype, 
   return launch_status(qmm::launch_dequantize(w, out, out_dtype, (cudaStream_t)stream));
 }
 
-qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
-                      const qmm_qweight* w, int transpose, void* y, qmm_dtype y_dtype,
-                      void* stream) {
+// argument rules of qmm_matmul for one weight (no launch)
+static qmm_status check_matmul(qmm_dtype x_dtype, int64_t M, int64_t K, const qmm_qweight* w, int transpose,
+                               qmm_dtype y_dtype) {
   qmm_status s = check_qweight(w);
   if (s != QMM_OK) return s;
   if (transpose != 0 && transpose != 1) return QMM_ERR_INVALID_ARG;
@@ -175,26 +182,99 @@ qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
   if (y_dtype != x_dtype && y_dtype != QMM_F32) return QMM_ERR_DTYPE;
   if (w->mode != QMM_MODE_AFFINE && !transpose) return QMM_ERR_UNSUPPORTED;
   if (M < 0 || K <= 0) return QMM_ERR_INVALID_ARG;
-  const int64_t N = transpose ? w->rows : w->cols;
   if ((transpose ? w->cols : w->rows) != K) return QMM_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return QMM_OK;
-  if (!aligned16(x) || !aligned16(y)) return QMM_ERR_ALIGNMENT;
-  s = device_check();
-  if (s != QMM_OK) return s;
-  cudaStream_t st = (cudaStream_t)stream;
-  if (w->mode != QMM_MODE_AFFINE) return launch_status(qmm::launch_matmul_mx(x, x_dtype, M, K, w, y, y_dtype, st));
+  return QMM_OK;
+}
+
+// the kernel choice of qmm_matmul; y rows are ldy elements apart
+static qmm_status matmul_dispatch(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
+                                  int transpose, void* y, int64_t ldy, qmm_dtype y_dtype, cudaStream_t st) {
+  if (w->mode != QMM_MODE_AFFINE)
+    return launch_status(qmm::launch_matmul_mx(x, x_dtype, M, K, w, y, ldy, y_dtype, st));
   const bool half_types = (x_dtype == QMM_BF16 || x_dtype == QMM_F16);
   if (transpose && half_types && M <= 16) {
-    qmm::QgemvParams p = qmm::make_dense_params(x, M, K, w, y, y_dtype);
+    qmm::QgemvParams p = qmm::make_dense_params(x, M, K, w, y, ldy, y_dtype);
     const cudaError_t e = qmm::launch_qgemv(p, w->bits, w->group_size, x_dtype, false, st);
     if (e == cudaErrorInvalidValue) return QMM_ERR_UNSUPPORTED;
     return launch_status(e);
   }
   if (transpose && half_types) {  // M > 16: tcgen05 tensor-core GEMM
-    const cudaError_t e = qmm::launch_qgemm_tc(x, x_dtype, M, K, w, y, y_dtype, st);
+    const cudaError_t e = qmm::launch_qgemm_tc(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
     if (e != cudaErrorNotSupported) return launch_status(e);
   }
-  return launch_status(qmm::launch_generic(x, x_dtype, M, K, w, transpose, y, y_dtype, st));
+  return launch_status(qmm::launch_generic(x, x_dtype, M, K, w, transpose, y, ldy, y_dtype, st));
+}
+
+qmm_status qmm_matmul(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
+                      const qmm_qweight* w, int transpose, void* y, qmm_dtype y_dtype,
+                      void* stream) {
+  qmm_status s = check_matmul(x_dtype, M, K, w, transpose, y_dtype);
+  if (s != QMM_OK) return s;
+  const int64_t N = transpose ? w->rows : w->cols;
+  if (M == 0 || N == 0) return QMM_OK;
+  if (!aligned16(x) || !aligned16(y)) return QMM_ERR_ALIGNMENT;
+  s = device_check();
+  if (s != QMM_OK) return s;
+  return matmul_dispatch(x, x_dtype, M, K, w, transpose, y, N, y_dtype, (cudaStream_t)stream);
+}
+
+qmm_status qmm_matmul_parts(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K, const qmm_qweight* parts,
+                            int n_parts, void* y, qmm_dtype y_dtype, void* stream) {
+  if (!parts || n_parts < 1 || n_parts > kMaxParts) return QMM_ERR_INVALID_ARG;
+  int64_t ldy = 0;
+  for (int i = 0; i < n_parts; ++i) {
+    const qmm_status s = check_matmul(x_dtype, M, K, &parts[i], 1, y_dtype);
+    if (s != QMM_OK) return s;
+    ldy += parts[i].rows;
+  }
+  if (M == 0 || ldy == 0) return QMM_OK;
+  if (!aligned16(x) || !aligned16(y)) return QMM_ERR_ALIGNMENT;
+  qmm_status s = device_check();
+  if (s != QMM_OK) return s;
+  const int esize = y_dtype == QMM_F32 ? 4 : 2;
+  int64_t off = 0;
+  for (int i = 0; i < n_parts; ++i) {
+    if (parts[i].rows > 0) {
+      s = matmul_dispatch(x, x_dtype, M, K, &parts[i], 1, static_cast<char*>(y) + off * esize, ldy, y_dtype,
+                          (cudaStream_t)stream);
+      if (s != QMM_OK) return s;
+    }
+    off += parts[i].rows;
+  }
+  return QMM_OK;
+}
+
+qmm_status qmm_quantize_dynamic_int8(const void* w, qmm_dtype w_dtype, int64_t n, int8_t* q, float* params,
+                                     void* stream) {
+  if (!dtype_ok(w_dtype)) return QMM_ERR_DTYPE;
+  if (n <= 0) return QMM_ERR_INVALID_ARG;
+  if (!aligned16(w) || !aligned16(q) || !aligned4(params)) return QMM_ERR_ALIGNMENT;
+  const qmm_status s = device_check();
+  if (s != QMM_OK) return s;
+  return launch_status(qmm::launch_quantize_dyn8(w, w_dtype, n, q, params, (cudaStream_t)stream));
+}
+
+qmm_status qmm_dequantize_dynamic_int8(const int8_t* q, int64_t n, const float* params, void* out,
+                                       qmm_dtype out_dtype, void* stream) {
+  if (!dtype_ok(out_dtype)) return QMM_ERR_DTYPE;
+  if (n < 0) return QMM_ERR_INVALID_ARG;
+  if (n == 0) return QMM_OK;
+  if (!aligned16(q) || !aligned16(out) || !aligned4(params)) return QMM_ERR_ALIGNMENT;
+  const qmm_status s = device_check();
+  if (s != QMM_OK) return s;
+  return launch_status(qmm::launch_dequantize_dyn8(q, n, params, out, out_dtype, (cudaStream_t)stream));
+}
+
+qmm_status qmm_matmul_dynamic_int8(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K, const int8_t* q,
+                                   int64_t N, const float* params, void* y, qmm_dtype y_dtype, void* stream) {
+  if (!dtype_ok(x_dtype) || !dtype_ok(y_dtype)) return QMM_ERR_DTYPE;
+  if (y_dtype != x_dtype && y_dtype != QMM_F32) return QMM_ERR_DTYPE;
+  if (M < 0 || K <= 0 || N < 0) return QMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return QMM_OK;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(y) || !aligned4(params)) return QMM_ERR_ALIGNMENT;
+  const qmm_status s = device_check();
+  if (s != QMM_OK) return s;
+  return launch_status(qmm::launch_matmul_dyn8(x, x_dtype, M, K, q, N, params, y, y_dtype, (cudaStream_t)stream));
 }
 
 static qmm_status moe_common(const void* a, qmm_dtype a_dtype, const int32_t* ids,

@@ -153,6 +153,7 @@ struct GemmParams {
   const void* scales;
   const void* biases;
   void* y;
+  int64_t ldy;  // elements between output rows
   int y_dtype;
   int M, N, K, G, wpr;
   // MoE prefill form (MOE instantiation): the schedule that the routing
@@ -606,7 +607,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
               const float f = failed ? __int_as_float(0x7fc00000) : __uint_as_float(v[jj]);
               // dense: token m0 + slot; MoE: the pair listed at m0 + slot
               const int64_t orow = MOE ? (int64_t)__ldg(p.ws_pairs + tl.m0 + slot) : (int64_t)(tl.m0 + slot);
-              put(orow * p.N + n, f);
+              put(orow * p.ldy + n, f);
             }
           }
         }
@@ -732,7 +733,7 @@ static bool make_x_map(CUtensorMap* m, const void* x, int x_dtype, int64_t rows,
 
 // cudaErrorNotSupported: the call does not fit this kernel (the caller falls back)
 cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
-                            void* y, int y_dtype, cudaStream_t st) {
+                            void* y, int64_t ldy, int y_dtype, cudaStream_t st) {
   if (M > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->rows > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
@@ -746,6 +747,7 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   prm.scales = w->scales;
   prm.biases = w->biases;
   prm.y = y;
+  prm.ldy = ldy;
   prm.y_dtype = y_dtype;
   prm.M = (int)M;
   prm.N = (int)w->rows;
@@ -779,6 +781,7 @@ cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const q
   prm.scales = w->scales;
   prm.biases = w->biases;
   prm.y = out;
+  prm.ldy = w->n_rows;
   prm.y_dtype = out_dtype;
   prm.M = 0;
   prm.N = (int)w->n_rows;

@@ -27,7 +27,7 @@ template <int B, typename TX>
 __global__ void __launch_bounds__(256)
 generic_t1_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ packed,
                   const TX* __restrict__ scales, const TX* __restrict__ biases, int64_t N, int gs,
-                  void* y, int y_dtype) {
+                  void* y, int64_t ldy, int y_dtype) {
   const int lane = threadIdx.x & 31;
   const int64_t n = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5);
   if (n >= N) return;
@@ -51,7 +51,7 @@ generic_t1_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t
     }
     if (lane == 0)
       for (int i = 0; i < kMB; ++i)
-        if (m0 + i < M) store_as(y, y_dtype, (m0 + i) * N + n, acc[i]);
+        if (m0 + i < M) store_as(y, y_dtype, (m0 + i) * ldy + n, acc[i]);
   }
 }
 
@@ -60,7 +60,7 @@ template <int B, typename TX>
 __global__ void __launch_bounds__(256)
 generic_t0_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ packed,
                   const TX* __restrict__ scales, const TX* __restrict__ biases, int64_t N, int gs,
-                  void* y, int y_dtype) {
+                  void* y, int64_t ldy, int y_dtype) {
   const int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   const int64_t m0 = (int64_t)blockIdx.y * kMB;
   if (n >= N) return;
@@ -76,44 +76,44 @@ generic_t0_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t
       if (m0 + i < M) acc[i] = fmaf(to_f32(x[(m0 + i) * K + k]), w, acc[i]);
   }
   for (int i = 0; i < kMB; ++i)
-    if (m0 + i < M) store_as(y, y_dtype, (m0 + i) * N + n, acc[i]);
+    if (m0 + i < M) store_as(y, y_dtype, (m0 + i) * ldy + n, acc[i]);
 }
 
 template <int B, typename TX>
 static cudaError_t launch_g(const void* x, int64_t M, int64_t K, const qmm_qweight* w,
-                            int transpose, void* y, int y_dtype, cudaStream_t st) {
+                            int transpose, void* y, int64_t ldy, int y_dtype, cudaStream_t st) {
   auto X = reinterpret_cast<const TX*>(x);
   auto S = reinterpret_cast<const TX*>(w->scales);
   auto Bi = reinterpret_cast<const TX*>(w->biases);
   if (transpose) {
     const int64_t N = w->rows;
     const int blocks = (int)((N + 7) / 8);
-    generic_t1_kernel<B, TX><<<blocks, 256, 0, st>>>(X, M, K, w->packed, S, Bi, N, w->group_size, y, y_dtype);
+    generic_t1_kernel<B, TX><<<blocks, 256, 0, st>>>(X, M, K, w->packed, S, Bi, N, w->group_size, y, ldy, y_dtype);
   } else {
     const int64_t N = w->cols;
     dim3 grid((unsigned)((N + 255) / 256), (unsigned)((M + kMB - 1) / kMB));
-    generic_t0_kernel<B, TX><<<grid, 256, 0, st>>>(X, M, K, w->packed, S, Bi, N, w->group_size, y, y_dtype);
+    generic_t0_kernel<B, TX><<<grid, 256, 0, st>>>(X, M, K, w->packed, S, Bi, N, w->group_size, y, ldy, y_dtype);
   }
   return cudaGetLastError();
 }
 
 template <typename TX>
 static cudaError_t launch_gb(const void* x, int64_t M, int64_t K, const qmm_qweight* w,
-                             int transpose, void* y, int y_dtype, cudaStream_t st) {
+                             int transpose, void* y, int64_t ldy, int y_dtype, cudaStream_t st) {
   switch (w->bits) {
-    case 2: return launch_g<2, TX>(x, M, K, w, transpose, y, y_dtype, st);
-    case 3: return launch_g<3, TX>(x, M, K, w, transpose, y, y_dtype, st);
-    case 4: return launch_g<4, TX>(x, M, K, w, transpose, y, y_dtype, st);
-    case 6: return launch_g<6, TX>(x, M, K, w, transpose, y, y_dtype, st);
-    default: return launch_g<8, TX>(x, M, K, w, transpose, y, y_dtype, st);
+    case 2: return launch_g<2, TX>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+    case 3: return launch_g<3, TX>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+    case 4: return launch_g<4, TX>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+    case 6: return launch_g<6, TX>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+    default: return launch_g<8, TX>(x, M, K, w, transpose, y, ldy, y_dtype, st);
   }
 }
 
 cudaError_t launch_generic(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w,
-                           int transpose, void* y, int y_dtype, cudaStream_t st) {
-  if (x_dtype == QMM_F32) return launch_gb<float>(x, M, K, w, transpose, y, y_dtype, st);
-  if (x_dtype == QMM_BF16) return launch_gb<__nv_bfloat16>(x, M, K, w, transpose, y, y_dtype, st);
-  return launch_gb<__half>(x, M, K, w, transpose, y, y_dtype, st);
+                           int transpose, void* y, int64_t ldy, int y_dtype, cudaStream_t st) {
+  if (x_dtype == QMM_F32) return launch_gb<float>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+  if (x_dtype == QMM_BF16) return launch_gb<__nv_bfloat16>(x, M, K, w, transpose, y, ldy, y_dtype, st);
+  return launch_gb<__half>(x, M, K, w, transpose, y, ldy, y_dtype, st);
 }
 
 }  // namespace qmm

@@ -93,7 +93,7 @@ constexpr int kMB = 8;  // tokens per pass
 template <int MODE, typename TX>
 __global__ void __launch_bounds__(256)
 matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ packed,
-                 const uint8_t* __restrict__ scales, int64_t N, void* y, int y_dtype) {
+                 const uint8_t* __restrict__ scales, int64_t N, void* y, int64_t ldy, int y_dtype) {
   using Md = Mode<MODE>;
   constexpr int B = Md::B, GS = Md::GS;
   const int lane = threadIdx.x & 31;
@@ -126,7 +126,7 @@ matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t*
       }
       if (lane == 0)
         for (int t = 0; t < kMB; ++t)
-          if (m0 + t < M) store_as(y, y_dtype, (m0 + t) * N + n, acc[t]);
+          if (m0 + t < M) store_as(y, y_dtype, (m0 + t) * ldy + n, acc[t]);
     }
   }
 }
@@ -148,17 +148,17 @@ static cudaError_t dequant_m(const qmm_qweight* w, void* out, int out_dtype, cud
 
 template <int MODE>
 static cudaError_t matmul_m(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
-                            int y_dtype, cudaStream_t st) {
+                            int64_t ldy, int y_dtype, cudaStream_t st) {
   auto S = reinterpret_cast<const uint8_t*>(w->scales);
   const int64_t N = w->rows;
   const int blocks = (int)std::min<int64_t>((N + 7) / 8, 148 * 8);
   if (x_dtype == QMM_F32)
-    matmul_mx_kernel<MODE, float><<<blocks, 256, 0, st>>>((const float*)x, M, K, w->packed, S, N, y, y_dtype);
+    matmul_mx_kernel<MODE, float><<<blocks, 256, 0, st>>>((const float*)x, M, K, w->packed, S, N, y, ldy, y_dtype);
   else if (x_dtype == QMM_BF16)
     matmul_mx_kernel<MODE, __nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)x, M, K, w->packed, S,
-                                                                  N, y, y_dtype);
+                                                                  N, y, ldy, y_dtype);
   else
-    matmul_mx_kernel<MODE, __half><<<blocks, 256, 0, st>>>((const __half*)x, M, K, w->packed, S, N, y, y_dtype);
+    matmul_mx_kernel<MODE, __half><<<blocks, 256, 0, st>>>((const __half*)x, M, K, w->packed, S, N, y, ldy, y_dtype);
   return cudaGetLastError();
 }
 
@@ -173,11 +173,11 @@ cudaError_t launch_dequantize_mx(const qmm_qweight* w, void* out, int out_dtype,
 }
 
 cudaError_t launch_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
-                             int y_dtype, cudaStream_t st) {
+                             int64_t ldy, int y_dtype, cudaStream_t st) {
   switch (w->mode) {
-    case QMM_MODE_MXFP4: return mx::matmul_m<QMM_MODE_MXFP4>(x, x_dtype, M, K, w, y, y_dtype, st);
-    case QMM_MODE_MXFP8: return mx::matmul_m<QMM_MODE_MXFP8>(x, x_dtype, M, K, w, y, y_dtype, st);
-    default: return mx::matmul_m<QMM_MODE_NVFP4>(x, x_dtype, M, K, w, y, y_dtype, st);
+    case QMM_MODE_MXFP4: return mx::matmul_m<QMM_MODE_MXFP4>(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
+    case QMM_MODE_MXFP8: return mx::matmul_m<QMM_MODE_MXFP8>(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
+    default: return mx::matmul_m<QMM_MODE_NVFP4>(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
   }
 }
 

@@ -40,7 +40,7 @@ struct QgemvParams {
 cudaError_t launch_qgemv(QgemvParams prm, int bits, int gs, int dtype, bool dual, cudaStream_t st);
 
 inline QgemvParams make_dense_params(const void* x, int64_t M, int64_t K, const qmm_qweight* w,
-                                     void* y, int y_dtype) {
+                                     void* y, int64_t ldy, int y_dtype) {
   QgemvParams p{};
   p.packed[0] = w->packed;
   p.scales[0] = w->scales;
@@ -57,7 +57,7 @@ inline QgemvParams make_dense_params(const void* x, int64_t M, int64_t K, const 
   p.n_pairs = (int)M;
   p.out = y;
   p.out_dtype = y_dtype;
-  p.out_ld = w->rows;
+  p.out_ld = ldy;
   p.d_status = nullptr;
   p.use_tma = 1;
   return p;
