@@ -1,10 +1,15 @@
 // Instantiations of the decode GEMV / MoE kernel family for 3-bit codes.
-#include "qgemv_impl.cuh"
+#include "qgemv_stream.cuh"
 
 namespace qmm {
 
 cudaError_t launch_qgemv_b3(const QgemvParams& prm, int gs, int dtype, int mt, bool dual,
                             cudaStream_t st) {
+  // the streaming kernel for group sizes 64 and 128, else the cp.async kernel
+  if (prm.use_tma && gs != 32) {
+    const cudaError_t es = stream::try_stream<3>(prm, gs, dtype, mt, dual, st);
+    if (es != cudaErrorNotSupported) return es;
+  }
   if (dtype == QMM_BF16) {
     if (gs == 32) return launch_mt<3, 32, __nv_bfloat16>(prm, mt, dual, st);
     if (gs == 64) return launch_mt<3, 64, __nv_bfloat16>(prm, mt, dual, st);

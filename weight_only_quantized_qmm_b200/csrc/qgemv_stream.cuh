@@ -56,7 +56,6 @@
 namespace qmm {
 namespace stream {
 
-constexpr int kRB = 2;          // partial-sum ring entries (tiles)
 constexpr int kMaxStages = 8;
 
 struct Params {
@@ -81,28 +80,59 @@ struct Params {
 //          from the word shifted right by 8);
 //   2-bit: pairs (j, j+8), offsets 0, 2, 4, 6, 8 for j < 5 and 0, 2, 4 for
 //          j = 5..7 (from the word shifted right by 10).
+// 3- and 6-bit codes straddle words, so quarter t is the contiguous run of
+// codes [kCodes t, kCodes (t + 1)) of the group's row, taken 16 codes (48 or
+// 96 bits) at a time:
+//   3-bit: three byte permutes place 16-bit windows of the run under the two
+//          halves of a register; per window up to three codes sit at bit
+//          offsets <= 7, and one lop3 per pair keeps one of them per half
+//          (3 prmt + 8 lop3 per 16 codes);
+//   6-bit: one funnel shift per pair puts code 4k (or 4k + 1) at bit 4 of the
+//          low half and code 4k + 2 (4k + 3) at bit 0 of the high half
+//          (8 shf + 8 lop3 per 16 codes).
 template <int BITS, int GS>
 struct Lanes {
-  static constexpr int kLPW = 32 / BITS;            // codes per packed word
-  static constexpr int kOPW = kLPW / 2;             // f16 pairs per word
-  static constexpr int kCodes = GS / 4;             // codes of a thread's quarter
-  static constexpr int kRegs = kCodes * BITS / 32;  // packed words of a quarter
-  static constexpr int kOuts = kCodes / 2;          // f16 pairs of a quarter
-  static constexpr int kSteps = kCodes / 4;         // m16n8k16 steps per group
+  static constexpr bool kWhole = BITS == 2 || BITS == 4 || BITS == 8;  // lanes never straddle words
+  static constexpr int kLPW = kWhole ? 32 / BITS : 1;  // codes per packed word
+  static constexpr int kOPW = kWhole ? kLPW / 2 : 1;   // f16 pairs per word
+  static constexpr int kCodes = GS / 4;                // codes of a thread's quarter
+  static constexpr int kQBits = kCodes * BITS;         // bits of a quarter
+  // packed words a thread reads per row: the quarter's own words, or (a
+  // 48-bit quarter) the two words that hold it
+  static constexpr int kRegs = (kQBits + 31) / 32;
+  static constexpr int kOuts = kCodes / 2;             // f16 pairs of a quarter
+  static constexpr int kSteps = kCodes / 4;            // m16n8k16 steps per group
   static constexpr int kWordsPerGroup = GS * BITS / 32;
-  static constexpr bool kOk = (BITS == 2 || BITS == 4 || BITS == 8) && (kCodes * BITS) % 32 == 0;
-  static constexpr uint32_t kMagic = 0x64006400u;   // f16 1024.0 in both halves
+  static constexpr bool kOk = kWhole ? kQBits % 32 == 0 : ((BITS == 3 || BITS == 6) && (GS == 64 || GS == 128));
+  static constexpr uint32_t kMagic = 0x64006400u;      // f16 1024.0 in both halves
   static constexpr float kOff = 1024.0f;
   __host__ __device__ static constexpr int pos(int j) {
     return BITS == 8 ? 0 : BITS == 4 ? (j & 1) * 4 : (j < 5 ? 2 * j : 2 * (j - 5));
   }
-  // pair o of the quarter -> code index (within the quarter) of its low and
-  // high half
-  __host__ __device__ static constexpr int lo_code(int o) { return (o / kOPW) * kLPW + o % kOPW; }
-  __host__ __device__ static constexpr int hi_code(int o) { return lo_code(o) + kOPW; }
-  __host__ __device__ static constexpr int lo_pos(int o) { return pos(o % kOPW); }
-  // first code (within the group) of word k of quarter t
-  __host__ __device__ static constexpr int word_code(int t, int k) { return (t + 4 * k) * kLPW; }
+  // pair o of the quarter -> code index (within the quarter) and bit offset
+  // of its low and high half
+  __host__ __device__ static constexpr int lo_code(int o) {
+    return kWhole ? (o / kOPW) * kLPW + o % kOPW
+                  : 16 * (o / 8) + (BITS == 3 ? "\x00\x01\x02\x08\x09\x0a\x06\x07"[o % 8]
+                                                : "\x00\x01\x04\x05\x08\x09\x0c\x0d"[o % 8]);
+  }
+  __host__ __device__ static constexpr int hi_code(int o) {
+    return kWhole ? lo_code(o) + kOPW
+                  : 16 * (o / 8) + (BITS == 3 ? "\x03\x04\x05\x0b\x0c\x0d\x0e\x0f"[o % 8]
+                                                : "\x02\x03\x06\x07\x0a\x0b\x0e\x0f"[o % 8]);
+  }
+  __host__ __device__ static constexpr int lo_pos(int o) {
+    return kWhole ? pos(o % kOPW) : (BITS == 3 ? "\x00\x03\x06\x00\x03\x06\x02\x05"[o % 8] : 4);
+  }
+  __host__ __device__ static constexpr int hi_pos(int o) {
+    return kWhole ? pos(o % kOPW) : (BITS == 3 ? "\x01\x04\x07\x01\x04\x07\x02\x05"[o % 8] : 0);
+  }
+  // code of the group held as code i of quarter t
+  __host__ __device__ static constexpr int gcode(int t, int i) {
+    return kWhole ? (t + 4 * (i / kLPW)) * kLPW + i % kLPW : kCodes * t + i;
+  }
+  // first packed word (within the group's row) that thread t reads
+  __host__ __device__ static constexpr int first_word(int t) { return (t * kQBits) >> 5; }
 };
 
 // Four 8x8 16-bit matrices from shared memory in the mma fragment layout
@@ -117,9 +147,9 @@ __device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, 
 // (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
 // matrices per pair (2: gate and up).  SB1: rows of G <= UG groups whose
 // scale/bias rows are not 16-byte strided (G % 8 != 0, e.g. K = 768 at group
-// 64): a unit is a whole row tile, its 16 scale (bias) rows arrive as one
-// contiguous 1-D bulk copy of 32 G bytes, unswizzled, and groups >= G are
-// skipped.
+// 64): a unit is TR = 4 whole row tiles (64 rows), its 64 scale (bias) rows
+// arrive as one contiguous 1-D bulk copy of 128 G bytes, unswizzled; KC / TR
+// consumers share a row tile, and groups >= G are skipped.
 template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false>
 struct Cfg {
   using L = Lanes<BITS, GS>;
@@ -130,18 +160,26 @@ struct Cfg {
   static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
   static constexpr int WPG = L::kWordsPerGroup;                   // words per group per row
   static constexpr int GPU = UG;                                  // groups per unit
-  static constexpr int GPW = GPU / KC;                            // groups per consumer per unit
+  static constexpr int TR = SB1 ? 4 : 1;                          // 16-row tiles per unit
+  static constexpr int ROWS = 16 * TR;                            // weight rows per unit
+  static constexpr int WPT = KC / TR;                             // consumers per row tile
+  static constexpr int GPW = GPU / WPT;                           // groups per consumer per unit
   static constexpr int Z = GPU * WPG / 32;                        // 128-byte slices per unit row
-  static constexpr int CODE_BYTES = Z * 16 * 128;                 // one matrix
-  static constexpr int SB_BYTES = 16 * GPU * 2;                   // scales (or biases) of one matrix
+  static constexpr int SLICE = ROWS * 128;                        // bytes of one slice (all rows)
+  static constexpr int CODE_BYTES = Z * SLICE;                    // one matrix
+  static constexpr int SB_BYTES = ROWS * GPU * 2;                 // scales (or biases) of one matrix
   static constexpr int TOKP = 8 * MT;
   static constexpr int CH = ONE ? 1 : TOKP;                       // pairs per segment
   static constexpr int XG = 4 * L::kCodes * 2;                    // staged f16 x bytes per group
-  static_assert(L::kOk, "integral-lane codes only");
-  static_assert(GPW >= 1 && GPW * KC == GPU, "whole groups per consumer");
+  static_assert(L::kOk, "a supported (bits, group size)");
+  static_assert(GPW >= 1 && GPW * WPT == GPU && WPT * TR == KC, "whole groups per consumer");
   static_assert(Z >= 1 && Z <= 16, "unit of at most 16 slices (32 KB)");
+  static_assert(GPU * WPG % 32 == 0, "units of whole 128-byte slices");
   static_assert(GPU * 2 == 32 || GPU * 2 == 64 || GPU * 2 == 128, "scale rows of one swizzle span");
-  static_assert((kRB & (kRB - 1)) == 0, "partial ring is a power of two");
+  // partial-sum ring entries (tiles): one token's partials are small, so
+  // that ring is deeper; the multi-token fragments would crowd the stages
+  static constexpr int RB = ONE ? 4 : 2;
+  static_assert((RB & (RB - 1)) == 0, "partial ring is a power of two");
 };
 
 __device__ __forceinline__ void sts32(uint32_t a, float v) {
@@ -230,17 +268,62 @@ __device__ __forceinline__ void word_pairs16(uint32_t w, uint32_t* o) {
   }
 }
 
+__device__ __forceinline__ uint32_t prmt_rt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// The kOuts f16 pairs of thread t's quarter (see Lanes).
+template <class L>
+__device__ __forceinline__ void quarter_pairs(const uint32_t (&r)[L::kRegs], int t, uint32_t* o) {
+  if constexpr (L::kWhole) {
+#pragma unroll
+    for (int k = 0; k < L::kRegs; ++k) word_pairs16<32 / L::kLPW>(r[k], o + k * L::kOPW);
+  } else if constexpr (L::kQBits / L::kCodes == 3) {
+#pragma unroll
+    for (int c = 0; c < L::kCodes / 16; ++c) {
+      // 16 codes = bytes B0..B5 of the word pair (lo, hi) from byte `off`
+      const uint32_t lo = L::kRegs == 2 ? r[0] : r[c], hi = L::kRegs == 2 ? r[1] : r[c + 1];
+      const uint32_t add = (L::kRegs == 2 ? (uint32_t)(t & 1) * 2u : (uint32_t)c * 2u) * 0x1111u;
+      const uint32_t r0 = prmt_rt(lo, hi, 0x2110u + add);  // (B0, B1 | B1, B2)
+      const uint32_t r1 = prmt_rt(lo, hi, 0x5443u + add);  // (B3, B4 | B4, B5)
+      const uint32_t r2 = prmt_rt(lo, hi, 0x5532u + add);  // (B2, B3 | B5, B5)
+      o[8 * c + 0] = mask_magic<0x000E0007u>(r0);
+      o[8 * c + 1] = mask_magic<0x00700038u>(r0);
+      o[8 * c + 2] = mask_magic<0x038001C0u>(r0);
+      o[8 * c + 3] = mask_magic<0x000E0007u>(r1);
+      o[8 * c + 4] = mask_magic<0x00700038u>(r1);
+      o[8 * c + 5] = mask_magic<0x038001C0u>(r1);
+      o[8 * c + 6] = mask_magic<0x001C001Cu>(r2);
+      o[8 * c + 7] = mask_magic<0x00E000E0u>(r2);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < L::kCodes / 16; ++c) {
+      // 16 codes = words w0..w2; the windows start at stream bits 24k - 4
+      // (codes 4k, 4k + 2) and 24k + 2 (codes 4k + 1, 4k + 3)
+      const uint32_t w0 = r[3 * c], w1 = r[3 * c + 1], w2 = r[3 * c + 2];
+      o[8 * c + 0] = mask_magic<0x003F03F0u>(__funnelshift_r(0u, w0, 28));
+      o[8 * c + 1] = mask_magic<0x003F03F0u>(__funnelshift_r(w0, w1, 2));
+      o[8 * c + 2] = mask_magic<0x003F03F0u>(__funnelshift_r(w0, w1, 20));
+      o[8 * c + 3] = mask_magic<0x003F03F0u>(__funnelshift_r(w0, w1, 26));
+      o[8 * c + 4] = mask_magic<0x003F03F0u>(__funnelshift_r(w1, w2, 12));
+      o[8 * c + 5] = mask_magic<0x003F03F0u>(__funnelshift_r(w1, w2, 18));
+      o[8 * c + 6] = mask_magic<0x003F03F0u>(__funnelshift_r(w2, 0u, 4));
+      o[8 * c + 7] = mask_magic<0x003F03F0u>(__funnelshift_r(w2, 0u, 10));
+    }
+  }
+}
+
 // Tensor-core partial dot of one group for 16 rows x 8 (per token tile)
 // columns: d = sum over the group's k16 steps of (1024 + q 2^p) * x''.
 template <class L, int MT>
 __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[L::kRegs], const uint32_t (&rawB)[L::kRegs],
-                                           const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4]) {
+                                           int t, const uint32_t (&xb)[MT], uint32_t xo, float (&d)[MT][4]) {
   uint32_t pA[L::kOuts], pB[L::kOuts];
-#pragma unroll
-  for (int k = 0; k < L::kRegs; ++k) {
-    word_pairs16<32 / L::kLPW>(rawA[k], pA + k * L::kOPW);
-    word_pairs16<32 / L::kLPW>(rawB[k], pB + k * L::kOPW);
-  }
+  quarter_pairs<L>(rawA, t, pA);
+  quarter_pairs<L>(rawB, t, pB);
 #pragma unroll
   for (int q2 = 0; q2 < L::kSteps / 2; ++q2) {
     uint4 bf[MT];
@@ -264,13 +347,10 @@ __device__ __forceinline__ void group_dot1(const uint32_t (&rawA)[L::kRegs], con
 // As group_dot1 for one token column, with the x fragments in registers.
 template <class L>
 __device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[L::kRegs], const uint32_t (&rawB)[L::kRegs],
-                                             const uint4 (&bf)[L::kSteps / 2], float (&d)[4]) {
+                                             int t, const uint4 (&bf)[L::kSteps / 2], float (&d)[4]) {
   uint32_t pA[L::kOuts], pB[L::kOuts];
-#pragma unroll
-  for (int k = 0; k < L::kRegs; ++k) {
-    word_pairs16<32 / L::kLPW>(rawA[k], pA + k * L::kOPW);
-    word_pairs16<32 / L::kLPW>(rawB[k], pB + k * L::kOPW);
-  }
+  quarter_pairs<L>(rawA, t, pA);
+  quarter_pairs<L>(rawB, t, pB);
   // even and odd k16 steps in two chains (half the dependent mma latency);
   // only column 0 (rows g, g + 8: d[0], d[2]) is merged, the others are idle
   float e[4];
@@ -353,20 +433,32 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     __align__(16) T xv[L::kCodes];
     if (act && gl < q.G) {
       const T* xg = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS;
-      constexpr int WB = L::kLPW * (int)sizeof(T);  // bytes of x under one packed word
+      if constexpr (L::kWhole) {
+        constexpr int WB = L::kLPW * (int)sizeof(T);  // bytes of x under one packed word
 #pragma unroll
-      for (int k = 0; k < L::kRegs; ++k) {
-        const T* xa = xg + L::word_code(tt, k);
-        T* dst = xv + k * L::kLPW;
-        if (WB % 16 == 0 && (reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
+        for (int k = 0; k < L::kRegs; ++k) {
+          const T* xa = xg + L::gcode(tt, k * L::kLPW);
+          T* dst = xv + k * L::kLPW;
+          if (WB % 16 == 0 && (reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
 #pragma unroll
-          for (int c = 0; c < WB / 16; ++c)
-            reinterpret_cast<uint4*>(dst)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
-        } else if (WB == 8 && (reinterpret_cast<uintptr_t>(xa) & 7) == 0) {
-          *reinterpret_cast<uint2*>(dst) = __ldg(reinterpret_cast<const uint2*>(xa));
+            for (int c = 0; c < WB / 16; ++c)
+              reinterpret_cast<uint4*>(dst)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
+          } else if (WB == 8 && (reinterpret_cast<uintptr_t>(xa) & 7) == 0) {
+            *reinterpret_cast<uint2*>(dst) = __ldg(reinterpret_cast<const uint2*>(xa));
+          } else {
+#pragma unroll
+            for (int c = 0; c < L::kLPW; ++c) dst[c] = xa[c];
+          }
+        }
+      } else {  // the quarter's codes are one contiguous run
+        const T* xa = xg + L::gcode(tt, 0);
+        if ((reinterpret_cast<uintptr_t>(xa) & 15) == 0) {
+#pragma unroll
+          for (int c = 0; c < L::kCodes * (int)sizeof(T) / 16; ++c)
+            reinterpret_cast<uint4*>(xv)[c] = __ldg(reinterpret_cast<const uint4*>(xa) + c);
         } else {
 #pragma unroll
-          for (int c = 0; c < L::kLPW; ++c) dst[c] = xa[c];
+          for (int c = 0; c < L::kCodes; ++c) xv[c] = xa[c];
         }
       }
     } else {
@@ -390,9 +482,8 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     __align__(16) uint32_t outv[L::kOuts];
 #pragma unroll
     for (int o = 0; o < L::kOuts; ++o) {
-      const float sc = exp2i(e - L::lo_pos(o));
       const float xl = to_f32(xv[L::lo_code(o)]), xh = to_f32(xv[L::hi_code(o)]);
-      const __half hl = __float2half_rn(xl * sc), hh = __float2half_rn(xh * sc);
+      const __half hl = __float2half_rn(xl * exp2i(e - L::lo_pos(o))), hh = __float2half_rn(xh * exp2i(e - L::hi_pos(o)));
       ss += __half2float(hl) + __half2float(hh);
       sx += xl + xh;
       outv[o] = (uint32_t)__half_as_ushort(hl) | ((uint32_t)__half_as_ushort(hh) << 16);
@@ -433,7 +524,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   const uint32_t sb_ring = smem_u32(smem + p.off_sb);
   const uint32_t bar_full = smem_u32(smem + p.off_bar);
   const uint32_t bar_pfull = bar_full + 16 * kMaxStages;  // after full[] and empty[]
-  const uint32_t bar_pempty = bar_pfull + 8 * kRB;
+  const uint32_t bar_pempty = bar_pfull + 8 * C::RB;
   const uint32_t part_sa = smem_u32(smem + p.off_part);
   uint8_t* xs = smem + p.off_xs;
   float4* xrec = reinterpret_cast<float4*>(smem + p.off_xsum);  // [Gpad][TOKP] group records
@@ -444,7 +535,10 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   int* s_dist = s_fill + E;
   int* s_seg = s_dist + E;  // E + 1 entries
   int* s_list = s_seg + E + 1;
-  __shared__ int s_nd;
+  // expert (weight block) of distinct entry j; shares the placement counters,
+  // which are dead once the plan is built
+  int* s_wexp = s_fill;
+  __shared__ int s_nd, s_direct;
   __shared__ int64_t s_xoff[16];  // activation row offsets of the staged x rows
 
   if (tid == 0) {
@@ -452,7 +546,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_full + 8 * kMaxStages + 8 * s, KC);
     }
-    for (int e = 0; e < kRB; ++e) {
+    for (int e = 0; e < C::RB; ++e) {
       mbar_init(bar_pfull + 8 * e, KC);
       mbar_init(bar_pempty + 8 * e, 1);
     }
@@ -471,7 +565,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     const int nun = min((te0 - tb0) * p.upt, STAGES);
     for (int i = 0; i < nun; ++i) {
       const int t = tb0 + i / p.upt, ku = i % p.upt;
-      const int y = (t % p.ntiles_e) * 16;
+      const int y = (t % p.ntiles_e) * C::ROWS;
       tma_prefetch_3d(&tmc0, 0, y, ku * C::Z);
       tma_prefetch_2d(&tms0, ku * GPU, y);
       tma_prefetch_2d(&tmb0, ku * GPU, y);
@@ -480,13 +574,45 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   // weights, ids and x may all come from the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (q.ids) {
-    build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, s_list + q.n_pairs, &s_nd);
-    if (tid == 0) {
-      int run = 0;
-      s_seg[0] = 0;
-      for (int j = 0; j < s_nd; ++j) {
-        run += (s_cnt[s_dist[j]] + CH - 1) / CH;
-        s_seg[j + 1] = run;
+    bool direct = false;
+    if constexpr (C::ONE) {
+      // One pair per segment: a segment's position in the list does not change
+      // what it computes, so when every id is in range segment j is simply
+      // pair j (one warp reads the ids; no sort, one barrier).
+      if (q.n_pairs <= 32 && q.n_pairs <= E) {
+        if (warp == 0) {
+          const int e = lane < q.n_pairs ? q.ids[lane] : 0;
+          const bool all_ok = __all_sync(0xffffffffu, e >= 0 && e < E);
+          if (all_ok && lane < q.n_pairs) {
+            s_cnt[lane] = 1;
+            s_start[lane] = lane;
+            s_list[lane] = lane;
+            s_dist[lane] = lane;
+            s_wexp[lane] = e;
+            s_seg[lane] = lane;
+          }
+          if (lane == 0) {
+            s_direct = all_ok;
+            if (all_ok) {
+              s_seg[q.n_pairs] = q.n_pairs;
+              s_nd = q.n_pairs;
+            }
+          }
+        }
+        __syncthreads();
+        direct = s_direct;
+      }
+    }
+    if (!direct) {  // pairs sorted by expert; out-of-range ids reported and zero-filled
+      build_plan(q, s_cnt, s_start, s_fill, s_dist, s_list, s_list + q.n_pairs, &s_nd);
+      if (tid == 0) {
+        int run = 0;
+        s_seg[0] = 0;
+        for (int j = 0; j < s_nd; ++j) {
+          run += (s_cnt[s_dist[j]] + CH - 1) / CH;
+          s_seg[j + 1] = run;
+          s_wexp[j] = s_dist[j];
+        }
       }
     }
   } else {
@@ -496,6 +622,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       s_cnt[0] = q.n_pairs;
       s_start[0] = 0;
       s_dist[0] = 0;
+      s_wexp[0] = 0;
       s_nd = 1;
       s_seg[0] = 0;
       s_seg[1] = (q.n_pairs + CH - 1) / CH;
@@ -527,14 +654,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           set_status(q.d_status, QMM_ERR_TIMEOUT);
           break;
         }
-        const int y = s_dist[w.j] * (int)q.n_rows + w.rt * 16;  // first row in the expert stack
+        const int y = s_wexp[w.j] * (int)q.n_rows + w.rt * C::ROWS;  // first row in the expert stack
         const uint32_t fb = bar_full + 8 * slot;
         mbar_arrive_expect_tx(fb, p.tx);
         const uint32_t cd = code_ring + (uint32_t)(slot * NS * C::CODE_BYTES);
         const uint32_t sd = sb_ring + (uint32_t)(slot * NS * 2 * C::SB_BYTES);
         tma_load_3d(cd, &tmc0, 0, y, ku * C::Z, fb);
-        if constexpr (SB1) {  // rows y .. y + 15 of the [rows, G] arrays, contiguous
-          const uint32_t nb = (uint32_t)(32 * q.G);
+        if constexpr (SB1) {  // rows y .. y + ROWS - 1 of the [rows, G] arrays, contiguous
+          const uint32_t nb = (uint32_t)(2 * C::ROWS * q.G);
           bulk_load_1d(sd, reinterpret_cast<const uint8_t*>(q.scales[0]) + (int64_t)y * q.G * 2, nb, fb);
           bulk_load_1d(sd + C::SB_BYTES, reinterpret_cast<const uint8_t*>(q.biases[0]) + (int64_t)y * q.G * 2, nb, fb);
         } else {
@@ -566,8 +693,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     Walk w;
     if (nt > 0) w.start(tb, p.ntiles_e, s_seg, nd);
     for (int jt = 0; jt < nt; ++jt) {
-      const int e = jt & (kRB - 1);
-      const bool ok = mbar_wait(bar_pfull + 8 * e, (uint32_t)(jt / kRB) & 1u, failed);
+      const int e = jt & (C::RB - 1);
+      const bool ok = mbar_wait(bar_pfull + 8 * e, (uint32_t)(jt / C::RB) & 1u, failed);
       if (__any_sync(0xffffffffu, !ok)) {
         if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
         failed = true;
@@ -577,22 +704,26 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         const int* pairs = s_list + s_start[ex] + chunk * CH;
         const int np = min(CH, s_cnt[ex] - chunk * CH);
         if constexpr (C::ONE) {
-          // partials: [entry][consumer][matrix][16 rows] floats
-          if (lane < 16) {
+          // partials: [entry][consumer][matrix][16 rows] floats; row tile rt of
+          // the unit sums its consumers rt * WPT .. rt * WPT + WPT - 1
+          for (int idx = lane; idx < 16 * C::TR; idx += 32) {
+            const int rr = idx & 15, rt = idx >> 4;
             float y[NS];
 #pragma unroll
             for (int ns = 0; ns < NS; ++ns) {
               y[ns] = 0.0f;
 #pragma unroll
-              for (int wc = 0; wc < KC; ++wc)
-                y[ns] += ldsf(part_sa + (uint32_t)((((e * KC + wc) * NS + ns) * 16 + lane) * 4));
+              for (int wc = 0; wc < C::WPT; ++wc)
+                y[ns] += ldsf(part_sa + (uint32_t)((((e * KC + rt * C::WPT + wc) * NS + ns) * 16 + rr) * 4));
             }
             const float v = NS == 2 ? y[0] / (1.0f + expf(-y[0])) * y[NS - 1] : y[0];
-            const int64_t row = (int64_t)w.rt * 16 + lane;
+            const int64_t row = (int64_t)w.rt * C::ROWS + rt * 16 + rr;
             if (row < q.n_rows) store_as(q.out, q.out_dtype, (int64_t)pairs[0] * q.out_ld + row, v);
           }
         } else {
           // partials: [entry][consumer][matrix][token tile][lane] float4 (the mma C fragment)
+#pragma unroll
+          for (int rt = 0; rt < C::TR; ++rt)
           for (int idx = lane; idx < 16 * np; idx += 32) {
             const int r = idx & 15, m = idx >> 4;
             const int mt = m >> 3, col = m & 7;
@@ -601,13 +732,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
             float y[NS];
 #pragma unroll
             for (int ns = 0; ns < NS; ++ns) {
-              const uint32_t a0 = part_sa + (uint32_t)(((((e * KC) * NS + ns) * MT + mt) * 32 + src) * 16 + ci * 4);
+              const uint32_t a0 =
+                  part_sa + (uint32_t)(((((e * KC + rt * C::WPT) * NS + ns) * MT + mt) * 32 + src) * 16 + ci * 4);
               y[ns] = 0.0f;
 #pragma unroll
-              for (int wc = 0; wc < KC; ++wc) y[ns] += ldsf(a0 + (uint32_t)(wc * NS * MT * 32 * 16));
+              for (int wc = 0; wc < C::WPT; ++wc) y[ns] += ldsf(a0 + (uint32_t)(wc * NS * MT * 32 * 16));
             }
             const float v = NS == 2 ? y[0] / (1.0f + expf(-y[0])) * y[NS - 1] : y[0];
-            const int64_t row = (int64_t)w.rt * 16 + r;
+            const int64_t row = (int64_t)w.rt * C::ROWS + rt * 16 + r;
             if (row < q.n_rows) store_as(q.out, q.out_dtype, (int64_t)pairs[m] * q.out_ld + row, v);
           }
         }
@@ -622,22 +754,26 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   // --------------------------------------------------------------- consumers
   const int g = lane >> 2, t = lane & 3;
   const uint32_t xs_sa = smem_u32(xs), xrec_sa = smem_u32(xrec);
+  // row tile (within the unit) and group slot of this consumer
+  const int rtl = warp / C::WPT, gw = warp % C::WPT;
   // per-group records of pairs 2t, 2t + 1 (pair 0 only for one pair per segment)
-  const uint32_t xrec_lane = xrec_sa + (uint32_t)((warp * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 16);
+  const uint32_t xrec_lane = xrec_sa + (uint32_t)((gw * GPW * TOKP + (C::ONE ? 0 : 2 * t)) * 16);
   // Code words of group u.  kRegs == 1: the lane's word t of rows g and
   // g + 8 (two 32-bit loads).  kRegs >= 2: ldmatrix.x4 per pair of words
   // (t + 4k, t + 4k + 4): lane l gives the row address of matrix l / 8 =
   // {row l%8, row l%8 + 8} x {chunk c, chunk c + 1}; the 128-byte swizzle puts
   // chunk c of row r at c ^ (r & 7).
   const int lr = lane & 7, lm = lane >> 3;
+  // (3- and 6-bit codes: the lane's words first_word(t) + k, one load each)
   auto code_addr = [&](int u, int k2) -> uint32_t {
-    const int w0 = (warp * GPW + u) * WPG;  // first word of the group in the unit row
-    if constexpr (L::kRegs == 1) {
-      const int wb = (w0 + t) & 31;
-      return (uint32_t)(((w0 + t) >> 5) * 2048 + g * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
+    const int w0 = (gw * GPW + u) * WPG;  // first word of the group in the unit row
+    if constexpr (L::kRegs == 1 || !L::kWhole) {
+      const int wr = w0 + (L::kWhole ? t : L::first_word(t) + k2);  // word in the unit row
+      const int wb = wr & 31;
+      return (uint32_t)((wr >> 5) * C::SLICE + (rtl * 16 + g) * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
     } else {
       const int ch = ((w0 & 31) >> 2) + 2 * k2 + (lm >> 1);  // 16-byte chunk within the 128-byte row
-      return (uint32_t)((w0 >> 5) * 2048 + (lr + 8 * (lm & 1)) * 128 + ((ch ^ lr) << 4));
+      return (uint32_t)((w0 >> 5) * C::SLICE + (rtl * 16 + lr + 8 * (lm & 1)) * 128 + ((ch ^ lr) << 4));
     }
   };
   // scale / bias offsets (within a slot) of rows g and g + 8 for this warp's
@@ -645,11 +781,11 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   // (SB1: plain [16][G] rows, pitch 2 G bytes)
   const int PITCH = SB1 ? 2 * q.G : GPU * 2;
   const int sfx = PITCH == 128 ? (g & 7) : PITCH == 64 ? ((g >> 1) & 3) : ((g >> 2) & 1);
-  const int sbyte = warp * GPW * 2;
-  const uint32_t soff = SB1 ? (uint32_t)(g * PITCH + sbyte)
+  const int sbyte = gw * GPW * 2;
+  const uint32_t soff = SB1 ? (uint32_t)((rtl * 16 + g) * PITCH + sbyte)
                             : (uint32_t)(g * PITCH + ((((sbyte >> 4) ^ sfx)) << 4) + (sbyte & 15));
   // SB1: this warp's groups past the row (>= G) take no part in the sums
-  const int live = SB1 ? min(GPW, max(0, q.G - warp * GPW)) : GPW;
+  const int live = SB1 ? min(GPW, max(0, q.G - gw * GPW)) : GPW;
 
   float acc[NS][MT][4];
 #pragma unroll
@@ -696,7 +832,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         for (int mt = 0; mt < MT; ++mt) {
           const int tr = (mt * 8 + g) < np ? mt * 8 + g : 0;  // idle columns reread pair 0
           xb[mt] = xs_sa + (uint32_t)(tr * p.tok_stride) + (uint32_t)(t * L::kCodes * 2) +
-                   (uint32_t)(warp * GPW * C::XG);
+                   (uint32_t)(gw * GPW * C::XG);
           xbu[mt] = xb[mt];
         }
         su = xrec_lane;
@@ -744,7 +880,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         for (int u = 0; u < GPW; ++u) {
           if (SB1 && u >= live) break;  // warp-uniform
           uint32_t rA[L::kRegs], rB[L::kRegs];
-          if constexpr (L::kRegs == 1) {
+          if constexpr (!L::kWhole) {
+#pragma unroll
+            for (int k = 0; k < L::kRegs; ++k) {
+              const uint32_t ca = csl + code_addr(u, k);
+              rA[k] = lds32(ca);
+              rB[k] = lds32(ca + 1024);
+            }
+          } else if constexpr (L::kRegs == 1) {
             const uint32_t ca = csl + code_addr(u, 0);
             rA[0] = lds32(ca);
             rB[0] = lds32(ca + 1024);
@@ -760,9 +903,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
             uint4 bf[L::kSteps / 2];
 #pragma unroll
             for (int q2 = 0; q2 < L::kSteps / 2; ++q2) bf[q2] = lds128(xbu[0] + (uint32_t)(u * C::XG + q2 * 16));
-            group_dot_rx<L>(rA, rB, bf, d[0]);
+            group_dot_rx<L>(rA, rB, t, bf, d[0]);
           } else
-            group_dot1<L, MT>(rA, rB, xbu, (uint32_t)(u * C::XG), d);
+            group_dot1<L, MT>(rA, rB, t, xbu, (uint32_t)(u * C::XG), d);
           const int hw = u & 1;
           const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
           const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
@@ -793,9 +936,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
     if (lane == 0) mbar_arrive(bfull + 8 * kMaxStages);  // the slot's `empty` barrier
 
     if (++ku == p.upt) {  // tile done: post this warp's partial
-      const int e = jt & (kRB - 1);
-      if (jt >= kRB) {
-        const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / kRB) - 1) & 1u, failed);
+      const int e = jt & (C::RB - 1);
+      if (jt >= C::RB) {
+        const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / C::RB) - 1) & 1u, failed);
         if (__any_sync(0xffffffffu, !okp)) {
           if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
           failed = true;
@@ -850,13 +993,15 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 
 // ------------------------------------------------------------------ host side
 // 3-D map over packed words [rows, wpr] seen as (word in slice, row, slice of
-// 32 words): a box is 16 rows x z slices, each slice 16 x 128 bytes, swizzled.
-inline bool make_code_map3(CUtensorMap* map, const uint32_t* packed, int64_t rows, int64_t wpr, int z) {
+// 32 words): a box is box_rows rows x z slices, each slice box_rows x 128 bytes,
+// swizzled.
+inline bool make_code_map3(CUtensorMap* map, const uint32_t* packed, int64_t rows, int64_t wpr, int z,
+                           int box_rows) {
   EncodeTiledFn enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {32, (cuuint64_t)rows, (cuuint64_t)(wpr / 32)};
   const cuuint64_t strides[2] = {(cuuint64_t)(wpr * 4), 128};
-  const cuuint32_t box[3] = {32, 16, (cuuint32_t)z};
+  const cuuint32_t box[3] = {32, (cuuint32_t)box_rows, (cuuint32_t)z};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(packed), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -891,7 +1036,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   if (SB1) {
     // one unit per row tile; 16-row tiles of every expert start on 16-byte
     // aligned scale/bias rows and never run past the arrays
-    if (q.G > C::GPU || q.n_rows % 16 != 0 || NS != 1) return cudaErrorNotSupported;
+    if (q.G > C::GPU || q.n_rows % C::ROWS != 0 || NS != 1) return cudaErrorNotSupported;
   } else if (q.G % 8 != 0 || q.G < C::GPU) {
     return cudaErrorNotSupported;
   }
@@ -902,17 +1047,17 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   Params p{};
   p.q = q;
   p.upt = (q.G + C::GPU - 1) / C::GPU;
-  p.ntiles_e = (int)((q.n_rows + 15) / 16);
+  p.ntiles_e = (int)((q.n_rows + C::ROWS - 1) / C::ROWS);
   p.CH = C::CH;
-  p.tx = (uint32_t)(NS * C::CODE_BYTES + NS * (SB1 ? 2 * 32 * q.G : 2 * C::SB_BYTES));
+  p.tx = (uint32_t)(NS * C::CODE_BYTES + NS * (SB1 ? 4 * C::ROWS * q.G : 2 * C::SB_BYTES));
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
   // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums | plan]
-  const size_t part = C::ONE ? (size_t)kRB * C::KC * NS * 16 * 4 : (size_t)kRB * C::KC * NS * C::MT * 32 * 16;
+  const size_t part = C::ONE ? (size_t)C::RB * C::KC * NS * 16 * 4 : (size_t)C::RB * C::KC * NS * C::MT * 32 * 16;
   const size_t xs = align128((size_t)C::CH * p.tok_stride);
   const size_t xsum = align128((size_t)Gpad * C::TOKP * 16);  // float4 records
-  const size_t bars = 8 * (2 * kMaxStages + 2 * kRB);
+  const size_t bars = 8 * (2 * kMaxStages + 2 * C::RB);
   const size_t plan = align128((size_t)(5 * q.num_experts + 1 + 2 * q.n_pairs) * sizeof(int));
   if (plan > 32 * 1024) return cudaErrorNotSupported;
   auto total = [&](int stages) {
@@ -937,7 +1082,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
 
   CUtensorMap tm[6];
   for (int ns = 0; ns < NS; ++ns) {
-    if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z)) return cudaErrorNotSupported;
+    if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z, C::ROWS)) return cudaErrorNotSupported;
     if (SB1) {  // no scale/bias maps: 1-D bulk copies
       tm[3 * ns + 1] = tm[3 * ns];
       tm[3 * ns + 2] = tm[3 * ns];
@@ -983,7 +1128,7 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
   using L = Lanes<BITS, GS>;
   if constexpr (L::kOk) {
     constexpr int WPG = L::kWordsPerGroup;
-    constexpr int UB = WPG >= 32 ? 16 : 32;  // base unit
+    constexpr int UB = WPG > 16 ? 16 : 32;   // base unit (at most 16 slices)
     constexpr int UW = WPG <= 8 ? 64 : UB;   // wide unit: 4 groups per consumer
     if (dual) {
       if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 2, true>(q, st);
