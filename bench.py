@@ -485,7 +485,8 @@ def _gbs(nbytes, ms, hbm_peak):
 def run_secondary(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
     out = {}
     for name, fn in (("moe", secondary_moe), ("sweep", secondary_sweep),
-                     ("prefill", secondary_prefill), ("moe_prefill", secondary_moe_prefill)):
+                     ("prefill", secondary_prefill), ("moe_prefill", secondary_moe_prefill),
+                     ("other_layouts", secondary_other_layouts)):
         try:
             out[name] = fn(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust)
         except Exception as e:  # pragma: no cover
@@ -623,6 +624,68 @@ def secondary_prefill(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sus
     return out
 
 
+def _rotating(torch, call, make, nbytes, stream):
+    """per-call device time (ms) of `call(item)` over copies of `make()` whose
+    rotation reads more than 3x L2 between reuses"""
+    items = [make() for _ in range(copies_for(nbytes))]
+
+    def fn():
+        for it in items:
+            call(it)
+    t = time_graph(torch, fn, stream, reps=10, inner=1) / len(items)
+    del items
+    return t
+
+
+def secondary_other_layouts(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16_sust):
+    """one-token decode in the other weight formats: the [K, N] layout
+    (transpose = 0), per-tensor int8, the microscaled modes, and a fused
+    three-part projection (4-bit q, 4-bit k, 6-bit v sharing K)"""
+    out = {}
+    K = 4096
+    x = wl.gen_x(1, K, 7001).to(dev)
+    for N in (4096, 14336):
+        w = wl.gen_weight(K, N, 7002 + N).to(dev)
+        qw = api.qmm_quantize(w, 64, 4, torch.bfloat16)  # stored [K, N]
+        y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        b = K * N // 2 + K * (N // 64) * 4 + 2 * K + 2 * N
+        t = _rotating(torch, lambda q: api.qmm_matmul(x, q, False, out=y, stream=stream),
+                      lambda: clone_qw(api, qw), b, stream)
+        out[f"transpose0_{K}x{N}"] = _gbs(b, t, hbm_peak)
+        del w, qw
+    for N in (4096, 14336):
+        q, prm = api.qmm_quantize_dynamic_int8(wl.gen_weight(N, K, 7003 + N).to(dev))
+        y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        b = N * K + 2 * K + 2 * N
+        t = _rotating(torch, lambda qq: api.qmm_matmul_dynamic_int8(x, qq, prm, out=y, stream=stream),
+                      lambda: q.clone(), b, stream)
+        out[f"int8_per_tensor_{N}x{K}"] = _gbs(b, t, hbm_peak)
+        del q
+    N = 14336
+    for name, mode in (("mxfp4", api.QMM_MODE_MXFP4), ("mxfp8", api.QMM_MODE_MXFP8), ("nvfp4", api.QMM_MODE_NVFP4)):
+        bits, gs = api.MX_PARAMS[mode]
+        g = torch.Generator(device=dev)
+        g.manual_seed(7004 + mode)
+        packed = torch.randint(-2**31, 2**31 - 1, (N, K * bits // 32), dtype=torch.int32, device=dev, generator=g)
+        lo, hi = (0x20, 0x50) if mode == api.QMM_MODE_NVFP4 else (110, 130)
+        sc = torch.randint(lo, hi, (N, K // gs), dtype=torch.uint8, device=dev, generator=g)
+        y = torch.empty(1, N, dtype=torch.bfloat16, device=dev)
+        b = N * K * bits // 8 + N * (K // gs) + 2 * K + 2 * N
+        t = _rotating(torch, lambda q: api.qmm_matmul(x, q, True, out=y, stream=stream),
+                      lambda: api.mx_qweight(packed.clone(), sc.clone(), mode, N, K), b, stream)
+        out[f"{name}_{N}x{K}"] = _gbs(b, t, hbm_peak)
+        del packed, sc
+    parts = [api.qmm_quantize(wl.gen_weight(4096, K, 7010).to(dev), 64, 4, torch.bfloat16),
+             api.qmm_quantize(wl.gen_weight(1024, K, 7011).to(dev), 64, 4, torch.bfloat16),
+             api.qmm_quantize(wl.gen_weight(1024, K, 7012).to(dev), 64, 6, torch.bfloat16)]
+    y = torch.empty(1, 6144, dtype=torch.bfloat16, device=dev)
+    b = sum(p.rows * K * p.bits // 8 + p.rows * (K // 64) * 4 for p in parts) + 2 * K + 2 * 6144
+    t = _rotating(torch, lambda ps: api.qmm_matmul_parts(x, ps, out=y, stream=stream),
+                  lambda: [clone_qw(api, p) for p in parts], b, stream)
+    out["fused_parts_q4096_k1024_v1024b6"] = _gbs(b, t, hbm_peak)
+    return out
+
+
 # ---------------------------------------------------------------- oracle arms
 def cpu_threads():
     try:
@@ -754,6 +817,14 @@ def run_profile(args):
                               torch.bfloat16)
         x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
         fn = lambda: api.qmm_matmul(x, qw)  # noqa: E731
+    elif name.startswith("moe_down"):
+        # the down projection of a one-token MoE step: 8 pairs, K = 768
+        case = [d for d in wl.WORKLOADS.moe if d.name == name.replace("moe_down", "moe")][0]
+        E, dff, dm, T, k = case.num_experts, case.d_ff, case.d_model, case.tokens, case.top_k
+        d = api.ExpertStack.from_qweight(api.qmm_quantize(wl.gen_weight(E * dm, dff, case.seed + 2).to(dev), 64, 4, torch.bfloat16), E)
+        h = wl.gen_x(T * k, dff, case.seed + 5).to(dev).reshape(-1)
+        ids = wl.gen_moe_ids(T, E, k, case.seed + 4).to(dev).reshape(-1)
+        fn = lambda: api.qmm_moe_gemv_id(h, ids, T * k, dff, d)  # noqa: E731
     elif name.startswith("moe"):
         case = [d for d in wl.WORKLOADS.moe if d.name == name][0]
         E, dff, dm, T, k = case.num_experts, case.d_ff, case.d_model, case.tokens, case.top_k

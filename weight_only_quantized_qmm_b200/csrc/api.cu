@@ -19,6 +19,8 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
 cudaError_t launch_dequantize_mx(const qmm_qweight* w, void* out, int out_dtype, cudaStream_t st);
 cudaError_t launch_matmul_mx(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
                              int64_t ldy, int y_dtype, cudaStream_t st);
+cudaError_t launch_qgemv_t0(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
+                            int64_t ldy, int y_dtype, cudaStream_t st);
 cudaError_t launch_quantize_dyn8(const void* w, int w_dtype, int64_t n, int8_t* q, float* params, cudaStream_t st);
 cudaError_t launch_dequantize_dyn8(const int8_t* q, int64_t n, const float* params, void* out, int out_dtype,
                                    cudaStream_t st);
@@ -200,6 +202,10 @@ static qmm_status matmul_dispatch(const void* x, qmm_dtype x_dtype, int64_t M, i
   }
   if (transpose && half_types) {  // M > 16: tcgen05 tensor-core GEMM
     const cudaError_t e = qmm::launch_qgemm_tc(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
+    if (e != cudaErrorNotSupported) return launch_status(e);
+  }
+  if (!transpose) {  // [K, N] weights, few tokens, whole-word codes
+    const cudaError_t e = qmm::launch_qgemv_t0(x, x_dtype, M, K, w, y, ldy, y_dtype, st);
     if (e != cudaErrorNotSupported) return launch_status(e);
   }
   return launch_status(qmm::launch_generic(x, x_dtype, M, K, w, transpose, y, ldy, y_dtype, st));

@@ -116,7 +116,17 @@ dequant_kernel(const int8_t* __restrict__ q, int64_t n, const float* __restrict_
   }
 }
 
-constexpr int kTok = 8;  // tokens per pass
+constexpr int kTok = 8;    // tokens per pass
+constexpr int kBatch = 8;  // 16-byte weight chunks a lane requests at once
+
+// 16 bytes read once: not kept in L1
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
 // byte j of w (already XOR-ed with 0x80) as a float: 2^23 + u, minus 2^23
 template <int J>
@@ -167,8 +177,22 @@ matmul_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const int8_t* __re
       for (int t = 0; t < kTok; ++t) acc[t] = 0.0f;
       const int8_t* row = q + n * K;
       if (VEC) {
-        for (int64_t c = lane; c < K / 16; c += 32) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + c);
+        // kBatch 16-byte chunks per lane are requested before any of them is
+        // used, so that a warp keeps up to kBatch * 512 bytes of its row in
+        // flight
+        const int64_t nch = K / 16;
+        for (int64_t cb = 0; cb < nch; cb += 32 * kBatch) {
+          uint4 vb[kBatch];
+#pragma unroll
+          for (int j = 0; j < kBatch; ++j) {
+            const int64_t c = cb + lane + 32 * j;
+            vb[j] = c < nch ? ld_stream(reinterpret_cast<const uint4*>(row) + c) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int jb = 0; jb < kBatch; ++jb) {
+          const int64_t c = cb + lane + 32 * jb;
+          if (c < nch) {
+          const uint4 v = vb[jb];
           const uint32_t wv[4] = {v.x ^ 0x80808080u, v.y ^ 0x80808080u, v.z ^ 0x80808080u, v.w ^ 0x80808080u};
           float u[16];
 #pragma unroll
@@ -197,6 +221,8 @@ matmul_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const int8_t* __re
                 acc[t] = fmaf(xv.w, u[j + 3], acc[t]);
               }
             }
+          }
+          }
           }
         }
       } else {
