@@ -586,7 +586,7 @@ def secondary_moe_prefill(torch, api, wl, dev, stream, hbm_peak, bf16_peak, bf16
         ids = wl.gen_moe_ids(T, E, k, 4602 + T).to(dev)
         a = wl.gen_x(T, dm, 4603 + T).to(dev)
         h = wl.gen_x(P, dff, 4604 + T).to(dev)
-        ws = api.moe_workspace(P, E, dev)
+        ws = api.moe_workspace(P, E, dev, n_cols=max(dm, dff))  # with room for the gathered rows
         og = torch.empty(P, dff, dtype=torch.bfloat16, device=dev)
         od = torch.empty(P, dm, dtype=torch.bfloat16, device=dev)
         t_r = time_graph(torch, lambda: api.qmm_moe_compute_ids_tpe(ids, E, ws, stream=stream), stream,

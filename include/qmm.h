@@ -323,6 +323,12 @@ qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype
  *                     pairs with an id outside [0, E) come last
  *   blk_e[nb] (pad), blk_s[nb] (pad)   expert and first entry of each block,
  *                     nb = ceil(n_pairs / 256) + E entries reserved
+ * Optionally, from the next 256-byte boundary, room for the activation rows
+ * gathered in pair-list order ([n_pairs, K] in a_dtype): a workspace of
+ * qmm_moe_gemm_workspace_bytes_gathered(n_pairs, num_experts, K) bytes lets
+ * qmm_moe_gemm_id copy each pair's row there once (one extra kernel) and
+ * load every tile's rows as one contiguous TMA box, instead of gathering
+ * them 4 rows per copy; same results.
  * A pair whose id is outside [0, E) gets a zero output row and sets
  * QMM_ERR_BAD_EXPERT_ID in *d_status (qmm_moe_compute_ids_tpe).
  * ------------------------------------------------------------------------ */
@@ -330,6 +336,10 @@ qmm_status qmm_moe_gemv_id_gate_up_silu_batched(const void* a, qmm_dtype a_dtype
 /* Workspace bytes for n_pairs pairs over num_experts experts (-1 when
  * n_pairs < 0, num_experts outside [1, 8192], or n_pairs > 2^30 - 1). */
 int64_t qmm_moe_gemm_workspace_bytes(int64_t n_pairs, int64_t num_experts);
+
+/* Workspace bytes that also hold the gathered activation rows of K = n_cols
+ * 16-bit columns (-1 for the cases above or n_cols outside [1, 2^24]). */
+int64_t qmm_moe_gemm_workspace_bytes_gathered(int64_t n_pairs, int64_t num_experts, int64_t n_cols);
 
 /* Routing (compute_ids_tpe): ids is device int32[n_pairs] (the [batch, top_k]
  * routing table, row-major).  Writes the workspace fields above; one CTA.
@@ -349,9 +359,10 @@ qmm_status qmm_moe_compute_ids_tpe(const int32_t* ids, int64_t n_pairs, int64_t 
  * Errors: INVALID_ARG (shapes, ne11 not 1 or top_k, workspace too small),
  * DTYPE, UNSUPPORTED (f32 activations, device), ALIGNMENT (a and out
  * 16-byte aligned, workspace 4-byte aligned), CUDA.  A device-side timeout
- * writes the affected tiles as NaN. */
+ * writes the affected tiles as NaN.  The call writes the workspace only in
+ * the gathered-rows region, when the workspace has one. */
 qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int64_t top_k,
-                           int64_t ne11, const void* workspace, int64_t workspace_bytes,
+                           int64_t ne11, void* workspace, int64_t workspace_bytes,
                            const qmm_expert_stack* w, void* out, qmm_dtype out_dtype,
                            void* stream);
 

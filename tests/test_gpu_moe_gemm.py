@@ -60,7 +60,7 @@ def test_routing_workspace(batch, top_k, E):
     assert int(status.item()) == 0
 
 
-def _moe_gemm_case(batch, top_k, ne11, E, n_rows, n_cols, bits, gs, dtype, seed, bad=()):
+def _moe_gemm_case(batch, top_k, ne11, E, n_rows, n_cols, bits, gs, dtype, seed, bad=(), gathered=False):
     st, ost = make_stack(E, n_rows, n_cols, bits, gs, seed, dtype)
     ids = wl.gen_moe_ids(batch, E, top_k, seed + 1)
     for (t, k) in bad:
@@ -68,7 +68,7 @@ def _moe_gemm_case(batch, top_k, ne11, E, n_rows, n_cols, bits, gs, dtype, seed,
     P = batch * top_k
     dts = {torch.bfloat16: "bf16", torch.float16: "f16"}[dtype]
     a = wl.gen_x(batch * ne11, n_cols, seed + 2, dts)
-    ws = api.moe_workspace(P, E)
+    ws = api.moe_workspace(P, E, n_cols=n_cols if gathered else None)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     g32, g16 = Guarded((P, n_rows), torch.float32), Guarded((P, n_rows), dtype)
     api.qmm_moe_compute_ids_tpe(ids.to(DEV), E, ws, status)
@@ -83,12 +83,22 @@ def _moe_gemm_case(batch, top_k, ne11, E, n_rows, n_cols, bits, gs, dtype, seed,
 
 @pytest.mark.parametrize("bits,gs", [(4, 64), (8, 32), (3, 128), (2, 64), (6, 64)])
 @pytest.mark.parametrize("ne11", [1, 4])
-def test_moe_gemm_widths_and_layouts(bits, gs, ne11):
+@pytest.mark.parametrize("gathered", [False, True])
+def test_moe_gemm_widths_and_layouts(bits, gs, ne11, gathered):
     out32, out16, ref, rc, st, _ = _moe_gemm_case(70, 4, ne11, 12, 200, 256, bits, gs, torch.bfloat16,
-                                                  800 + bits + gs + ne11)
+                                                  800 + bits + gs + ne11, gathered=gathered)
     assert rc == oracle.ORC_OK and st == 0
     gate(out32.cpu().numpy(), ref, f"moe gemm b{bits} g{gs} ne11={ne11}")
     rne_equal(out16, out32)
+
+
+def test_moe_gemm_gathered_rows_give_the_same_bits():
+    """the workspace with room for the gathered rows changes how the rows
+    reach the tile, not the arithmetic: both paths agree bit for bit"""
+    a32, a16, *_ = _moe_gemm_case(300, 8, 1, 128, 256, 512, 4, 64, torch.bfloat16, 880)
+    b32, b16, *_ = _moe_gemm_case(300, 8, 1, 128, 256, 512, 4, 64, torch.bfloat16, 880, gathered=True)
+    assert torch.equal(a32.view(torch.int32), b32.view(torch.int32))
+    assert torch.equal(a16.view(torch.int16), b16.view(torch.int16))
 
 
 def test_moe_gemm_fp16_and_many_blocks_per_expert():
@@ -101,7 +111,7 @@ def test_moe_gemm_fp16_and_many_blocks_per_expert():
 
 def test_moe_gemm_bad_ids_zero_rows_and_status():
     bad = [(3, 1), (10, 0), (11, 3)]
-    out32, _, ref, rc, st, ids = _moe_gemm_case(40, 4, 4, 8, 128, 256, 4, 64, torch.bfloat16, 870, bad)
+    out32, _, ref, rc, st, ids = _moe_gemm_case(40, 4, 4, 8, 128, 256, 4, 64, torch.bfloat16, 870, bad, gathered=True)
     assert rc == oracle.ORC_ERR_ID and st & 7 == 7
     o = out32.cpu().numpy()
     for (t, k) in bad:
@@ -120,7 +130,7 @@ def test_moe_prefill_full_size(T):
     ids = wl.gen_moe_ids(T, E, k, 4502 + T)
     a = wl.gen_x(T, dm, 4503 + T)
     P = T * k
-    ws = api.moe_workspace(P, E)
+    ws = api.moe_workspace(P, E, n_cols=dm)  # room for the gathered rows of either projection
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     gg = Guarded((P, dff), torch.float32)
     api.qmm_moe_compute_ids_tpe(ids.to(DEV), E, ws, status)

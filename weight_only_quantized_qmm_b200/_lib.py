@@ -32,7 +32,7 @@ EXPORTS = (
     "qmm_moe_gemv_id_gate_up_silu_batched", "qmm_moe_gemm_workspace_bytes",
     "qmm_moe_compute_ids_tpe", "qmm_moe_gemm_id", "qmm_moe_gemm_id_noalloc",
     "qmm_selftest_bounded_wait", "qmm_matmul_parts", "qmm_quantize_dynamic_int8",
-    "qmm_dequantize_dynamic_int8", "qmm_matmul_dynamic_int8",
+    "qmm_dequantize_dynamic_int8", "qmm_matmul_dynamic_int8", "qmm_moe_gemm_workspace_bytes_gathered",
 )
 
 
@@ -94,6 +94,8 @@ def load() -> ctypes.CDLL:
     L.qmm_moe_gemv_id_gate_up_silu_batched.restype = c_int
     L.qmm_moe_gemm_workspace_bytes.argtypes = [i64, i64]
     L.qmm_moe_gemm_workspace_bytes.restype = i64
+    L.qmm_moe_gemm_workspace_bytes_gathered.argtypes = [i64, i64, i64]
+    L.qmm_moe_gemm_workspace_bytes_gathered.restype = i64
     L.qmm_moe_compute_ids_tpe.argtypes = [vp, i64, i64, vp, i64, vp, vp]
     L.qmm_moe_compute_ids_tpe.restype = c_int
     L.qmm_moe_gemm_id.argtypes = [vp, c_int, i64, i64, i64, vp, i64, stp, vp, c_int, vp]

@@ -440,9 +440,18 @@ def qmm_moe_gemm_workspace_bytes(n_pairs: int, num_experts: int) -> int:
     return int(_lib.load().qmm_moe_gemm_workspace_bytes(n_pairs, num_experts))
 
 
-def moe_workspace(n_pairs: int, num_experts: int, device=None) -> torch.Tensor:
-    """A device workspace of the size qmm_moe_compute_ids_tpe needs (int32)."""
-    nb = qmm_moe_gemm_workspace_bytes(n_pairs, num_experts)
+def qmm_moe_gemm_workspace_bytes_gathered(n_pairs: int, num_experts: int, n_cols: int) -> int:
+    return int(_lib.load().qmm_moe_gemm_workspace_bytes_gathered(n_pairs, num_experts, n_cols))
+
+
+def moe_workspace(n_pairs: int, num_experts: int, device=None, n_cols: int | None = None) -> torch.Tensor:
+    """A device workspace of the size qmm_moe_compute_ids_tpe needs (int32);
+    with n_cols, also room for the activation rows gathered in pair order
+    (the GEMM then loads each tile's rows as one box)."""
+    if n_cols is None:
+        nb = qmm_moe_gemm_workspace_bytes(n_pairs, num_experts)
+    else:
+        nb = qmm_moe_gemm_workspace_bytes_gathered(n_pairs, num_experts, n_cols)
     if nb < 0:
         check("qmm_moe_gemm_workspace_bytes", _lib.QMM_ERR_INVALID_ARG)
     return torch.empty((nb + 3) // 4, dtype=torch.int32, device=device or "cuda")

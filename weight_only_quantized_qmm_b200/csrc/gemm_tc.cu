@@ -165,6 +165,10 @@ struct GemmParams {
   const int32_t* ws_blk_e;  // expert of block b
   const int32_t* ws_blk_s;  // first entry (into ws_pairs) of block b
   int E, top_k, ne11, n_pairs;
+  // MoE: the activation rows already gathered in pair-list order (row i of
+  // the x map is the row of the pair listed at entry i), so a tile's rows
+  // are one contiguous box; 0: the producer gathers them 4 at a time
+  int xg;
 };
 
 // ------------------------------------------------------------------ dequant helpers
@@ -332,7 +336,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
       const TileOf tl = tile_of<MOE>(p, lt, m_tiles, n_tiles);
       const int wrow0 = tl.e * p.N + tl.n0;  // first row of the (stacked) weight matrix
       int rw[8];
-      if constexpr (MOE) {
+      if (MOE && !p.xg) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) rw[q] = moe_a_row(p, tl, 8 * lane + q);
       }
@@ -366,7 +370,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
           break;
         }
         constexpr uint32_t kTx = kXStage + PL::CODE_STAGE;
-        if constexpr (MOE) {
+        if (MOE && !p.xg) {
           if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, kTx);
           __syncwarp();
           const uint32_t d = su32(xs + s * kXStage) + (uint32_t)(lane * 8 * 128);
@@ -766,13 +770,16 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
 cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const qmm_expert_stack* w,
                              const int32_t* ws_off, const int32_t* ws_args, const int32_t* ws_pairs,
                              const int32_t* ws_blk_e, const int32_t* ws_blk_s, int top_k, int ne11,
-                             int n_pairs, void* out, int out_dtype, cudaStream_t st) {
+                             int n_pairs, const void* xg, void* out, int out_dtype, cudaStream_t st) {
   const int64_t K = w->n_cols;
   if (a_rows > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->n_rows * w->num_experts > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
-  CUtensorMap tm[4];  // x: one-row boxes (the producer gathers 4 rows per copy)
-  if (!make_x_map(&tm[0], a, a_dtype, a_rows, K, 1)) return cudaErrorNotSupported;
+  // x: 256-row boxes over the gathered rows, or one-row boxes over `a` (the
+  // producer gathers 4 rows per copy)
+  CUtensorMap tm[4];
+  if (xg ? !make_x_map(&tm[0], xg, a_dtype, n_pairs, K, gemm::kBN) : !make_x_map(&tm[0], a, a_dtype, a_rows, K, 1))
+    return cudaErrorNotSupported;
   const bool tw = make_w_maps(&tm[1], &tm[2], &tm[3], w->packed, w->scales, w->biases,
                               w->n_rows * w->num_experts, K * w->bits / 32, K / w->group_size, w->bits);
   if (!tw) tm[1] = tm[2] = tm[3] = tm[0];
@@ -797,6 +804,7 @@ cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const q
   prm.top_k = top_k;
   prm.ne11 = ne11;
   prm.n_pairs = n_pairs;
+  prm.xg = xg != nullptr;
   // the work list is known only on the device: one CTA per SM
   const int grid = qmm_host::num_sms();
   if (a_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, true>(w->bits, w->group_size, tw, prm, tm, grid, st);

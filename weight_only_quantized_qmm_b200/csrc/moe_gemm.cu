@@ -31,7 +31,7 @@ namespace qmm {
 cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const qmm_expert_stack* w,
                              const int32_t* ws_off, const int32_t* ws_args, const int32_t* ws_pairs,
                              const int32_t* ws_blk_e, const int32_t* ws_blk_s, int top_k, int ne11,
-                             int n_pairs, void* out, int out_dtype, cudaStream_t st);
+                             int n_pairs, const void* xg, void* out, int out_dtype, cudaStream_t st);
 
 constexpr int kMoeBlock = 256;         // pairs per GEMM block (the tile's token columns)
 constexpr int kRouteThreads = 1024;
@@ -137,6 +137,32 @@ moe_route_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int32_t* _
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Byte offset (from the workspace start) of the gathered activation rows,
+// and the workspace bytes with them: 256-byte aligned rows region after the
+// schedule.
+constexpr int64_t moe_xg_offset(int64_t n_pairs, int64_t E) { return (moe_ws_layout(n_pairs, E).total * 4 + 255) / 256 * 256; }
+constexpr int64_t moe_xg_bytes(int64_t n_pairs, int64_t E, int64_t K) {
+  return moe_xg_offset(n_pairs, E) + n_pairs * K * 2;
+}
+
+// xg[i, :] = a[row(pairs[i]), :] for every entry i of the pair list (the
+// schedule's order), one warp per row, 16-byte copies (K * 2 % 16 == 0).
+__global__ void __launch_bounds__(256)
+moe_gather_kernel(const uint4* __restrict__ a, const int32_t* __restrict__ pairs, int n_pairs, int top_k, int ne11,
+                  int K, uint4* __restrict__ xg) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int vpr = K * 2 / 16;  // 16-byte vectors per row
+  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n_pairs; i += gridDim.x * (blockDim.x >> 5)) {
+    const int pr = __ldg(pairs + i);
+    const int64_t row = ne11 == 1 ? pr / top_k : pr;
+    const uint4* src = a + row * vpr;
+    uint4* dst = xg + (int64_t)i * vpr;
+    for (int v = lane; v < vpr; v += 32) dst[v] = __ldg(src + v);
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace qmm
 
 using qmm::MoeWs;
@@ -208,8 +234,13 @@ qmm_status qmm_moe_compute_ids_tpe(const int32_t* ids, int64_t n_pairs, int64_t 
   return route(ids, n_pairs, num_experts, workspace, workspace_bytes, d_status, (cudaStream_t)stream);
 }
 
+int64_t qmm_moe_gemm_workspace_bytes_gathered(int64_t n_pairs, int64_t num_experts, int64_t n_cols) {
+  if (qmm_moe_gemm_workspace_bytes(n_pairs, num_experts) < 0 || n_cols < 1 || n_cols > (int64_t)1 << 24) return -1;
+  return qmm::moe_xg_bytes(n_pairs, num_experts, n_cols);
+}
+
 qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int64_t top_k, int64_t ne11,
-                           const void* workspace, int64_t workspace_bytes, const qmm_expert_stack* w, void* out,
+                           void* workspace, int64_t workspace_bytes, const qmm_expert_stack* w, void* out,
                            qmm_dtype out_dtype, void* stream) {
   qmm_status s = check_moe_gemm_stack(w);
   if (s != QMM_OK) return s;
@@ -228,9 +259,29 @@ qmm_status qmm_moe_gemm_id(const void* a, qmm_dtype a_dtype, int64_t batch, int6
   s = qmm_device_check();
   if (s != QMM_OK) return s;
   const int32_t* ws = static_cast<const int32_t*>(workspace);
+  cudaStream_t st = (cudaStream_t)stream;
+  // a workspace with room for the gathered rows: copy them once in the
+  // schedule's order, so that the GEMM loads each tile's rows as one box
+  void* xg = nullptr;
+  if (workspace_bytes >= qmm::moe_xg_bytes(n_pairs, w->num_experts, w->n_cols)) {
+    xg = static_cast<char*>(workspace) + qmm::moe_xg_offset(n_pairs, w->num_experts);
+    if ((reinterpret_cast<uintptr_t>(xg) & 15) != 0) return QMM_ERR_ALIGNMENT;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<int64_t>((n_pairs + 7) / 8, (int64_t)qmm_host::num_sms() * 8));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, qmm::moe_gather_kernel, static_cast<const uint4*>(a), ws + L.pairs, (int)n_pairs,
+                           (int)top_k, (int)ne11, (int)w->n_cols, static_cast<uint4*>(xg)) != cudaSuccess)
+      return QMM_ERR_CUDA;
+  }
   const cudaError_t e =
       qmm::launch_qgemm_moe(a, a_dtype, batch * ne11, w, ws + L.off, ws + L.args, ws + L.pairs, ws + L.blk_e,
-                            ws + L.blk_s, (int)top_k, (int)ne11, (int)n_pairs, out, out_dtype, (cudaStream_t)stream);
+                            ws + L.blk_s, (int)top_k, (int)ne11, (int)n_pairs, xg, out, out_dtype, st);
   if (e == cudaErrorNotSupported) return QMM_ERR_UNSUPPORTED;
   return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
 }
@@ -304,7 +355,7 @@ extern "C" qmm_status qmm_moe_gemm_id_noalloc(const void* a, qmm_dtype a_dtype, 
   const MoeWs L = qmm::moe_ws_layout(n_pairs, w->num_experts);
   const cudaError_t e =
       qmm::launch_qgemm_moe(a, a_dtype, batch * ne11, w, ws + L.off, ws + L.args, ws + L.pairs, ws + L.blk_e,
-                            ws + L.blk_s, (int)top_k, (int)ne11, (int)n_pairs, out, out_dtype, st);
+                            ws + L.blk_s, (int)top_k, (int)ne11, (int)n_pairs, nullptr, out, out_dtype, st);
   if (e == cudaErrorNotSupported) return QMM_ERR_UNSUPPORTED;
   return e == cudaSuccess ? QMM_OK : QMM_ERR_CUDA;
 }
