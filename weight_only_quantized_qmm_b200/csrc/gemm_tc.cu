@@ -497,9 +497,12 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
         // before this stage's copies, whose landing the wait above saw)
         uint32_t cw[2 * B];
         const uint32_t crow = su32(cs + s * PL::CODE_STAGE) + (uint32_t)(r * 8 * B);
+        // 16-byte chunk q of the row sits at q ^ f(r) under the map's swizzle
+        // (32-byte rows: f = bit 2 of r; 64-byte rows: f = bits 1..2 of r)
+        const int cf = B == 4 ? (r >> 2) & 1 : B == 8 ? (r >> 1) & 3 : 0;
 #pragma unroll
         for (int q = 0; q < B / 2; ++q) {
-          const uint4 v = lds128(crow + 16 * q);
+          const uint4 v = lds128(crow + 16 * (q ^ cf));
           cw[4 * q] = v.x; cw[4 * q + 1] = v.y; cw[4 * q + 2] = v.z; cw[4 * q + 3] = v.w;
         }
         T cs_[NGS], cb_[NGS];
@@ -704,8 +707,13 @@ static bool make_w_maps(CUtensorMap* tc, CUtensorMap* ts, CUtensorMap* tb, const
     const cuuint64_t dims[2] = {(cuuint64_t)wpr, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(wpr * 4)};
     const cuuint32_t box[2] = {(cuuint32_t)(2 * bits), (cuuint32_t)gemm::kBM};
+    // rows of 32 or 64 bytes are swizzled at their width, so that the eight
+    // rows a quarter warp reads at one chunk fall in different banks
+    const CUtensorMapSwizzle swz = bits == 4 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                   : bits == 8 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_NONE;
     if (enc(tc, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(packed), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return false;
   }

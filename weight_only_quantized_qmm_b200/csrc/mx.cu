@@ -11,7 +11,9 @@
 // Kernels: the standalone dequantization (bit-exact: one fp32 product, one
 // rounding to the output dtype) and a CUDA-core matmul for these modes
 // (fp32 products and sums; one warp per weight row, the lanes splitting K in
-// 32-code chunks, up to 8 tokens per pass).
+// 32-code chunks requested several at a time, each lane decoded by shifts
+// into an exact f16, the group scale applied once per group partial; up to 8
+// tokens per pass).
 #include <algorithm>
 
 #include "common.cuh"
@@ -86,37 +88,122 @@ dequant_mx_kernel(const uint32_t* __restrict__ packed, const uint8_t* __restrict
   for (int i = 0; i < (int)(32 * sizeof(TO) / 16); ++i) dst[i] = v4[i];
 }
 
-constexpr int kMB = 8;  // tokens per pass
+constexpr int kMB = 8;      // tokens per pass
+constexpr int kBatch = 4;   // 32-code chunks a lane requests at once
+constexpr int64_t kXsMax = 128 * 1024;  // shared-memory bytes for staged x
 
-// y[m, n] = sum_k x[m, k] w_hat[n, k]: one warp per row n (grid-stride), lane
-// l takes the 32-lane chunks l, l + 32, ... of the row.
-template <int MODE, typename TX>
+// Lanes of one packed word as exact f16 pairs, scaled by a power of two that
+// the group scale takes back:
+//   E2M1 (4-bit): the code's exponent and mantissa bits under bits 9..11 of
+//     an f16 read as 2^-14 * lane (the exponent bias 15 against E2M1's 1; a
+//     zero exponent field gives the f16 subnormal 2^-15 m, which is
+//     2^-14 * 0.5 m); pair j = codes j and j + 4;
+//   E4M3 (8-bit, the page's decode): the low 7 bits under bits 7..13 of an
+//     f16 read as lane / 256; pair j = codes j and j + 2.
+template <int B>
+__device__ __forceinline__ void lanes_f32(uint32_t w, float* v) {
+  if constexpr (B == 4) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t x = w >> (4 * j);
+      const uint32_t h = ((x << 9) & 0x0E000E00u) | ((x << 12) & 0x80008000u);
+      __half2 hh;
+      memcpy(&hh, &h, 4);
+      const float2 f = __half22float2(hh);
+      v[j] = f.x;
+      v[j + 4] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t x = w >> (8 * j);
+      const uint32_t h = ((x & 0x007F007Fu) << 7) | ((x & 0x00800080u) << 8);
+      __half2 hh;
+      memcpy(&hh, &h, 4);
+      const float2 f = __half22float2(hh);
+      v[j] = f.x;
+      v[j + 2] = f.y;
+    }
+  }
+}
+
+// y[m, n] = sum_k x[m, k] w_hat[n, k]: one warp per row n (grid-stride); lane
+// l takes the 32-code chunks l, l + 32, ..., kBatch of them per request; per
+// group the partial dot sum_k x_k lane_k is taken first and then scaled.
+// XS: x staged in shared memory as fp32.
+template <int MODE, typename TX, bool XS>
 __global__ void __launch_bounds__(256)
 matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ packed,
                  const uint8_t* __restrict__ scales, int64_t N, void* y, int64_t ldy, int y_dtype) {
   using Md = Mode<MODE>;
-  constexpr int B = Md::B, GS = Md::GS;
+  constexpr int B = Md::B, GS = Md::GS, GPC = 32 / GS;  // groups per 32-code chunk
+  constexpr float kLaneUnit = B == 4 ? 16384.0f : 256.0f;
+  extern __shared__ float xs[];  // [kMB][K] when XS
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
   const int64_t chunks = K / 32, wpr = K * B / 32, G = K / GS;
-  for (int64_t n = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); n < N; n += warps) {
-    const uint32_t* row = packed + n * wpr;
-    for (int64_t m0 = 0; m0 < M; m0 += kMB) {
+  for (int64_t m0 = 0; m0 < M; m0 += kMB) {
+    const int mb = (int)(M - m0 < kMB ? M - m0 : kMB);
+    if (XS) {
+      __syncthreads();
+      for (int64_t i = threadIdx.x; i < (int64_t)mb * K; i += blockDim.x) xs[i] = to_f32(x[m0 * K + i]);
+      __syncthreads();
+    }
+    for (int64_t n = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); n < N; n += warps) {
+      const uint32_t* row = packed + n * wpr;
       float acc[kMB];
 #pragma unroll
-      for (int i = 0; i < kMB; ++i) acc[i] = 0.0f;
-      for (int64_t c = lane; c < chunks; c += 32) {
-        uint32_t wr[B];
+      for (int t = 0; t < kMB; ++t) acc[t] = 0.0f;
+      for (int64_t cb = 0; cb < chunks; cb += 32 * kBatch) {
+        uint32_t wv[kBatch][B];
+        uint32_t sb[kBatch];
 #pragma unroll
-        for (int i = 0; i < B; ++i) wr[i] = __ldg(row + c * B + i);
+        for (int j = 0; j < kBatch; ++j) {
+          const int64_t c = cb + lane + 32 * j;
+          const int64_t cc = c < chunks ? c : 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint32_t q = (wr[(i * B) >> 5] >> ((i * B) & 31)) & ((1u << B) - 1u);
-          const int64_t k = c * 32 + i;
-          const float w = Md::lane(q) * Md::scale(__ldg(scales + n * G + k / GS));
+          for (int q = 0; q < B / 4; ++q) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(row + cc * B) + q);
+            wv[j][4 * q] = v.x; wv[j][4 * q + 1] = v.y; wv[j][4 * q + 2] = v.z; wv[j][4 * q + 3] = v.w;
+          }
+          sb[j] = GPC == 1 ? (uint32_t)__ldg(scales + n * G + cc)
+                           : (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(scales + n * G) + cc);
+        }
 #pragma unroll
-          for (int t = 0; t < kMB; ++t)
-            if (m0 + t < M) acc[t] = fmaf(to_f32(x[(m0 + t) * K + k]), w, acc[t]);
+        for (int j = 0; j < kBatch; ++j) {
+          const int64_t c = cb + lane + 32 * j;
+          if (c < chunks) {
+            float lv[32];
+#pragma unroll
+            for (int q = 0; q < B; ++q) lanes_f32<B>(wv[j][q], lv + q * (32 / B));
+            float sc[GPC];
+#pragma unroll
+            for (int gi = 0; gi < GPC; ++gi) sc[gi] = Md::scale(sb[j] >> (8 * gi)) * kLaneUnit;
+#pragma unroll
+            for (int t = 0; t < kMB; ++t) {
+              if (t < mb) {
+#pragma unroll
+                for (int gi = 0; gi < GPC; ++gi) {
+                  float part = 0.0f;
+#pragma unroll
+                  for (int i = gi * GS; i < (gi + 1) * GS; i += 4) {
+                    float4 xv;
+                    if (XS) {
+                      xv = *reinterpret_cast<const float4*>(xs + t * K + c * 32 + i);
+                    } else {
+                      const TX* xp = x + (m0 + t) * K + c * 32 + i;
+                      xv = make_float4(to_f32(xp[0]), to_f32(xp[1]), to_f32(xp[2]), to_f32(xp[3]));
+                    }
+                    part = fmaf(xv.x, lv[i], part);
+                    part = fmaf(xv.y, lv[i + 1], part);
+                    part = fmaf(xv.z, lv[i + 2], part);
+                    part = fmaf(xv.w, lv[i + 3], part);
+                  }
+                  acc[t] = fmaf(sc[gi], part, acc[t]);
+                }
+              }
+            }
+          }
         }
       }
 #pragma unroll
@@ -125,8 +212,7 @@ matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t*
         for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
       }
       if (lane == 0)
-        for (int t = 0; t < kMB; ++t)
-          if (m0 + t < M) store_as(y, y_dtype, (m0 + t) * ldy + n, acc[t]);
+        for (int t = 0; t < mb; ++t) store_as(y, y_dtype, (m0 + t) * ldy + n, acc[t]);
     }
   }
 }
@@ -146,20 +232,31 @@ static cudaError_t dequant_m(const qmm_qweight* w, void* out, int out_dtype, cud
   return cudaGetLastError();
 }
 
+template <int MODE, typename TX>
+static cudaError_t matmul_x(const TX* x, int64_t M, int64_t K, const qmm_qweight* w, void* y, int64_t ldy,
+                            int y_dtype, cudaStream_t st) {
+  auto S = reinterpret_cast<const uint8_t*>(w->scales);
+  const int64_t N = w->rows;
+  const bool xs = (M < kMB ? M : kMB) * K * 4 <= kXsMax;
+  const size_t smem = xs ? (size_t)(M < kMB ? M : kMB) * K * 4 : 0;
+  const int blocks = (int)std::min<int64_t>((N + 7) / 8, (int64_t)qmm_host::num_sms() * (smem > 64 * 1024 ? 1 : 2));
+  if (xs) {
+    auto k = matmul_mx_kernel<MODE, TX, true>;
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kXsMax);
+    if (e != cudaSuccess) return e;
+    k<<<blocks, 256, smem, st>>>(x, M, K, w->packed, S, N, y, ldy, y_dtype);
+  } else {
+    matmul_mx_kernel<MODE, TX, false><<<blocks, 256, 0, st>>>(x, M, K, w->packed, S, N, y, ldy, y_dtype);
+  }
+  return cudaGetLastError();
+}
+
 template <int MODE>
 static cudaError_t matmul_m(const void* x, int x_dtype, int64_t M, int64_t K, const qmm_qweight* w, void* y,
                             int64_t ldy, int y_dtype, cudaStream_t st) {
-  auto S = reinterpret_cast<const uint8_t*>(w->scales);
-  const int64_t N = w->rows;
-  const int blocks = (int)std::min<int64_t>((N + 7) / 8, 148 * 8);
-  if (x_dtype == QMM_F32)
-    matmul_mx_kernel<MODE, float><<<blocks, 256, 0, st>>>((const float*)x, M, K, w->packed, S, N, y, ldy, y_dtype);
-  else if (x_dtype == QMM_BF16)
-    matmul_mx_kernel<MODE, __nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16*)x, M, K, w->packed, S,
-                                                                  N, y, ldy, y_dtype);
-  else
-    matmul_mx_kernel<MODE, __half><<<blocks, 256, 0, st>>>((const __half*)x, M, K, w->packed, S, N, y, ldy, y_dtype);
-  return cudaGetLastError();
+  if (x_dtype == QMM_F32) return matmul_x<MODE>((const float*)x, M, K, w, y, ldy, y_dtype, st);
+  if (x_dtype == QMM_BF16) return matmul_x<MODE>((const __nv_bfloat16*)x, M, K, w, y, ldy, y_dtype, st);
+  return matmul_x<MODE>((const __half*)x, M, K, w, y, ldy, y_dtype, st);
 }
 
 }  // namespace mx
