@@ -351,21 +351,16 @@ __device__ __forceinline__ void group_dot_rx(const uint32_t (&rawA)[L::kRegs], c
   uint32_t pA[L::kOuts], pB[L::kOuts];
   quarter_pairs<L>(rawA, t, pA);
   quarter_pairs<L>(rawB, t, pB);
-  // even and odd k16 steps in two chains (half the dependent mma latency);
-  // only column 0 (rows g, g + 8: d[0], d[2]) is merged, the others are idle
-  float e[4];
+  // one dependent chain of k16 steps (measured: fewer instructions beat two
+  // shorter chains merged at the end); only column 0 (rows g, g + 8: d[0],
+  // d[2]) is used, the other columns repeat it
 #pragma unroll
   for (int q = 0; q < L::kSteps; ++q) {
     const uint32_t b0 = (q & 1) ? bf[q >> 1].z : bf[q >> 1].x, b1 = (q & 1) ? bf[q >> 1].w : bf[q >> 1].y;
-    float(&acc)[4] = (q & 1) ? e : d;
-    if (q < 2)
-      mma_f16_first(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
+    if (q == 0)
+      mma_f16_first(d, pA[0], pB[0], pA[1], pB[1], b0, b1);
     else
-      mma16816<__half>(acc, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
-  }
-  if constexpr (L::kSteps > 1) {
-    d[0] += e[0];
-    d[2] += e[2];
+      mma16816<__half>(d, pA[2 * q], pB[2 * q], pA[2 * q + 1], pB[2 * q + 1], b0, b1);
   }
 }
 
@@ -544,10 +539,10 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_full + 8 * kMaxStages + 8 * s, KC);
+      mbar_init(bar_full + 8 * kMaxStages + 8 * s, KC * 32);  // every consumer lane arrives
     }
     for (int e = 0; e < C::RB; ++e) {
-      mbar_init(bar_pfull + 8 * e, KC);
+      mbar_init(bar_pfull + 8 * e, KC * 32);
       mbar_init(bar_pempty + 8 * e, 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -838,11 +833,14 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         su = xrec_lane;
       }
     }
-    bool ok = mbar_try_wait(bfull, phase);
-    if (!ok) ok = mbar_wait(bfull, phase, failed);
-    if (__any_sync(0xffffffffu, !ok)) {
-      if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
-      failed = true;
+    // (one poll by every lane is the usual case; the vote keeps the branch
+    // warp-uniform)
+    if (!__all_sync(0xffffffffu, mbar_try_wait(bfull, phase))) {
+      const bool ok = mbar_wait(bfull, phase, failed);
+      if (__any_sync(0xffffffffu, !ok)) {
+        if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
+        failed = true;
+      }
     }
     if (!failed) {
 #pragma unroll
@@ -932,24 +930,29 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bfull + 8 * kMaxStages);  // the slot's `empty` barrier
+    mbar_arrive(bfull + 8 * kMaxStages);  // the slot's `empty` barrier: each lane after its own reads
 
     if (++ku == p.upt) {  // tile done: post this warp's partial
       const int e = jt & (C::RB - 1);
       if (jt >= C::RB) {
-        const bool okp = mbar_wait(bar_pempty + 8 * e, (uint32_t)((jt / C::RB) - 1) & 1u, failed);
-        if (__any_sync(0xffffffffu, !okp)) {
-          if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
-          failed = true;
+        const uint32_t pe = bar_pempty + 8 * e, pp = (uint32_t)((jt / C::RB) - 1) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_try_wait(pe, pp))) {
+          const bool okp = mbar_wait(pe, pp, failed);
+          if (__any_sync(0xffffffffu, !okp)) {
+            if (!failed && lane == 0) set_status(q.d_status, QMM_ERR_TIMEOUT);
+            failed = true;
+          }
         }
       }
 #pragma unroll
       for (int ns = 0; ns < NS; ++ns) {
         if constexpr (C::ONE) {
+          // lane t = 0 of each quad stores rows g and g + 8 (a predicated
+          // store, no divergent region)
+          float* pr = reinterpret_cast<float*>(smem + p.off_part) + ((e * KC + warp) * NS + ns) * 16 + g;
           if (t == 0) {
-            sts32(part_sa + (uint32_t)((((e * KC + warp) * NS + ns) * 16 + g) * 4), acc[ns][0][0]);
-            sts32(part_sa + (uint32_t)((((e * KC + warp) * NS + ns) * 16 + g + 8) * 4), acc[ns][0][2]);
+            pr[0] = acc[ns][0][0];
+            pr[8] = acc[ns][0][2];
           }
         } else {
 #pragma unroll
@@ -962,8 +965,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
           for (int k = 0; k < 4; ++k) acc[ns][mt][k] = 0.0f;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pfull + 8 * e);
+      mbar_arrive(bar_pfull + 8 * e);  // each lane after its own stores
       ku = 0;
       ++jt;
       if constexpr (MOE) {
