@@ -793,6 +793,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[ns][mt][i] = 0.0f;
   bool failed = false;
+  const int gw_end = q.G - gw * GPW;  // this consumer's groups of unit ku start at ku GPU + gw GPW
 
   // unit i: slot i % STAGES with phase (i / STAGES) & 1, k-unit ku of tile jt
   int slot = 0, ku = 0, jt = 0, cur_sg = -1, cur_np = -1;
@@ -845,7 +846,9 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         failed = true;
       }
     }
-    if (!failed) {
+    // (a consumer whose groups of this unit all lie past the row skips it:
+    // they would add exact zeros)
+    if (!failed && (SB1 || ku * GPU < gw_end)) {
 #pragma unroll
       for (int ns = 0; ns < NS; ++ns) {
         const uint32_t csl = cslot + (uint32_t)(ns * C::CODE_BYTES);
@@ -1154,7 +1157,11 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
       if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, UB, 1, true>(q, st);
       return launch_stream<BITS, GS, T, 1, UB, 1, true>(q, st);
     }
-    const bool wide = (q.G % UW) == 0;
+    // wide units also for rows of whole base units past one wide unit (e.g.
+    // K = 14336 at g64: 224 groups, 3.5 wide units): the last unit's groups
+    // past the row read zeros and the consumers holding only those skip it,
+    // which beats twice the units with half the groups per consumer
+    const bool wide = (q.G % UW) == 0 || (q.G > UW && q.G % UB == 0);
     if (q.n_pairs == 1)
       return wide ? launch_stream<BITS, GS, T, 0, UW, 1, false>(q, st) : launch_stream<BITS, GS, T, 0, UB, 1, false>(q, st);
     if (mt == 1)
