@@ -339,3 +339,30 @@ def test_gemv_activation_dynamic_range(bits, M, dtype):
     y = g32.check("y32")
     yref = oracle.matmul(np_storage(x), ORC[dtype], p, s, b, ORC[dtype], N, gs, bits)
     gate(y.cpu().numpy(), yref, f"dynamic range b{bits} M{M}")
+
+
+@pytest.mark.parametrize("bits,gs,M,N,K", [(4, 64, 1, 4096, 4096), (4, 64, 1, 2048, 14336), (4, 64, 5, 2368, 4096),
+                                           (4, 64, 16, 1024, 4096), (2, 128, 1, 2048, 8192), (3, 64, 1, 2048, 4096),
+                                           (6, 64, 3, 2048, 4096), (8, 32, 1, 2048, 4096)])
+def test_gemv_chained_through_x(bits, gs, M, N, K):
+    """A GEMV whose x is the output of the GEMV launched just before it on the
+    stream.  The first one lets its dependents launch early (programmatic
+    dependent launch, after its plan barrier), so the second one runs its
+    prologue and L2 prefetches while the first one still writes x: x must be
+    read only after the first one completes.  Same bits as a call made after
+    a synchronize."""
+    seed = 1200 + 10 * bits + M
+    _, qa, _ = _quant_pair(K, 1024, 4, 64, torch.bfloat16, seed)       # writes x: [M, K]
+    _, qb, _ = _quant_pair(N, K, bits, gs, torch.bfloat16, seed + 1)
+    xa = wl.gen_x(M, 1024, seed + 2).to(DEV)
+    x = torch.empty(M, K, dtype=torch.bfloat16, device=DEV)
+    ys = []
+    for _ in range(3):
+        x.zero_()
+        api.qmm_matmul(xa, qa, True, out=x)
+        ys.append(api.qmm_matmul(x, qb, True, torch.float32))
+    torch.cuda.synchronize()
+    yref = api.qmm_matmul(x, qb, True, torch.float32)
+    torch.cuda.synchronize()
+    for y in ys:
+        assert torch.equal(y, yref)

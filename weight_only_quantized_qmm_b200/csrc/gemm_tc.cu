@@ -94,9 +94,9 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 // instruction descriptor: fp32 accumulator, A/B = bf16 (1) or f16 (0), both K-major
 template <typename T>
-__device__ __forceinline__ uint32_t mma_idesc() {
+__device__ __forceinline__ uint32_t mma_idesc(int n) {  // n: a multiple of 16 in [16, 256]
   constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(gemm::kBN >> 3) << 17) |
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(n >> 3) << 17) |
          ((uint32_t)(gemm::kBM >> 4) << 24);
 }
 __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
@@ -345,6 +345,9 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
 #pragma unroll
         for (int q = 0; q < 8; ++q) rw[q] = moe_a_row(p, tl, 8 * lane + q);
       }
+      // gathered rows: only the tile's (a MoE block often holds far fewer than
+      // 256 pairs), 8 per lane
+      const int ngl = (tl.cnt + 7) / 8;
       for (int i = 0; i < nk; ++i, ++j) {
         const int s = j % kStages, u = j / kStages;
         bool ok = true;
@@ -382,15 +385,18 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
             tma_2d(su32(cs + s * PL::CODE_STAGE), &tmc, i * 2 * B, wrow0, cfull0 + 8 * s);
           }
         }
-        constexpr uint32_t kTx = kXStage;
         if (MOE && !p.xg) {
-          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, kTx);
+          if (lane == 0) mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)(ngl * 8 * 128));
           __syncwarp();
-          const uint32_t d = su32(xs + s * kXStage) + (uint32_t)(lane * 8 * 128);
-          tma_gather4(d, &tmx, i * kBK, rw[0], rw[1], rw[2], rw[3], full0 + 8 * s);
-          tma_gather4(d + 512, &tmx, i * kBK, rw[4], rw[5], rw[6], rw[7], full0 + 8 * s);
+          if (lane < ngl) {
+            const uint32_t d = su32(xs + s * kXStage) + (uint32_t)(lane * 8 * 128);
+            tma_gather4(d, &tmx, i * kBK, rw[0], rw[1], rw[2], rw[3], full0 + 8 * s);
+            tma_gather4(d + 512, &tmx, i * kBK, rw[4], rw[5], rw[6], rw[7], full0 + 8 * s);
+          }
         } else if (lane == 0) {
-          mbar_arrive_expect_tx(full0 + 8 * s, kTx);
+          // one 256-row box (measured: eight 32-row boxes per stage cost a
+          // third of the dense GEMM's throughput)
+          mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
           tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, tl.m0, full0 + 8 * s);
         }
         issued = j + 1;
@@ -409,11 +415,13 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = mma_idesc<T>();
       int j = 0;
       bool stop = false;
       for (int lt = 0; lt < my_tiles && !stop; ++lt) {
         const int b = lt & 1;
+        // N of the tile's MMAs: its token count rounded up to 16 (columns past
+        // the count read rows that are never stored)
+        const uint32_t idesc = mma_idesc<T>(min(kBN, (tile_of<MOE>(p, lt, m_tiles, n_tiles).cnt + 15) & ~15));
         // accumulator b is free once the epilogue has read out tile lt - 2
         if (lt >= 2 && !bar_wait(tfree0 + 8 * b, ((lt >> 1) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
@@ -615,7 +623,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
         failed = __any_sync(0xffffffffu, failed);
       }
       tc_fence_after();
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < (tl.cnt + 31) / 32; ++c) {  // the TMEM columns the tile's tokens use
         uint32_t v[32];
         if (!failed) tmem_ld32(tmem + ((uint32_t)(qq * 32) << 16) + (uint32_t)(b * kBN + c * 32), v);
         if (n < p.N) {
