@@ -92,18 +92,22 @@ def test_moe_gemm_widths_and_layouts(bits, gs, ne11, gathered):
     rne_equal(out16, out32)
 
 
-def test_moe_gemm_gathered_rows_give_the_same_bits():
+@pytest.mark.parametrize("E", [128, 40])
+def test_moe_gemm_gathered_rows_give_the_same_bits(E):
     """the workspace with room for the gathered rows changes how the rows
-    reach the tile, not the arithmetic: both paths agree bit for bit"""
-    a32, a16, *_ = _moe_gemm_case(300, 8, 1, 128, 256, 512, 4, 64, torch.bfloat16, 880)
-    b32, b16, *_ = _moe_gemm_case(300, 8, 1, 128, 256, 512, 4, 64, torch.bfloat16, 880, gathered=True)
+    reach the tile, not the arithmetic: both paths agree bit for bit (E = 128:
+    ~19 pairs per expert; E = 40: ~60)"""
+    a32, a16, *_ = _moe_gemm_case(300, 8, 1, E, 256, 512, 4, 64, torch.bfloat16, 880)
+    b32, b16, *_ = _moe_gemm_case(300, 8, 1, E, 256, 512, 4, 64, torch.bfloat16, 880, gathered=True)
     assert torch.equal(a32.view(torch.int32), b32.view(torch.int32))
     assert torch.equal(a16.view(torch.int16), b16.view(torch.int16))
 
 
-def test_moe_gemm_fp16_and_many_blocks_per_expert():
+@pytest.mark.parametrize("gathered", [False, True])
+def test_moe_gemm_fp16_and_many_blocks_per_expert(gathered):
     """an expert with more than 256 pairs spans several blocks"""
-    out32, out16, ref, rc, st, ids = _moe_gemm_case(700, 2, 1, 3, 160, 512, 4, 64, torch.float16, 850)
+    out32, out16, ref, rc, st, ids = _moe_gemm_case(700, 2, 1, 3, 160, 512, 4, 64, torch.float16, 850,
+                                                    gathered=gathered)
     assert int(np.bincount(ids.numpy().reshape(-1)).max()) > 256
     gate(out32.cpu().numpy(), ref, "moe gemm f16 long groups")
     rne_equal(out16, out32)
