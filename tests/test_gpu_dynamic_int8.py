@@ -105,3 +105,23 @@ def test_matmul_decode_shape_all_outputs():
     y32 = g32.check("int8 decode")
     gate(y32.cpu().numpy(), yref, "dynamic int8 decode 4096x4096")
     rne_equal(g16.check("int8 decode bf16"), y32)
+
+
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M", [1, 5, 16])
+@pytest.mark.parametrize("N,K", [(200, 2048), (1000, 14336)])
+def test_matmul_streaming_kernel_shapes(x_dtype, M, N, K):
+    """few tokens, 16-bit x and K a multiple of 512: the streaming tensor-core
+    GEMV with the per-tensor scale (K = 14336: 224 groups, a partial last
+    unit; N = 200: a ragged last row tile); every output compared"""
+    w = weights(N, K, 70 + K + M)
+    q, params = api.qmm_quantize_dynamic_int8(w.to(DEV))
+    x = wl.gen_x(M, K, 71 + M, _NAME[x_dtype])
+    g32, gx = Guarded((M, N), torch.float32), Guarded((M, N), x_dtype)
+    api.qmm_matmul_dynamic_int8(x.to(DEV), q, params, out=g32.out)
+    api.qmm_matmul_dynamic_int8(x.to(DEV), q, params, out=gx.out)
+    torch.cuda.synchronize()
+    y32, yx = g32.check("int8 stream y32"), gx.check("int8 stream y")
+    yref = oracle.matmul_dynamic_int8(np_storage(x), ORC[x_dtype], q.cpu().numpy(), params.cpu().numpy())
+    gate(y32.cpu().numpy(), yref, f"dynamic int8 stream M{M} {N}x{K}")
+    rne_equal(yx, y32)

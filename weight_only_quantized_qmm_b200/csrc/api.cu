@@ -280,6 +280,14 @@ qmm_status qmm_matmul_dynamic_int8(const void* x, qmm_dtype x_dtype, int64_t M, 
   if (!aligned16(x) || !aligned16(q) || !aligned16(y) || !aligned4(params)) return QMM_ERR_ALIGNMENT;
   const qmm_status s = device_check();
   if (s != QMM_OK) return s;
+  // few tokens, 16-bit x, rows of whole 32-group units (K % 512 == 0,
+  // K >= 2048): the streaming tensor-core GEMV with the per-tensor scale
+  if ((x_dtype == QMM_BF16 || x_dtype == QMM_F16) && M <= 16 && K % 512 == 0 && K >= 2048 &&
+      K <= (int64_t)INT32_MAX && N >= 16) {
+    const qmm::QgemvParams p = qmm::make_pt_params(x, M, K, q, N, params, y, y_dtype);
+    const cudaError_t e = qmm::launch_qgemv_pt(p, x_dtype, (cudaStream_t)stream);
+    if (e != cudaErrorNotSupported) return launch_status(e);
+  }
   return launch_status(qmm::launch_matmul_dyn8(x, x_dtype, M, K, q, N, params, y, y_dtype, (cudaStream_t)stream));
 }
 

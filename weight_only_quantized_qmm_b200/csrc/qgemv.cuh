@@ -38,6 +38,9 @@ struct QgemvParams {
 // Launch planner (qgemv.cu); cudaErrorInvalidValue when a size limit of the
 // kernel is exceeded.
 cudaError_t launch_qgemv(QgemvParams prm, int bits, int gs, int dtype, bool dual, cudaStream_t st);
+// per-tensor dynamic-range int8 [N, K] on the streaming kernel (params from
+// make_pt_params); cudaErrorNotSupported when the shape does not fit it
+cudaError_t launch_qgemv_pt(const QgemvParams& prm, int dtype, cudaStream_t st);
 
 inline QgemvParams make_dense_params(const void* x, int64_t M, int64_t K, const qmm_qweight* w,
                                      void* y, int64_t ldy, int y_dtype) {
@@ -58,6 +61,32 @@ inline QgemvParams make_dense_params(const void* x, int64_t M, int64_t K, const 
   p.out = y;
   p.out_dtype = y_dtype;
   p.out_ld = ldy;
+  p.d_status = nullptr;
+  p.use_tma = 1;
+  return p;
+}
+
+// W is int8 [N, K] row-major (as 32-bit words of 4 codes); params: the
+// device float[4] {in_min, in_max, out_min, out_max}
+inline QgemvParams make_pt_params(const void* x, int64_t M, int64_t K, const int8_t* q, int64_t N,
+                                  const float* params, void* y, int y_dtype) {
+  QgemvParams p{};
+  p.packed[0] = reinterpret_cast<const uint32_t*>(q);
+  p.scales[0] = params;
+  p.biases[0] = params;
+  p.n_rows = N;
+  p.K = K;
+  p.wpr = K / 4;
+  p.G = (int)(K / 64);
+  p.num_experts = 1;
+  p.a = x;
+  p.amode = 0;
+  p.top_k = 1;
+  p.ids = nullptr;
+  p.n_pairs = (int)M;
+  p.out = y;
+  p.out_dtype = y_dtype;
+  p.out_ld = N;
   p.d_status = nullptr;
   p.use_tma = 1;
   return p;

@@ -31,6 +31,22 @@ static cudaError_t try_tma(const QgemvParams& prm, int gs, int dtype, int mt, bo
   return launch_tma_mt<128, __half>(prm, rows_total, mt, dual, st);
 }
 
+// per-tensor int8: 8-bit lanes (u = q + 128) in 64-code groups of 32-group
+// units, one scale and bias for the tensor
+template <typename T>
+static cudaError_t launch_pt_t(const QgemvParams& prm, cudaStream_t st) {
+  if (prm.n_pairs == 1) return stream::launch_stream<8, 64, T, 0, 32, 1, false, false, true>(prm, st);
+  if (prm.n_pairs <= 8) return stream::launch_stream<8, 64, T, 1, 32, 1, false, false, true>(prm, st);
+  if (prm.n_pairs <= 16) return stream::launch_stream<8, 64, T, 2, 32, 1, false, false, true>(prm, st);
+  return cudaErrorNotSupported;
+}
+
+cudaError_t launch_qgemv_pt(const QgemvParams& prm, int dtype, cudaStream_t st) {
+  if (dtype == QMM_BF16) return launch_pt_t<__nv_bfloat16>(prm, st);
+  if (dtype == QMM_F16) return launch_pt_t<__half>(prm, st);
+  return cudaErrorNotSupported;
+}
+
 cudaError_t launch_qgemv_b8(const QgemvParams& prm, int gs, int dtype, int mt, bool dual,
                             cudaStream_t st) {
   if (prm.use_tma) {

@@ -504,7 +504,12 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     if (idx % TOKP >= np) rec[idx] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1>
+// PT (8-bit codes only): per-tensor dynamic-range int8 ("mlex 0.1.3
+// src/quant.rs"): the codes are int8 q, u = q + 128 is the code the lanes
+// decode, and one scale fl((out_max - out_min) / 255) with bias out_min
+// serves every group (scales[0] points to the four float params; no
+// scale/bias copies).
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1, bool PT>
 __global__ void __launch_bounds__(Cfg<BITS, GS, T, MODE, UG, NS, MOE, SB1>::THREADS, 1)
 qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, const __grid_constant__ CUtensorMap tms0,
                     const __grid_constant__ CUtensorMap tmb0, const __grid_constant__ CUtensorMap tmc1,
@@ -565,12 +570,20 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
       const int t = tb0 + i / p.upt, ku = i % p.upt;
       const int y = (t % p.ntiles_e) * C::ROWS;
       tma_prefetch_3d(&tmc0, 0, y, ku * C::Z);
-      tma_prefetch_2d(&tms0, ku * GPU, y);
-      tma_prefetch_2d(&tmb0, ku * GPU, y);
+      if constexpr (!PT) {
+        tma_prefetch_2d(&tms0, ku * GPU, y);
+        tma_prefetch_2d(&tmb0, ku * GPU, y);
+      }
     }
   }
   // weights, ids and x may all come from the previous kernel in the stream
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  float pt_s = 0.0f, pt_b = 0.0f;  // PT: the per-tensor scale fl((out_max - out_min) / 255) and out_min
+  if constexpr (PT) {
+    const float* pp = reinterpret_cast<const float*>(q.scales[0]);
+    pt_s = __fdiv_rn(__fsub_rn(__ldg(pp + 3), __ldg(pp + 2)), 255.0f);
+    pt_b = __ldg(pp + 2);
+  }
   if (q.ids) {
     bool direct = false;
     if constexpr (C::ONE) {
@@ -658,7 +671,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
         const uint32_t cd = code_ring + (uint32_t)(slot * NS * C::CODE_BYTES);
         const uint32_t sd = sb_ring + (uint32_t)(slot * NS * 2 * C::SB_BYTES);
         tma_load_3d(cd, &tmc0, 0, y, ku * C::Z, fb);
-        if constexpr (SB1) {  // rows y .. y + ROWS - 1 of the [rows, G] arrays, contiguous
+        if constexpr (PT) {
+        } else if constexpr (SB1) {  // rows y .. y + ROWS - 1 of the [rows, G] arrays, contiguous
           const uint32_t nb = (uint32_t)(2 * C::ROWS * q.G);
           bulk_load_1d(sd, reinterpret_cast<const uint8_t*>(q.scales[0]) + (int64_t)y * q.G * 2, nb, fb);
           bulk_load_1d(sd + C::SB_BYTES, reinterpret_cast<const uint8_t*>(q.biases[0]) + (int64_t)y * q.G * 2, nb, fb);
@@ -858,7 +872,8 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const uint32_t ra = ssl + (uint32_t)(h * 8 * PITCH);
-          if constexpr (SB1) {  // 2-byte aligned only: one value at a time
+          if constexpr (PT) {  // (the per-tensor scale and bias: no copies)
+          } else if constexpr (SB1) {  // 2-byte aligned only: one value at a time
 #pragma unroll
             for (int c = 0; c < (GPW + 1) / 2; ++c) {
               sv[h][c] = lds16(ra + 4 * c) | (2 * c + 1 < GPW ? lds16(ra + 4 * c + 2) << 16 : 0u);
@@ -900,6 +915,13 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
             for (int k2 = 0; k2 < L::kRegs / 2; ++k2)
               ldsm_x4(csl + code_addr(u, k2), rA[2 * k2], rB[2 * k2], rA[2 * k2 + 1], rB[2 * k2 + 1]);
           }
+          if constexpr (PT) {  // int8 q -> u = q + 128: the top bit of each byte flipped
+#pragma unroll
+            for (int k = 0; k < L::kRegs; ++k) {
+              rA[k] ^= 0x80808080u;
+              rB[k] ^= 0x80808080u;
+            }
+          }
           float d[MT][4];
           if constexpr (C::ONE) {
             // this group's x fragments (staged in the mma's k order); measured:
@@ -911,8 +933,10 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
           } else
             group_dot1<L, MT>(rA, rB, t, xbu, (uint32_t)(u * C::XG), d);
           const int hw = u & 1;
-          const float sa = half_to_f32<T>(sv[0][u >> 1], hw), sb_ = half_to_f32<T>(sv[1][u >> 1], hw);
-          const float ba = half_to_f32<T>(bv[0][u >> 1], hw), bb = half_to_f32<T>(bv[1][u >> 1], hw);
+          const float sa = PT ? pt_s : half_to_f32<T>(sv[0][u >> 1], hw);
+          const float sb_ = PT ? pt_s : half_to_f32<T>(sv[1][u >> 1], hw);
+          const float ba = PT ? pt_b : half_to_f32<T>(bv[0][u >> 1], hw);
+          const float bb = PT ? pt_b : half_to_f32<T>(bv[1][u >> 1], hw);
           // y += s * (2^-e * D - 1024 * 2^-e * sum x'') + b * sum x, per (row, pair)
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
@@ -1035,8 +1059,9 @@ inline bool make_sb_map(CUtensorMap* map, const void* base, int64_t rows, int G,
 }
 
 // cudaErrorNotSupported sends the caller to the general kernels.
-template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false>
+template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false, bool PT = false>
 cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
+  static_assert(!PT || (BITS == 8 && NS == 1 && !MOE && !SB1), "per-tensor int8: dense 8-bit lanes");
   using C = Cfg<BITS, GS, T, MODE, UG, NS, MOE, SB1>;
   if (MOE != (q.ids != nullptr)) return cudaErrorNotSupported;
   const int64_t rows_total = q.n_rows * q.num_experts;
@@ -1050,14 +1075,15 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   }
   if (rows_total + 16 >= ((int64_t)1 << 31) || (int64_t)q.n_pairs * q.K >= ((int64_t)1 << 31)) return cudaErrorNotSupported;
   for (int ns = 0; ns < NS; ++ns)
-    if (((uintptr_t)q.packed[ns] | (uintptr_t)q.scales[ns] | (uintptr_t)q.biases[ns]) & 15) return cudaErrorNotSupported;
+    if (((uintptr_t)q.packed[ns] | (PT ? 0 : ((uintptr_t)q.scales[ns] | (uintptr_t)q.biases[ns]))) & 15)
+      return cudaErrorNotSupported;
 
   Params p{};
   p.q = q;
   p.upt = (q.G + C::GPU - 1) / C::GPU;
   p.ntiles_e = (int)((q.n_rows + C::ROWS - 1) / C::ROWS);
   p.CH = C::CH;
-  p.tx = (uint32_t)(NS * C::CODE_BYTES + NS * (SB1 ? 4 * C::ROWS * q.G : 2 * C::SB_BYTES));
+  p.tx = (uint32_t)(NS * C::CODE_BYTES + (PT ? 0 : NS * (SB1 ? 4 * C::ROWS * q.G : 2 * C::SB_BYTES)));
   const int Gpad = p.upt * C::GPU;
   p.tok_stride = Gpad * C::XG + 16;
 
@@ -1091,7 +1117,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   CUtensorMap tm[6];
   for (int ns = 0; ns < NS; ++ns) {
     if (!make_code_map3(&tm[3 * ns], q.packed[ns], rows_total, q.wpr, C::Z, C::ROWS)) return cudaErrorNotSupported;
-    if (SB1) {  // no scale/bias maps: 1-D bulk copies
+    if (SB1 || PT) {  // no scale/bias maps: 1-D bulk copies, or none
       tm[3 * ns + 1] = tm[3 * ns];
       tm[3 * ns + 2] = tm[3 * ns];
     } else if (!make_sb_map(&tm[3 * ns + 1], q.scales[ns], rows_total, q.G, C::GPU) ||
@@ -1101,7 +1127,7 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
   }
   if (NS == 1) { tm[3] = tm[0]; tm[4] = tm[1]; tm[5] = tm[2]; }
 
-  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS, MOE, SB1>;
+  auto k = qgemv_stream_kernel<BITS, GS, T, MODE, UG, NS, MOE, SB1, PT>;
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
