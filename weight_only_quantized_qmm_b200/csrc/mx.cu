@@ -130,23 +130,31 @@ __device__ __forceinline__ void lanes_f32(uint32_t w, float* v) {
 // y[m, n] = sum_k x[m, k] w_hat[n, k]: one warp per row n (grid-stride); lane
 // l takes the 32-code chunks l, l + 32, ..., kBatch of them per request; per
 // group the partial dot sum_k x_k lane_k is taken first and then scaled.
-// XS: x staged in shared memory as fp32.
-template <int MODE, typename TX, bool XS>
+// XS: x staged in shared memory as fp32, each 32-value chunk padded to 36
+// floats so that the lanes' 16-byte reads of their chunks (144 bytes apart)
+// fall in distinct banks.  MB: tokens per pass (1 for a single
+// token, so that no predicated-off token work is issued; else kMB).
+template <int MODE, typename TX, bool XS, int MB>
 __global__ void __launch_bounds__(256)
 matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ packed,
                  const uint8_t* __restrict__ scales, int64_t N, void* y, int64_t ldy, int y_dtype) {
+  constexpr int kMB = MB;
   using Md = Mode<MODE>;
   constexpr int B = Md::B, GS = Md::GS, GPC = 32 / GS;  // groups per 32-code chunk
   constexpr float kLaneUnit = B == 4 ? 16384.0f : 256.0f;
-  extern __shared__ float xs[];  // [kMB][K] when XS
+  extern __shared__ float xs[];  // [kMB][K / 32][36] when XS
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
   const int64_t chunks = K / 32, wpr = K * B / 32, G = K / GS;
+  const int64_t KP = chunks * 36;  // padded staged row
   for (int64_t m0 = 0; m0 < M; m0 += kMB) {
     const int mb = (int)(M - m0 < kMB ? M - m0 : kMB);
     if (XS) {
       __syncthreads();
-      for (int64_t i = threadIdx.x; i < (int64_t)mb * K; i += blockDim.x) xs[i] = to_f32(x[m0 * K + i]);
+      for (int64_t i = threadIdx.x; i < (int64_t)mb * K; i += blockDim.x) {
+        const int64_t t = i / K, k = i - t * K;
+        xs[t * KP + (k >> 5) * 36 + (k & 31)] = to_f32(x[m0 * K + i]);
+      }
       __syncthreads();
     }
     for (int64_t n = blockIdx.x * (int64_t)(blockDim.x / 32) + (threadIdx.x >> 5); n < N; n += warps) {
@@ -189,7 +197,7 @@ matmul_mx_kernel(const TX* __restrict__ x, int64_t M, int64_t K, const uint32_t*
                   for (int i = gi * GS; i < (gi + 1) * GS; i += 4) {
                     float4 xv;
                     if (XS) {
-                      xv = *reinterpret_cast<const float4*>(xs + t * K + c * 32 + i);
+                      xv = *reinterpret_cast<const float4*>(xs + t * KP + c * 36 + i);
                     } else {
                       const TX* xp = x + (m0 + t) * K + c * 32 + i;
                       xv = make_float4(to_f32(xp[0]), to_f32(xp[1]), to_f32(xp[2]), to_f32(xp[3]));
@@ -237,17 +245,17 @@ static cudaError_t matmul_x(const TX* x, int64_t M, int64_t K, const qmm_qweight
                             int y_dtype, cudaStream_t st) {
   auto S = reinterpret_cast<const uint8_t*>(w->scales);
   const int64_t N = w->rows;
-  const bool xs = (M < kMB ? M : kMB) * K * 4 <= kXsMax;
-  const size_t smem = xs ? (size_t)(M < kMB ? M : kMB) * K * 4 : 0;
+  const int64_t row_bytes = (K / 32) * 36 * 4;  // a staged (padded) row of x
+  const bool xs = (M < kMB ? M : kMB) * row_bytes <= kXsMax;
+  const size_t smem = xs ? (size_t)(M < kMB ? M : kMB) * row_bytes : 0;
   const int blocks = (int)std::min<int64_t>((N + 7) / 8, (int64_t)qmm_host::num_sms() * (smem > 64 * 1024 ? 1 : 2));
+  auto k = xs ? (M == 1 ? matmul_mx_kernel<MODE, TX, true, 1> : matmul_mx_kernel<MODE, TX, true, kMB>)
+              : (M == 1 ? matmul_mx_kernel<MODE, TX, false, 1> : matmul_mx_kernel<MODE, TX, false, kMB>);
   if (xs) {
-    auto k = matmul_mx_kernel<MODE, TX, true>;
     const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kXsMax);
     if (e != cudaSuccess) return e;
-    k<<<blocks, 256, smem, st>>>(x, M, K, w->packed, S, N, y, ldy, y_dtype);
-  } else {
-    matmul_mx_kernel<MODE, TX, false><<<blocks, 256, 0, st>>>(x, M, K, w->packed, S, N, y, ldy, y_dtype);
   }
+  k<<<blocks, 256, smem, st>>>(x, M, K, w->packed, S, N, y, ldy, y_dtype);
   return cudaGetLastError();
 }
 
