@@ -147,9 +147,9 @@ __device__ __forceinline__ void ldsm_x4(uint32_t a, uint32_t& r0, uint32_t& r1, 
 // (32, or 64 when the row length allows; 16 for 32-word groups).  NS: weight
 // matrices per pair (2: gate and up).  SB1: rows of G <= UG groups whose
 // scale/bias rows are not 16-byte strided (G % 8 != 0, e.g. K = 768 at group
-// 64): a unit is TR = 4 whole row tiles (64 rows), its 64 scale (bias) rows
-// arrive as one contiguous 1-D bulk copy of 128 G bytes, unswizzled; KC / TR
-// consumers share a row tile, and groups >= G are skipped.
+// 64): a unit is TR = 8 whole row tiles (128 rows, one per consumer warp),
+// its 128 scale (bias) rows arrive as one contiguous 1-D bulk copy of 256 G
+// bytes, unswizzled; groups >= G are skipped.
 template <int BITS, int GS, typename T, int MODE, int UG, int NS, bool MOE, bool SB1 = false>
 struct Cfg {
   using L = Lanes<BITS, GS>;
@@ -163,7 +163,7 @@ struct Cfg {
   static constexpr int PRODUCER = KC, EPILOGUE = KC + 1;          // warp indices
   static constexpr int WPG = L::kWordsPerGroup;                   // words per group per row
   static constexpr int GPU = UG;                                  // groups per unit
-  static constexpr int TR = SB1 ? 4 : 1;                          // 16-row tiles per unit
+  static constexpr int TR = SB1 ? 8 : 1;                          // 16-row tiles per unit (measured: 8 beats 2 and 4)
   static constexpr int ROWS = 16 * TR;                            // weight rows per unit
   static constexpr int WPT = KC / TR;                             // consumers per row tile
   static constexpr int GPW = GPU / WPT;                           // groups per consumer per unit
