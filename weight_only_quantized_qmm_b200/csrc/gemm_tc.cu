@@ -172,6 +172,9 @@ struct GemmParams {
   // the x map is the row of the pair listed at entry i), so a tile's rows
   // are one contiguous box; 0: the producer gathers them 4 at a time
   int xg;
+  // dense: tokens per tile, 256, or 128 when 256-token tiles would leave SMs
+  // idle (few tokens, few weight rows)
+  int tbn;
 };
 
 // ------------------------------------------------------------------ dequant helpers
@@ -238,7 +241,7 @@ __device__ __forceinline__ TileOf tile_of(const GemmParams& p, int lt, int m_til
     return TileOf{nt * gemm::kBM, m0, min(gemm::kBN, __ldg(p.ws_off + e + 1) - m0), e};
   } else {
     const int nt = t / m_tiles, mt = t - nt * m_tiles;
-    return TileOf{nt * gemm::kBM, mt * gemm::kBN, min(gemm::kBN, p.M - mt * gemm::kBN), 0};
+    return TileOf{nt * gemm::kBM, mt * p.tbn, min(p.tbn, p.M - mt * p.tbn), 0};
   }
 }
 // row of the activation matrix that token slot j of a MoE tile reads
@@ -295,7 +298,7 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = (p.K + kBK - 1) / kBK;
-  const int m_tiles = (p.M + kBN - 1) / kBN;
+  const int m_tiles = (p.M + p.tbn - 1) / p.tbn;
   const int n_tiles = (p.N + kBM - 1) / kBM;
 
   if (threadIdx.x == 0) {
@@ -394,9 +397,10 @@ qgemm_tc_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmx, con
             tma_gather4(d + 512, &tmx, i * kBK, rw[4], rw[5], rw[6], rw[7], full0 + 8 * s);
           }
         } else if (lane == 0) {
-          // one 256-row box (measured: eight 32-row boxes per stage cost a
+          // one box of the tile's token rows (256, or 128 for a dense call of
+          // 128-token tiles; measured: eight 32-row boxes per stage cost a
           // third of the dense GEMM's throughput)
-          mbar_arrive_expect_tx(full0 + 8 * s, kXStage);
+          mbar_arrive_expect_tx(full0 + 8 * s, MOE ? (uint32_t)kXStage : (uint32_t)(p.tbn * kBK * 2));
           tma_2d(su32(xs + s * kXStage), &tmx, i * kBK, tl.m0, full0 + 8 * s);
         }
         issued = j + 1;
@@ -769,8 +773,11 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   if (M > (int64_t)INT32_MAX || K > (int64_t)INT32_MAX || w->rows > (int64_t)INT32_MAX)
     return cudaErrorNotSupported;
   if ((K * 2) % 16 != 0) return cudaErrorNotSupported;
+  // 128-token tiles when 256-token tiles would not give every SM one
+  const int64_t n_tiles = (w->rows + gemm::kBM - 1) / gemm::kBM;
+  const int tbn = (n_tiles * ((M + gemm::kBN - 1) / gemm::kBN) < qmm_host::num_sms() && M > 128) ? 128 : gemm::kBN;
   CUtensorMap tm[4];
-  if (!make_x_map(&tm[0], x, x_dtype, M, K, gemm::kBN)) return cudaErrorNotSupported;
+  if (!make_x_map(&tm[0], x, x_dtype, M, K, tbn)) return cudaErrorNotSupported;
   const bool tw = make_w_maps(&tm[1], &tm[2], &tm[3], w->packed, w->scales, w->biases, w->rows,
                               K * w->bits / 32, K / w->group_size, w->bits);
   if (!tw) tm[1] = tm[2] = tm[3] = tm[0];
@@ -786,8 +793,9 @@ cudaError_t launch_qgemm_tc(const void* x, int x_dtype, int64_t M, int64_t K, co
   prm.K = (int)K;
   prm.G = (int)(K / w->group_size);
   prm.wpr = (int)(K * w->bits / 32);
+  prm.tbn = tbn;
   // persistent: one CTA per SM (or per tile when there are fewer tiles)
-  const int64_t tiles = ((prm.N + gemm::kBM - 1) / gemm::kBM) * (int64_t)((prm.M + gemm::kBN - 1) / gemm::kBN);
+  const int64_t tiles = n_tiles * (int64_t)((prm.M + tbn - 1) / tbn);
   const int grid = (int)std::min<int64_t>(tiles, qmm_host::num_sms());
   if (x_dtype == QMM_BF16) return launch_gemm_b<__nv_bfloat16, false>(w->bits, w->group_size, tw, prm, tm, grid, st);
   return launch_gemm_b<__half, false>(w->bits, w->group_size, tw, prm, tm, grid, st);
@@ -828,6 +836,7 @@ cudaError_t launch_qgemm_moe(const void* a, int a_dtype, int64_t a_rows, const q
   prm.ws_pairs = ws_pairs;
   prm.ws_blk_e = ws_blk_e;
   prm.ws_blk_s = ws_blk_s;
+  prm.tbn = gemm::kBN;  // (blocks of up to 256 pairs)
   prm.E = (int)w->num_experts;
   prm.top_k = top_k;
   prm.ne11 = ne11;
