@@ -59,14 +59,28 @@ __device__ __forceinline__ float ld_peer(const float* p, uint32_t rank) {
   return v;
 }
 
-// the thread's kCS codes of one row (its packed words) as floats: each
-// code's bits under the exponent of 2^23, minus 2^23
+// the thread's kCS codes of one row (its packed words) as the floats
+// 1024 + code: two codes per 32-bit word at a time under the exponent of an
+// f16 pair (one lop3 each, both halves exact), widened to fp32.  The 1024s
+// are taken back once per token at the end (1024 times the sum of the x s
+// the codes were multiplied by).
 template <int B>
-__device__ __forceinline__ void codes_f32(const uint32_t* w, float* q) {
-  constexpr int CPW = 32 / B;
+__device__ __forceinline__ void codes_1024(const uint32_t* w, float* q) {
+  constexpr int CPW = 32 / B;   // codes per word
+  constexpr int HALF = CPW / 2; // code j pairs with code j + HALF (the upper 16 bits)
+  constexpr uint32_t M = ((1u << B) - 1u) * 0x00010001u;
 #pragma unroll
-  for (int c = 0; c < kCS; ++c)
-    q[c] = __int_as_float((int)(((w[c / CPW] >> (B * (c % CPW))) & ((1u << B) - 1u)) | 0x4B000000u)) - 8388608.0f;
+  for (int k = 0; k < kCS / CPW; ++k) {
+#pragma unroll
+    for (int j = 0; j < HALF; ++j) {
+      const uint32_t h = ((w[k] >> (B * j)) & M) | 0x64006400u;
+      __half2 hh;
+      memcpy(&hh, &h, 4);
+      const float2 f = __half22float2(hh);
+      q[k * CPW + j] = f.x;
+      q[k * CPW + j + HALF] = f.y;
+    }
+  }
 }
 
 template <int B, typename T, int kTok>
@@ -90,10 +104,11 @@ qgemv_t0_kernel(const T* __restrict__ x, int M, int K, const uint32_t* __restric
   const uint32_t* wbase = packed + (live ? ncol * B / 32 : 0);
   for (int m0 = 0; m0 < M; m0 += kTok) {
     const int mb = min(kTok, M - m0);
-    float acc[kTok][kCS], bacc[kTok];
+    float acc[kTok][kCS], bacc[kTok], sxs[kTok];
 #pragma unroll
     for (int t = 0; t < kTok; ++t) {
       bacc[t] = 0.0f;
+      sxs[t] = 0.0f;
 #pragma unroll
       for (int c = 0; c < kCS; ++c) acc[t][c] = 0.0f;
     }
@@ -131,12 +146,13 @@ qgemv_t0_kernel(const T* __restrict__ x, int M, int K, const uint32_t* __restric
             const int kk = kk0 + j * kRPI;
             if (kk < kn) {
               float q[kCS];
-              codes_f32<B>(wv[j], q);
+              codes_1024<B>(wv[j], q);
 #pragma unroll
               for (int t = 0; t < kTok; ++t) {
                 const float xk = xs[t][kk];
                 const float xsk = xk * sv[j];
                 bacc[t] = fmaf(xk, bv[j], bacc[t]);
+                sxs[t] += xsk;
 #pragma unroll
                 for (int c = 0; c < kCS; ++c) acc[t][c] = fmaf(xsk, q[c], acc[t][c]);
               }
@@ -149,7 +165,7 @@ qgemv_t0_kernel(const T* __restrict__ x, int M, int K, const uint32_t* __restric
 #pragma unroll
     for (int t = 0; t < kTok; ++t)
 #pragma unroll
-      for (int c = 0; c < kCS; ++c) red[t][lw * kCS + c][rs] = acc[t][c] + bacc[t];
+      for (int c = 0; c < kCS; ++c) red[t][lw * kCS + c][rs] = fmaf(-1024.0f, sxs[t], acc[t][c]) + bacc[t];
     __syncthreads();
     for (int i = tid; i < kTok * kCB; i += kThreads) {
       const int t = i / kCB, c = i - t * kCB;
