@@ -97,13 +97,16 @@ struct Lanes {
   static constexpr int kOPW = kWhole ? kLPW / 2 : 1;   // f16 pairs per word
   static constexpr int kCodes = GS / 4;                // codes of a thread's quarter
   static constexpr int kQBits = kCodes * BITS;         // bits of a quarter
+  // a 16-bit quarter (2-bit codes, group 32): half of word t / 2, spread over
+  // both halves of a register before the masks (see quarter_pairs)
+  static constexpr bool kHalf = kWhole && kQBits == 16;
   // packed words a thread reads per row: the quarter's own words, or (a
   // 48-bit quarter) the two words that hold it
   static constexpr int kRegs = (kQBits + 31) / 32;
   static constexpr int kOuts = kCodes / 2;             // f16 pairs of a quarter
   static constexpr int kSteps = kCodes / 4;            // m16n8k16 steps per group
   static constexpr int kWordsPerGroup = GS * BITS / 32;
-  static constexpr bool kOk = kWhole ? kQBits % 32 == 0 : ((BITS == 3 || BITS == 6) && (GS == 64 || GS == 128));
+  static constexpr bool kOk = kWhole ? (kQBits % 32 == 0 || kHalf) : ((BITS == 3 || BITS == 6) && (GS == 64 || GS == 128));
   static constexpr uint32_t kMagic = 0x64006400u;      // f16 1024.0 in both halves
   static constexpr float kOff = 1024.0f;
   __host__ __device__ static constexpr int pos(int j) {
@@ -112,12 +115,12 @@ struct Lanes {
   // pair o of the quarter -> code index (within the quarter) and bit offset
   // of its low and high half
   __host__ __device__ static constexpr int lo_code(int o) {
-    return kWhole ? (o / kOPW) * kLPW + o % kOPW
+    return kHalf ? o : kWhole ? (o / kOPW) * kLPW + o % kOPW
                   : 16 * (o / 8) + (BITS == 3 ? "\x00\x01\x02\x08\x09\x0a\x06\x07"[o % 8]
                                                 : "\x00\x01\x04\x05\x08\x09\x0c\x0d"[o % 8]);
   }
   __host__ __device__ static constexpr int hi_code(int o) {
-    return kWhole ? lo_code(o) + kOPW
+    return kHalf ? o + 4 : kWhole ? lo_code(o) + kOPW
                   : 16 * (o / 8) + (BITS == 3 ? "\x03\x04\x05\x0b\x0c\x0d\x0e\x0f"[o % 8]
                                                 : "\x02\x03\x06\x07\x0a\x0b\x0e\x0f"[o % 8]);
   }
@@ -129,7 +132,7 @@ struct Lanes {
   }
   // code of the group held as code i of quarter t
   __host__ __device__ static constexpr int gcode(int t, int i) {
-    return kWhole ? (t + 4 * (i / kLPW)) * kLPW + i % kLPW : kCodes * t + i;
+    return (kWhole && !kHalf) ? (t + 4 * (i / kLPW)) * kLPW + i % kLPW : kCodes * t + i;
   }
   // first packed word (within the group's row) that thread t reads
   __host__ __device__ static constexpr int first_word(int t) { return (t * kQBits) >> 5; }
@@ -277,7 +280,15 @@ __device__ __forceinline__ uint32_t prmt_rt(uint32_t a, uint32_t b, uint32_t sel
 // The kOuts f16 pairs of thread t's quarter (see Lanes).
 template <class L>
 __device__ __forceinline__ void quarter_pairs(const uint32_t (&r)[L::kRegs], int t, uint32_t* o) {
-  if constexpr (L::kWhole) {
+  if constexpr (L::kHalf) {
+    // the quarter's two bytes, (b0, b1), into the low bytes of the two halves:
+    // pair j = codes j and j + 4, at bit 2j of each half
+    const uint32_t v = prmt_rt((t & 1) ? (r[0] >> 16) : r[0], 0u, 0x4140u);
+    uint32_t tmp[8];
+    word_pairs16<2>(v, tmp);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o[j] = tmp[j];
+  } else if constexpr (L::kWhole) {
 #pragma unroll
     for (int k = 0; k < L::kRegs; ++k) word_pairs16<32 / L::kLPW>(r[k], o + k * L::kOPW);
   } else if constexpr (L::kQBits / L::kCodes == 3) {
@@ -428,7 +439,7 @@ __device__ __forceinline__ void stage_x(const QgemvParams& q, const int* pairs, 
     __align__(16) T xv[L::kCodes];
     if (act && gl < q.G) {
       const T* xg = reinterpret_cast<const T*>(q.a) + pair_offset(q, pairs[m]) + (int64_t)gl * GS;
-      if constexpr (L::kWhole) {
+      if constexpr (L::kWhole && !L::kHalf) {
         constexpr int WB = L::kLPW * (int)sizeof(T);  // bytes of x under one packed word
 #pragma unroll
         for (int k = 0; k < L::kRegs; ++k) {
@@ -777,7 +788,7 @@ qgemv_stream_kernel(const Params p, const __grid_constant__ CUtensorMap tmc0, co
   auto code_addr = [&](int u, int k2) -> uint32_t {
     const int w0 = (gw * GPW + u) * WPG;  // first word of the group in the unit row
     if constexpr (L::kRegs == 1 || !L::kWhole) {
-      const int wr = w0 + (L::kWhole ? t : L::first_word(t) + k2);  // word in the unit row
+      const int wr = w0 + ((L::kWhole && !L::kHalf) ? t : L::first_word(t) + k2);  // word in the unit row
       const int wb = wr & 31;
       return (uint32_t)((wr >> 5) * C::SLICE + (rtl * 16 + g) * 128 + (((wb >> 2) ^ g) << 4) + ((wb & 3) << 2));
     } else {
