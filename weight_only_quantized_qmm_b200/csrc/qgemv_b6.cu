@@ -5,8 +5,8 @@ namespace qmm {
 
 cudaError_t launch_qgemv_b6(const QgemvParams& prm, int gs, int dtype, int mt, bool dual,
                             cudaStream_t st) {
-  // the streaming kernel for group sizes 64 and 128, else the cp.async kernel
-  if (prm.use_tma && gs != 32) {
+  // the streaming kernel, else (shapes it does not take) the cp.async kernel
+  if (prm.use_tma) {
     const cudaError_t es = stream::try_stream<6>(prm, gs, dtype, mt, dual, st);
     if (es != cudaErrorNotSupported) return es;
   }

@@ -102,11 +102,11 @@ struct Lanes {
   static constexpr bool kHalf = kWhole && kQBits == 16;
   // packed words a thread reads per row: the quarter's own words, or (a
   // 48-bit quarter) the two words that hold it
-  static constexpr int kRegs = (kQBits + 31) / 32;
+  static constexpr int kRegs = kQBits == 24 ? 2 : (kQBits + 31) / 32;  // (3-bit group 32: 3 bytes, may straddle)
   static constexpr int kOuts = kCodes / 2;             // f16 pairs of a quarter
   static constexpr int kSteps = kCodes / 4;            // m16n8k16 steps per group
   static constexpr int kWordsPerGroup = GS * BITS / 32;
-  static constexpr bool kOk = kWhole ? (kQBits % 32 == 0 || kHalf) : ((BITS == 3 || BITS == 6) && (GS == 64 || GS == 128));
+  static constexpr bool kOk = kWhole ? (kQBits % 32 == 0 || kHalf) : (BITS == 3 || BITS == 6);
   static constexpr uint32_t kMagic = 0x64006400u;      // f16 1024.0 in both halves
   static constexpr float kOff = 1024.0f;
   __host__ __device__ static constexpr int pos(int j) {
@@ -114,21 +114,28 @@ struct Lanes {
   }
   // pair o of the quarter -> code index (within the quarter) and bit offset
   // of its low and high half
+  // (a 3-bit quarter of 8 codes, group 32: pair 3 is codes 6 and 7 of byte
+  // 2, at bits 2 and 5 of the two halves)
+  static constexpr bool k3g32 = BITS == 3 && kCodes == 8;
   __host__ __device__ static constexpr int lo_code(int o) {
     return kHalf ? o : kWhole ? (o / kOPW) * kLPW + o % kOPW
+                  : k3g32 ? "\x00\x01\x02\x06"[o]
                   : 16 * (o / 8) + (BITS == 3 ? "\x00\x01\x02\x08\x09\x0a\x06\x07"[o % 8]
-                                                : "\x00\x01\x04\x05\x08\x09\x0c\x0d"[o % 8]);
+                                              : "\x00\x01\x04\x05\x08\x09\x0c\x0d"[o % 8]);
   }
   __host__ __device__ static constexpr int hi_code(int o) {
     return kHalf ? o + 4 : kWhole ? lo_code(o) + kOPW
+                  : k3g32 ? "\x03\x04\x05\x07"[o]
                   : 16 * (o / 8) + (BITS == 3 ? "\x03\x04\x05\x0b\x0c\x0d\x0e\x0f"[o % 8]
-                                                : "\x02\x03\x06\x07\x0a\x0b\x0e\x0f"[o % 8]);
+                                              : "\x02\x03\x06\x07\x0a\x0b\x0e\x0f"[o % 8]);
   }
   __host__ __device__ static constexpr int lo_pos(int o) {
-    return kWhole ? pos(o % kOPW) : (BITS == 3 ? "\x00\x03\x06\x00\x03\x06\x02\x05"[o % 8] : 4);
+    return kWhole ? pos(o % kOPW)
+                  : k3g32 ? "\x00\x03\x06\x02"[o] : (BITS == 3 ? "\x00\x03\x06\x00\x03\x06\x02\x05"[o % 8] : 4);
   }
   __host__ __device__ static constexpr int hi_pos(int o) {
-    return kWhole ? pos(o % kOPW) : (BITS == 3 ? "\x01\x04\x07\x01\x04\x07\x02\x05"[o % 8] : 0);
+    return kWhole ? pos(o % kOPW)
+                  : k3g32 ? "\x01\x04\x07\x05"[o] : (BITS == 3 ? "\x01\x04\x07\x01\x04\x07\x02\x05"[o % 8] : 0);
   }
   // code of the group held as code i of quarter t
   __host__ __device__ static constexpr int gcode(int t, int i) {
@@ -291,6 +298,15 @@ __device__ __forceinline__ void quarter_pairs(const uint32_t (&r)[L::kRegs], int
   } else if constexpr (L::kWhole) {
 #pragma unroll
     for (int k = 0; k < L::kRegs; ++k) word_pairs16<32 / L::kLPW>(r[k], o + k * L::kOPW);
+  } else if constexpr (L::k3g32) {
+    // 8 codes = bytes B0..B2 of the word pair (lo, hi) from byte 3t mod 4
+    const uint32_t add = (uint32_t)((3 * t) & 3) * 0x1111u;
+    const uint32_t r0 = prmt_rt(r[0], r[1], 0x2110u + add);  // (B0, B1 | B1, B2)
+    const uint32_t r2 = prmt_rt(r[0], r[1], 0x2222u + add);  // (B2, B2 | B2, B2)
+    o[0] = mask_magic<0x000E0007u>(r0);
+    o[1] = mask_magic<0x00700038u>(r0);
+    o[2] = mask_magic<0x038001C0u>(r0);
+    o[3] = mask_magic<0x00E0001Cu>(r2);
   } else if constexpr (L::kQBits / L::kCodes == 3) {
 #pragma unroll
     for (int c = 0; c < L::kCodes / 16; ++c) {
@@ -309,6 +325,15 @@ __device__ __forceinline__ void quarter_pairs(const uint32_t (&r)[L::kRegs], int
       o[8 * c + 6] = mask_magic<0x001C001Cu>(r2);
       o[8 * c + 7] = mask_magic<0x00E000E0u>(r2);
     }
+  } else if constexpr (L::kCodes == 8) {
+    // 6-bit, group 32: 8 codes = 48 bits of the word pair (lo, hi) from bit
+    // 16 (t odd) or 0; the windows start at quarter bits -4, 2, 20, 26
+    const uint32_t lo = r[0], hi = r[1];
+    const bool b = (t & 1) != 0;
+    o[0] = mask_magic<0x003F03F0u>(__funnelshift_r(b ? lo : 0u, b ? hi : lo, b ? 12 : 28));
+    o[1] = mask_magic<0x003F03F0u>(__funnelshift_r(lo, hi, b ? 18 : 2));
+    o[2] = mask_magic<0x003F03F0u>(__funnelshift_r(b ? hi : lo, b ? 0u : hi, b ? 4 : 20));
+    o[3] = mask_magic<0x003F03F0u>(__funnelshift_r(b ? hi : lo, b ? 0u : hi, b ? 10 : 26));
   } else {
 #pragma unroll
     for (int c = 0; c < L::kCodes / 16; ++c) {
@@ -1178,9 +1203,11 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
     }
     if (q.ids) {
       if (q.G % 8 != 0 || q.G < UB) {  // short or odd rows (e.g. the MoE down projection)
-        if (q.G <= 16) {
-          if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, 16, 1, true, true>(q, st);
-          return launch_stream<BITS, GS, T, 1, 16, 1, true, true>(q, st);
+        if constexpr (WPG % 2 == 0) {  // 16-group units of whole 128-byte slices
+          if (q.G <= 16) {
+            if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, 16, 1, true, true>(q, st);
+            return launch_stream<BITS, GS, T, 1, 16, 1, true, true>(q, st);
+          }
         }
         if constexpr (WPG <= 16) {  // a 32-group unit of at most 16 slices
           if (q.n_pairs <= 8) return launch_stream<BITS, GS, T, 0, 32, 1, true, true>(q, st);
