@@ -1122,7 +1122,9 @@ cudaError_t launch_stream(const QgemvParams& q, cudaStream_t st) {
 
   // [codes (1024-aligned) | scales+biases | mbarriers | partials | x | sums | plan]
   const size_t part = C::ONE ? (size_t)C::RB * C::KC * NS * 16 * 4 : (size_t)C::RB * C::KC * NS * C::MT * 32 * 16;
-  const size_t xs = align128((size_t)C::CH * p.tok_stride);
+  // staged x rows: a segment's pairs (a dense call stages only its own
+  // tokens, leaving the rest of shared memory to the weight ring)
+  const size_t xs = align128((size_t)(MOE ? C::CH : std::min(C::CH, q.n_pairs)) * p.tok_stride);
   const size_t xsum = align128((size_t)Gpad * C::TOKP * 16);  // float4 records
   const size_t bars = 8 * (2 * kMaxStages + 2 * C::RB);
   const size_t plan = align128((size_t)(5 * q.num_experts + 1 + 2 * q.n_pairs) * sizeof(int));
