@@ -1229,7 +1229,19 @@ cudaError_t try_stream_t(const QgemvParams& q, int mt, bool dual, cudaStream_t s
       return wide ? launch_stream<BITS, GS, T, 0, UW, 1, false>(q, st) : launch_stream<BITS, GS, T, 0, UB, 1, false>(q, st);
     if (mt == 1)
       return wide ? launch_stream<BITS, GS, T, 1, UW, 1, false>(q, st) : launch_stream<BITS, GS, T, 1, UB, 1, false>(q, st);
-    return launch_stream<BITS, GS, T, 2, UB, 1, false>(q, st);
+    const cudaError_t e2 = launch_stream<BITS, GS, T, 2, UB, 1, false>(q, st);
+    if (e2 != cudaErrorNotSupported || q.n_pairs <= 8 || q.amode != 0) return e2;
+    // sixteen tokens' x rows do not fit beside the ring: two passes of up to
+    // eight tokens each (tokens 8.. read x and write y eight rows further on)
+    QgemvParams lo = q, hi = q;
+    lo.n_pairs = 8;
+    hi.n_pairs = q.n_pairs - 8;
+    hi.a = reinterpret_cast<const T*>(q.a) + 8 * q.K;
+    hi.out = reinterpret_cast<uint8_t*>(q.out) + 8 * q.out_ld * (q.out_dtype == QMM_F32 ? 4 : 2);
+    const cudaError_t e = wide ? launch_stream<BITS, GS, T, 1, UW, 1, false>(lo, st)
+                               : launch_stream<BITS, GS, T, 1, UB, 1, false>(lo, st);
+    if (e != cudaSuccess) return e;
+    return wide ? launch_stream<BITS, GS, T, 1, UW, 1, false>(hi, st) : launch_stream<BITS, GS, T, 1, UB, 1, false>(hi, st);
   } else {
     return cudaErrorNotSupported;
   }
