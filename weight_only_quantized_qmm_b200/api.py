@@ -8,6 +8,7 @@ uint32 words).  All tensors must be CUDA tensors on the current device.
 from __future__ import annotations
 
 import ctypes
+import functools
 from dataclasses import dataclass
 
 import torch
@@ -61,15 +62,17 @@ def _on_device(**named) -> None:
     for what, t in named.items():
         if t is None:
             continue
-        if not t.is_cuda:
+        d = t.get_device()  # -1: host memory
+        if d < 0:
             raise ValueError(f"qmm: {what} must be a CUDA tensor, got one on {t.device}")
         if cur is None:
             cur = torch.cuda.current_device()
-        if t.device.index != cur:
+        if d != cur:
             raise ValueError(f"qmm: {what} is on {t.device}, but the current device is cuda:{cur} "
                              "(the call runs there)")
 
 
+@functools.lru_cache(maxsize=1024)
 def _words(cols: int, bits: int) -> int:
     wpr = qmm_packed_words_per_row(cols, bits)
     if wpr < 0:
@@ -77,6 +80,7 @@ def _words(cols: int, bits: int) -> int:
     return wpr
 
 
+@functools.lru_cache(maxsize=1024)
 def _groups(cols: int, group_size: int) -> int:
     G = qmm_groups_per_row(cols, group_size)
     if G < 0:
@@ -89,8 +93,10 @@ _FLOAT = (torch.float32, torch.float16, torch.bfloat16)
 
 
 def _stream(stream=None) -> int:
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return int(s.cuda_stream)
+    if stream is not None:
+        return int(stream.cuda_stream)
+    # the current stream's handle without building a Stream object
+    return int(torch._C._cuda_getCurrentRawStream(torch.cuda.current_device()))
 
 
 @dataclass
@@ -253,7 +259,7 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
     """y = x . dequant(W)^T (transpose) or x . dequant(W); x [..., K]."""
     lead = x.shape[:-1]
     K = x.shape[-1]
-    x2 = x.reshape(-1, K).contiguous()
+    x2 = x if x.dim() == 2 and x.is_contiguous() else x.reshape(-1, K).contiguous()
     M = x2.shape[0]
     N = qw.rows if transpose else qw.cols
     _need(x2, "x", M * K, _FLOAT)
@@ -269,7 +275,7 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
                                 int(bool(transpose)), _ptr(out), dtype_code(out.dtype),
                                 _stream(stream))
     check("qmm_matmul", rc)
-    return out.reshape(*lead, N)
+    return out if out.dim() == 2 and len(lead) == 1 and out.shape[0] == M else out.reshape(*lead, N)
 
 
 def qmm_matmul_parts(x: torch.Tensor, parts, y_dtype: torch.dtype | None = None, out=None,
