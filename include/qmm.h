@@ -247,8 +247,9 @@ qmm_status qmm_dequantize_dynamic_int8(const int8_t* q, int64_t n, const float* 
  * float x; y_dtype is x_dtype or QMM_F32.  fp32 accumulation, the row dot
  * regrouped as scale * sum x (q + 128) + output_min * sum x (M <= 16 with
  * 16-bit x, K a multiple of 512 and N >= 16: the tensor-core streaming
- * kernel, q + 128 exact in f16 and x exact in f16 after a per-64 power-of-two
- * scaling).  M == 0 or N == 0 is a no-op.
+ * kernel: q + 128 exact in f16, x rounded to f16 after a power-of-two
+ * scaling per 64 values that puts their largest magnitude in [2^14, 2^15)).
+ * M == 0 or N == 0 is a no-op.
  * Errors: DTYPE, INVALID_ARG (M < 0, K <= 0, N < 0), ALIGNMENT (x, q, y
  * 16-byte; params 4-byte), UNSUPPORTED, CUDA. */
 qmm_status qmm_matmul_dynamic_int8(const void* x, qmm_dtype x_dtype, int64_t M, int64_t K,
