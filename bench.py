@@ -831,6 +831,19 @@ def run_profile(args):
                               torch.bfloat16)
         x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
         fn = lambda: api.qmm_matmul(x, qw)  # noqa: E731
+    elif name.startswith("moe_prefill_t"):
+        # the gate projection of a MoE prefill (128 experts, top-8, 768 x 2048),
+        # routed once on the device, activation rows gathered in schedule order
+        T = int(name[len("moe_prefill_t"):])
+        E, dff, dm, k = 128, 768, 2048, 8
+        g = api.ExpertStack.from_qweight(
+            api.qmm_quantize(wl.gen_weight(E * dff, dm, 4600).to(dev), 64, 4, torch.bfloat16), E)
+        ids = wl.gen_moe_ids(T, E, k, 4602 + T).to(dev)
+        a = wl.gen_x(T, dm, 4603 + T).to(dev)
+        ws = api.moe_workspace(T * k, E, dev, n_cols=dm)
+        api.qmm_moe_compute_ids_tpe(ids, E, ws)
+        og = torch.empty(T * k, dff, dtype=torch.bfloat16, device=dev)
+        fn = lambda: api.qmm_moe_gemm_id(a, T, k, 1, ws, g, out=og)  # noqa: E731
     elif name.startswith("moe_down"):
         # the down projection of a one-token MoE step: 8 pairs, K = 768
         case = [d for d in wl.WORKLOADS.moe if d.name == name.replace("moe_down", "moe")][0]
