@@ -831,6 +831,26 @@ def run_profile(args):
                               torch.bfloat16)
         x = wl.gen_x(c.M, c.K, c.seed + 1).to(dev)
         fn = lambda: api.qmm_matmul(x, qw)  # noqa: E731
+    elif name.startswith("transpose0_"):
+        # one token against the [K, N] layout (quantized along N), K = 4096
+        K, N = (int(v) for v in name[len("transpose0_"):].split("x"))
+        qw = api.qmm_quantize(wl.gen_weight(K, N, 7002 + N).to(dev), 64, 4, torch.bfloat16)
+        x = wl.gen_x(1, K, 7001).to(dev)
+        fn = lambda: api.qmm_matmul(x, qw, False)  # noqa: E731
+    elif name.split("_")[0] in ("mxfp4", "mxfp8", "nvfp4"):
+        # one token against a microscaled [N, K] matrix (random codes and scales)
+        mname, shape = name.split("_")
+        N, K = (int(v) for v in shape.split("x"))
+        mode = {"mxfp4": api.QMM_MODE_MXFP4, "mxfp8": api.QMM_MODE_MXFP8, "nvfp4": api.QMM_MODE_NVFP4}[mname]
+        bits, gs = api.MX_PARAMS[mode]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(7004 + mode)
+        packed = torch.randint(-2**31, 2**31 - 1, (N, K * bits // 32), dtype=torch.int32, device=dev, generator=gen)
+        lo, hi = (0x20, 0x50) if mode == api.QMM_MODE_NVFP4 else (110, 130)
+        sc = torch.randint(lo, hi, (N, K // gs), dtype=torch.uint8, device=dev, generator=gen)
+        mq = api.mx_qweight(packed, sc, mode, N, K)
+        x = wl.gen_x(1, K, 7001).to(dev)
+        fn = lambda: api.qmm_matmul(x, mq, True)  # noqa: E731
     elif name.startswith("moe_prefill_t"):
         # the gate projection of a MoE prefill (128 experts, top-8, 768 x 2048),
         # routed once on the device, activation rows gathered in schedule order
