@@ -136,6 +136,27 @@ class QWeight:
                         dtype_code(self.scales.dtype), self.rows, self.cols, self.group_size,
                         self.bits, self.mode)
 
+    def prepared(self):
+        """validate(), then (the CUDA device all the tensors are on, the C
+        struct), or (None, None) when they are not all on one CUDA device.
+        The result is kept while the fields and every tensor's data pointer,
+        element count and dtype stay the same: a replaced, resized or retyped
+        tensor is checked again before the next call."""
+        p, s, b = self.packed, self.scales, self.biases
+        key = (self.rows, self.cols, self.group_size, self.bits, self.mode,
+               p.data_ptr(), p.numel(), p.dtype, s.data_ptr(), s.numel(), s.dtype,
+               None if b is None else (b.data_ptr(), b.numel(), b.dtype))
+        hit = self.__dict__.get("_prep")
+        if hit is not None and hit[0] == key:
+            return hit[1], hit[2]
+        ws = self.validate()
+        devs = {t.get_device() for t in ws.values()}
+        if len(devs) != 1 or min(devs) < 0:
+            return None, None
+        dev, c = devs.pop(), self.c()
+        self.__dict__["_prep"] = (key, dev, c)
+        return dev, c
+
 
 def mx_qweight(packed: torch.Tensor, scales: torch.Tensor, mode: int, rows: int, cols: int) -> QWeight:
     """A microscaled matrix (mxfp4 / mxfp8 / nvfp4): packed [rows,
@@ -257,25 +278,27 @@ def qmm_dequantize(qw: QWeight, out_dtype: torch.dtype = torch.float32, out=None
 def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
                y_dtype: torch.dtype | None = None, out=None, stream=None) -> torch.Tensor:
     """y = x . dequant(W)^T (transpose) or x . dequant(W); x [..., K]."""
-    lead = x.shape[:-1]
+    two_d = x.dim() == 2
     K = x.shape[-1]
-    x2 = x if x.dim() == 2 and x.is_contiguous() else x.reshape(-1, K).contiguous()
+    x2 = x if two_d and x.is_contiguous() else x.reshape(-1, K).contiguous()
     M = x2.shape[0]
     N = qw.rows if transpose else qw.cols
     _need(x2, "x", M * K, _FLOAT)
-    ws = qw.validate()
+    wdev, c = qw.prepared()
     if out is None:
         out = torch.empty(M, N, dtype=y_dtype or x.dtype, device=x2.device)
     _need(out, "out", M * N, _FLOAT)
     if out.numel() != M * N:
         raise ValueError(f"qmm_matmul: out holds {out.numel()} elements, expected {M}x{N}")
-    _on_device(x=x2, out=out, **ws)
-    c = qw.c()
+    _on_device(x=x2, out=out)
+    if c is None or wdev != x2.get_device():
+        _on_device(**qw.validate())  # names the weight tensor that is elsewhere
+        raise ValueError(f"qmm: the weights are not all on {x2.device}")
     rc = _lib.load().qmm_matmul(_ptr(x2), dtype_code(x2.dtype), M, K, ctypes.byref(c),
                                 int(bool(transpose)), _ptr(out), dtype_code(out.dtype),
                                 _stream(stream))
     check("qmm_matmul", rc)
-    return out if out.dim() == 2 and len(lead) == 1 and out.shape[0] == M else out.reshape(*lead, N)
+    return out if two_d and out.dim() == 2 and out.shape[0] == M else out.reshape(*x.shape[:-1], N)
 
 
 def qmm_matmul_parts(x: torch.Tensor, parts, y_dtype: torch.dtype | None = None, out=None,
