@@ -290,13 +290,16 @@ def qmm_matmul(x: torch.Tensor, qw: QWeight, transpose: bool = True,
     _need(out, "out", M * N, _FLOAT)
     if out.numel() != M * N:
         raise ValueError(f"qmm_matmul: out holds {out.numel()} elements, expected {M}x{N}")
-    _on_device(x=x2, out=out)
-    if c is None or wdev != x2.get_device():
-        _on_device(**qw.validate())  # names the weight tensor that is elsewhere
+    dx = x2.get_device()  # -1: host memory
+    cur = torch.cuda.current_device() if dx >= 0 and c is not None else -1
+    if not (dx == out.get_device() == wdev == cur):
+        # the slow checks name the tensor that is elsewhere
+        _on_device(x=x2, out=out)
+        _on_device(**qw.validate())
         raise ValueError(f"qmm: the weights are not all on {x2.device}")
-    rc = _lib.load().qmm_matmul(_ptr(x2), dtype_code(x2.dtype), M, K, ctypes.byref(c),
-                                int(bool(transpose)), _ptr(out), dtype_code(out.dtype),
-                                _stream(stream))
+    st = int(stream.cuda_stream) if stream is not None else int(torch._C._cuda_getCurrentRawStream(cur))
+    rc = _lib.load().qmm_matmul(x2.data_ptr(), dtype_code(x2.dtype), M, K, ctypes.byref(c),
+                                int(bool(transpose)), out.data_ptr(), dtype_code(out.dtype), st)
     check("qmm_matmul", rc)
     return out if two_d and out.dim() == 2 and out.shape[0] == M else out.reshape(*x.shape[:-1], N)
 
