@@ -55,3 +55,27 @@ def test_host_weights_are_refused_after_a_device_call():
     qw.biases = qw.biases.cpu()
     with pytest.raises(ValueError, match="CUDA tensor"):
         api.qmm_matmul(x, qw)
+
+
+def test_changed_expert_stacks_are_checked_again():
+    E, n_rows, n_cols, k = 8, 128, 256, 4
+    q = api.qmm_quantize(wl.gen_weight(E * n_rows, n_cols, 35).to(DEV), 64, 4, torch.bfloat16)
+    gate = api.ExpertStack.from_qweight(q, E)
+    up = api.ExpertStack.from_qweight(
+        api.qmm_quantize(wl.gen_weight(E * n_rows, n_cols, 36).to(DEV), 64, 4, torch.bfloat16), E)
+    a = wl.gen_x(1, n_cols, 37).to(DEV).reshape(-1)
+    ids = torch.tensor([0, 3, 5, 7], dtype=torch.int32, device=DEV)
+    h0 = api.qmm_moe_gemv_id_gate_up_silu(a, ids, k, gate, up, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    scales = up.scales
+    up.scales = scales.reshape(-1)[: scales.numel() - 1].clone()  # one element short
+    with pytest.raises(ValueError, match="up.scales holds"):
+        api.qmm_moe_gemv_id_gate_up_silu(a, ids, k, gate, up)
+    up.scales = scales
+    gate.num_experts = E + 1  # a stated size the tensors do not hold
+    with pytest.raises(ValueError, match="holds"):
+        api.qmm_moe_gemv_id_gate_up_silu(a, ids, k, gate, up)
+    gate.num_experts = E
+    h1 = api.qmm_moe_gemv_id_gate_up_silu(a, ids, k, gate, up, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(h0, h1)

@@ -193,6 +193,25 @@ class ExpertStack:
                             dtype_code(self.scales.dtype), self.num_experts, self.n_rows,
                             self.n_cols, self.group_size, self.bits)
 
+    def prepared(self, role: str = ""):
+        """validate(role), then (the CUDA device all the tensors are on, the C
+        struct), or (None, None) when they are not all on one CUDA device;
+        kept like QWeight.prepared while nothing about the tensors changes."""
+        p, s, b = self.packed, self.scales, self.biases
+        key = (self.num_experts, self.n_rows, self.n_cols, self.group_size, self.bits,
+               p.data_ptr(), p.numel(), p.dtype, s.data_ptr(), s.numel(), s.dtype,
+               b.data_ptr(), b.numel(), b.dtype)
+        hit = self.__dict__.get("_prep")
+        if hit is not None and hit[0] == key:
+            return hit[1], hit[2]
+        ws = self.validate(role)
+        devs = {t.get_device() for t in ws.values()}
+        if len(devs) != 1 or min(devs) < 0:
+            return None, None
+        dev, c = devs.pop(), self.c()
+        self.__dict__["_prep"] = (key, dev, c)
+        return dev, c
+
     @staticmethod
     def from_qweight(q: "QWeight", num_experts: int) -> "ExpertStack":
         assert q.rows % num_experts == 0
@@ -387,15 +406,25 @@ def qmm_matmul_dynamic_int8(x: torch.Tensor, q: torch.Tensor, params: torch.Tens
 
 
 def _moe_checks(a, ids, n_pairs, top_k, outer, inner, stacks, out, n_out_rows, d_status):
+    """Sizes, dtypes and layouts, then one device for everything; returns the
+    stacks' C structs."""
     _need(a, "a", _last_pair_end(n_pairs, top_k, outer, inner, stacks[0].n_cols), _FLOAT)
-    named = {}
-    for role, st in zip(("", "up."), stacks):
-        named.update(st.validate(role))
+    preps = [st.prepared(role) for role, st in zip(("", "up."), stacks)]
     _need(ids, "ids", n_pairs, (torch.int32,))
     _need(out, "out", n_pairs * n_out_rows, _FLOAT)
     if d_status is not None:
         _need(d_status, "d_status", 1, (torch.int32,))
-    _on_device(a=a, ids=ids, out=out, d_status=d_status, **named)
+    da = a.get_device()  # -1: host memory
+    cur = torch.cuda.current_device() if da >= 0 and all(c is not None for _, c in preps) else -1
+    if not (da == cur and ids.get_device() == cur and out.get_device() == cur
+            and (d_status is None or d_status.get_device() == cur) and all(d == cur for d, _ in preps)):
+        # the slow checks name the tensor that is elsewhere
+        named = {}
+        for role, st in zip(("", "up."), stacks):
+            named.update(st.validate(role))
+        _on_device(a=a, ids=ids, out=out, d_status=d_status, **named)
+        raise ValueError(f"qmm: the MoE arguments are not all on {a.device}")
+    return [c for _, c in preps]
 
 
 def qmm_moe_gemv_id(a: torch.Tensor, ids: torch.Tensor, n_selected: int, src1_stride: int,
@@ -403,8 +432,7 @@ def qmm_moe_gemv_id(a: torch.Tensor, ids: torch.Tensor, n_selected: int, src1_st
                     d_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(n_selected, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
-    _moe_checks(a, ids, n_selected, 1, src1_stride, 0, (w,), out, w.n_rows, d_status)
-    c = w.c()
+    (c,) = _moe_checks(a, ids, n_selected, 1, src1_stride, 0, (w,), out, w.n_rows, d_status)
     rc = _lib.load().qmm_moe_gemv_id(_ptr(a), dtype_code(a.dtype), _ptr(ids), n_selected,
                                      src1_stride, ctypes.byref(c), _ptr(out),
                                      dtype_code(out.dtype), _ptr(d_status), _stream(stream))
@@ -419,9 +447,10 @@ def qmm_moe_gemv_id_batched(a: torch.Tensor, ids: torch.Tensor, m: int, top_k: i
     if out is None:
         out = torch.empty(m * top_k, w.n_rows, dtype=out_dtype or a.dtype, device=a.device)
     if top_k > 0:
-        _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (w,), out, w.n_rows,
-                    d_status)
-    c = w.c()
+        (c,) = _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (w,), out, w.n_rows,
+                           d_status)
+    else:
+        c = w.c()
     rc = _lib.load().qmm_moe_gemv_id_batched(_ptr(a), dtype_code(a.dtype), _ptr(ids), m, top_k,
                                              outer_stride, inner_stride, ctypes.byref(c),
                                              _ptr(out), dtype_code(out.dtype), _ptr(d_status),
@@ -437,8 +466,7 @@ def qmm_moe_gemv_id_gate_up_silu(a: torch.Tensor, ids: torch.Tensor, n_selected:
                                  stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(n_selected, gate.n_rows, dtype=out_dtype or a.dtype, device=a.device)
-    _moe_checks(a, ids, n_selected, 1, 0, 0, (gate, up), out, gate.n_rows, d_status)
-    cg, cu = gate.c(), up.c()
+    cg, cu = _moe_checks(a, ids, n_selected, 1, 0, 0, (gate, up), out, gate.n_rows, d_status)
     rc = _lib.load().qmm_moe_gemv_id_gate_up_silu(_ptr(a), dtype_code(a.dtype), _ptr(ids),
                                                   n_selected, ctypes.byref(cg), ctypes.byref(cu),
                                                   _ptr(out), dtype_code(out.dtype),
@@ -456,9 +484,10 @@ def qmm_moe_gemv_id_gate_up_silu_batched(a: torch.Tensor, ids: torch.Tensor, m: 
     if out is None:
         out = torch.empty(m * top_k, gate.n_rows, dtype=out_dtype or a.dtype, device=a.device)
     if top_k > 0:
-        _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (gate, up), out,
-                    gate.n_rows, d_status)
-    cg, cu = gate.c(), up.c()
+        cg, cu = _moe_checks(a, ids, m * top_k, top_k, outer_stride, inner_stride, (gate, up), out,
+                             gate.n_rows, d_status)
+    else:
+        cg, cu = gate.c(), up.c()
     rc = _lib.load().qmm_moe_gemv_id_gate_up_silu_batched(
         _ptr(a), dtype_code(a.dtype), _ptr(ids), m, top_k, outer_stride, inner_stride,
         ctypes.byref(cg), ctypes.byref(cu), _ptr(out), dtype_code(out.dtype), _ptr(d_status),
