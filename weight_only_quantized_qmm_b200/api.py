@@ -337,18 +337,30 @@ def qmm_matmul_parts(x: torch.Tensor, parts, y_dtype: torch.dtype | None = None,
     M = x2.shape[0]
     Ntot = sum(p.rows for p in parts)
     _need(x2, "x", M * K, _FLOAT)
-    named = {}
+    preps = []
     for i, p in enumerate(parts):
-        named.update({f"part{i}.{k}": v for k, v in p.validate().items()})
+        try:
+            preps.append(p.prepared())
+        except ValueError as e:
+            raise ValueError(f"qmm_matmul_parts: part {i}: {e}") from None
     if out is None:
         out = torch.empty(M, Ntot, dtype=y_dtype or x.dtype, device=x2.device)
     _need(out, "out", M * Ntot, _FLOAT)
     if out.numel() != M * Ntot:
         raise ValueError(f"qmm_matmul_parts: out holds {out.numel()} elements, expected {M}x{Ntot}")
-    _on_device(x=x2, out=out, **named)
-    arr = (QWeightC * len(parts))(*[p.c() for p in parts])
-    rc = _lib.load().qmm_matmul_parts(_ptr(x2), dtype_code(x2.dtype), M, K, arr, len(parts), _ptr(out),
-                                      dtype_code(out.dtype), _stream(stream))
+    dx = x2.get_device()  # -1: host memory
+    cur = torch.cuda.current_device() if dx >= 0 and all(c is not None for _, c in preps) else -1
+    if not (dx == out.get_device() == cur and all(d == cur for d, _ in preps)):
+        # the slow checks name the tensor that is elsewhere
+        named = {}
+        for i, p in enumerate(parts):
+            named.update({f"part{i}.{k}": v for k, v in p.validate().items()})
+        _on_device(x=x2, out=out, **named)
+        raise ValueError(f"qmm_matmul_parts: the parts are not all on {x2.device}")
+    arr = (QWeightC * len(parts))(*[c for _, c in preps])
+    st = int(stream.cuda_stream) if stream is not None else int(torch._C._cuda_getCurrentRawStream(cur))
+    rc = _lib.load().qmm_matmul_parts(x2.data_ptr(), dtype_code(x2.dtype), M, K, arr, len(parts),
+                                      out.data_ptr(), dtype_code(out.dtype), st)
     check("qmm_matmul_parts", rc)
     return out.reshape(*lead, Ntot)
 
